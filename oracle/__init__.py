@@ -1,0 +1,135 @@
+"""CPU fp64 oracle for multi-head causal self-attention -- TEST INFRASTRUCTURE.
+
+Only the tests, the smoke check in ``__graft_entry__`` and the CPU-baseline
+leg of ``bench.py`` may import this package.  The CUDA library never touches
+it, and it imports nothing from the CUDA package: the two share only the
+seeded input generators, which hold none of the method's arithmetic.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, double precision,
+OpenMP over the independent (batch, head) pairs).  This module compiles it
+with gcc on first use and marshals numpy float64 arrays through ctypes.
+
+What is computed (see the C file header for the passages it follows):
+  forward:   S = scale * Q K^T, S_ij = -inf for j > i (and, with a document
+             mask, for j < doc_start[i]), P = softmax_rows(S), O = P V,
+             LSE_i = log sum_j exp(S_ij)  (natural log, scaled scores)
+  backward:  dV = P^T dO, dP = dO V^T, dS_i = (diag(p_i) - p_i p_i^T) dP_i
+             with the Jacobian formed explicitly, dQ = scale dS K,
+             dK = scale dS^T Q.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB = os.path.join(_HERE, "_attn_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile attn_oracle.c into _attn_oracle.so (gcc, -O2, OpenMP).  Returns the path."""
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        lib.oracle_attn_fwd.argtypes = [dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_double, ip, dp, dp, dp]
+        lib.oracle_attn_fwd.restype = ctypes.c_int
+        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_double, ip, dp, dp, dp]
+        lib.oracle_attn_bwd.restype = ctypes.c_int
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    """Exact upcast to a C-contiguous float64 array (bf16/fp32 values are exact in fp64)."""
+    if hasattr(x, "detach"):  # torch tensor (CPU)
+        import torch
+        x = x.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: Optional[np.ndarray], ctype):
+    if a is None:
+        return ctypes.cast(None, ctypes.POINTER(ctype))
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _doc(doc_start, B, T) -> Optional[np.ndarray]:
+    if doc_start is None:
+        return None
+    if hasattr(doc_start, "detach"):
+        doc_start = doc_start.detach().cpu().numpy()
+    a = np.ascontiguousarray(np.asarray(doc_start, dtype=np.int32))
+    if a.shape != (B, T):
+        raise ValueError(f"doc_start must be [B,T]=({B},{T}), got {a.shape}")
+    return a
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def attention_forward(q, k, v, scale: float, doc_start=None, return_probs: bool = False):
+    """O [B,H,T,d], LSE [B,H,T] (float64); with return_probs also P [B,H,T,T]."""
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, T, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B,H,T,d] shape")
+    doc = _doc(doc_start, B, T)
+    o = np.empty_like(q)
+    lse = np.empty((B, H, T), dtype=np.float64)
+    probs = np.empty((B, H, T, T), dtype=np.float64) if return_probs else None
+    rc = lib.oracle_attn_fwd(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
+                             _ptr(v, ctypes.c_double), B, H, T, d, float(scale),
+                             _ptr(doc, ctypes.c_int32), _ptr(o, ctypes.c_double),
+                             _ptr(lse, ctypes.c_double), _ptr(probs, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd failed with code {rc}")
+    return (o, lse, probs) if return_probs else (o, lse)
+
+
+def attention_backward(q, k, v, dout, scale: float, doc_start=None) -> Tuple[np.ndarray, ...]:
+    """dQ, dK, dV [B,H,T,d] float64, by the explicit softmax Jacobian."""
+    lib = _load()
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, T, d = q.shape
+    for t in (k, v, dout):
+        if t.shape != q.shape:
+            raise ValueError("q, k, v, dout must share one [B,H,T,d] shape")
+    doc = _doc(doc_start, B, T)
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    rc = lib.oracle_attn_bwd(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
+                             _ptr(v, ctypes.c_double), _ptr(dout, ctypes.c_double),
+                             B, H, T, d, float(scale), _ptr(doc, ctypes.c_int32),
+                             _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+                             _ptr(dv, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_bwd failed with code {rc}")
+    return dq, dk, dv

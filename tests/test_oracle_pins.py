@@ -1,0 +1,273 @@
+"""Pins for the CPU fp64 oracle: checks against facts that do not come from the
+oracle itself -- closed forms derived by hand, invariants of the definition,
+central finite differences, and an independent library routine (torch's CPU
+scaled_dot_product_attention in float64 with autograd).
+
+The definition being pinned: "Stanford CS336 walkthrough" (lmnt.cn), section
+5.1 model.py CausalSelfAttention.forward (scores q k^T / sqrt(d), upper
+triangle -inf, row softmax, att @ v) and section 3.3 (masked weights are zero
+after the softmax); the mask keeps the diagonal (torch.tril(ones) in
+"Train Your Own LLM from Scratch", section 1).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from causal_self_attention_mha_b200 import inputs
+
+
+def rnd(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def fwd(q, k, v, scale, doc=None, probs=False):
+    return oracle.attention_forward(q, k, v, scale, doc, return_probs=probs)
+
+
+def bwd(q, k, v, do, scale, doc=None):
+    return oracle.attention_backward(q, k, v, do, scale, doc)
+
+
+# ---------------------------------------------------------------- closed forms
+
+def test_single_token_closed_form():
+    """T = 1: softmax over one key is 1, so O = v_0, LSE = scale <q0,k0>, dQ = dK = 0, dV = dO."""
+    B, H, T, d = 2, 3, 1, 8
+    q, k, v, do = (rnd((B, H, T, d), s) for s in range(4))
+    scale = 0.37
+    o, lse = fwd(q, k, v, scale)
+    np.testing.assert_array_equal(o, v)
+    np.testing.assert_allclose(lse, scale * np.einsum("bhtc,bhtc->bht", q, k), rtol=0, atol=1e-14)
+    dq, dk, dv = bwd(q, k, v, do, scale)
+    assert np.all(dq == 0) and np.all(dk == 0)
+    np.testing.assert_array_equal(dv, do)
+
+
+def test_first_row_sees_only_itself():
+    """Row 0 has a single visible key (the diagonal): O_0 = v_0 and LSE_0 = scale <q0,k0>."""
+    B, H, T, d = 1, 2, 9, 4
+    q, k, v = (rnd((B, H, T, d), s) for s in range(3))
+    o, lse = fwd(q, k, v, 0.5)
+    np.testing.assert_array_equal(o[:, :, 0], v[:, :, 0])
+    np.testing.assert_allclose(lse[:, :, 0], 0.5 * np.sum(q[:, :, 0] * k[:, :, 0], -1), atol=1e-14)
+
+
+def test_two_token_closed_form():
+    """T = 2 by hand.  Row 1 mixes v0, v1 with p11 = sigmoid(scale <q1, k1 - k0>):
+         O_1   = v0 + p11 (v1 - v0),  LSE_1 = log(e^{s10} + e^{s11})
+         g     = p10 p11 <dO_1, v1 - v0>
+         dQ_1  = scale g (k1 - k0),   dQ_0 = 0
+         dK_0  = -scale g q1,         dK_1 = +scale g q1
+         dV_0  = dO_0 + p10 dO_1,     dV_1 = p11 dO_1
+    """
+    d, scale = 5, 0.8
+    q, k, v, do = (rnd((1, 1, 2, d), 10 + s) for s in range(4))
+    q0, q1 = q[0, 0]
+    k0, k1 = k[0, 0]
+    v0, v1 = v[0, 0]
+    do0, do1 = do[0, 0]
+    s10, s11 = scale * q1 @ k0, scale * q1 @ k1
+    p11 = 1.0 / (1.0 + math.exp(-(s11 - s10)))
+    p10 = 1.0 - p11
+    o, lse = fwd(q, k, v, scale)
+    np.testing.assert_allclose(o[0, 0, 1], v0 + p11 * (v1 - v0), atol=1e-14)
+    np.testing.assert_allclose(lse[0, 0, 1], math.log(math.exp(s10) + math.exp(s11)), atol=1e-14)
+    g = p10 * p11 * (do1 @ (v1 - v0))
+    dq, dk, dv = bwd(q, k, v, do, scale)
+    np.testing.assert_allclose(dq[0, 0, 0], 0.0, atol=1e-15)
+    np.testing.assert_allclose(dq[0, 0, 1], scale * g * (k1 - k0), atol=1e-14)
+    np.testing.assert_allclose(dk[0, 0, 0], -scale * g * q1, atol=1e-14)
+    np.testing.assert_allclose(dk[0, 0, 1], scale * g * q1, atol=1e-14)
+    np.testing.assert_allclose(dv[0, 0, 0], do0 + p10 * do1, atol=1e-14)
+    np.testing.assert_allclose(dv[0, 0, 1], p11 * do1, atol=1e-14)
+
+
+def test_uniform_values_give_that_value():
+    """All v_j equal to u: every row is a convex combination of copies of u, so O_i = u;
+    dP_ij = <dO_i, u> is constant along the row, so dS = 0 and dQ = dK = 0."""
+    B, H, T, d = 2, 2, 33, 6
+    q, k, do = (rnd((B, H, T, d), s) for s in range(3))
+    u = rnd((d,), 7)
+    v = np.broadcast_to(u, (B, H, T, d)).copy()
+    o, _ = fwd(q, k, v, 0.4)
+    np.testing.assert_allclose(o, v, atol=1e-13)
+    dq, dk, dv = bwd(q, k, v, do, 0.4)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-13)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-13)
+
+
+# ------------------------------------------------------------------ invariants
+
+def test_probability_rows():
+    """Rows of P sum to 1, the strict upper triangle is exactly 0, the diagonal is positive."""
+    B, H, T, d = 2, 2, 40, 8
+    q, k, v = (rnd((B, H, T, d), s) for s in range(3))
+    _, _, p = fwd(q, k, v, 1 / math.sqrt(d), probs=True)
+    np.testing.assert_allclose(p.sum(-1), 1.0, atol=1e-12)
+    iu = np.triu_indices(T, 1)
+    assert np.all(p[:, :, iu[0], iu[1]] == 0.0)
+    assert np.all(np.diagonal(p, axis1=2, axis2=3) > 0)
+
+
+def test_probability_rows_with_documents():
+    """With a document mask, P_ij = 0 outside [doc_start(i), i] and rows still sum to 1."""
+    B, H, T, d = 2, 1, 50, 4
+    q, k, v = (rnd((B, H, T, d), s) for s in range(3))
+    doc = inputs.random_doc_start(B, T, 3, 3, 17).numpy()
+    _, _, p = fwd(q, k, v, 0.6, doc, probs=True)
+    np.testing.assert_allclose(p.sum(-1), 1.0, atol=1e-12)
+    for b in range(B):
+        for i in range(T):
+            outside = np.ones(T, bool)
+            outside[doc[b, i]:i + 1] = False
+            assert np.all(p[b, :, i, outside] == 0.0)
+
+
+@pytest.mark.parametrize("t", [0, 5, 17])
+def test_future_perturbation_leaves_past_unchanged(t):
+    """Changing q, k, v at positions > t leaves O, LSE at positions <= t bit-identical;
+    with dO = 0 after t, the gradients at positions <= t are bit-identical too."""
+    B, H, T, d = 1, 2, 24, 4
+    q, k, v, do = (rnd((B, H, T, d), 20 + s) for s in range(4))
+    do[:, :, t + 1:] = 0.0
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for a, s in ((q2, 1), (k2, 2), (v2, 3)):
+        a[:, :, t + 1:] += rnd(a[:, :, t + 1:].shape, 100 + s)
+    o1, l1 = fwd(q, k, v, 0.5)
+    o2, l2 = fwd(q2, k2, v2, 0.5)
+    np.testing.assert_array_equal(o1[:, :, :t + 1], o2[:, :, :t + 1])
+    np.testing.assert_array_equal(l1[:, :, :t + 1], l2[:, :, :t + 1])
+    assert not np.allclose(o1[:, :, t + 1:], o2[:, :, t + 1:])
+    g1 = bwd(q, k, v, do, 0.5)
+    g2 = bwd(q2, k2, v2, do, 0.5)
+    for a, b in zip(g1, g2):
+        np.testing.assert_array_equal(a[:, :, :t + 1], b[:, :, :t + 1])
+
+
+def test_gradient_sums():
+    """A common shift of every key adds a per-row constant to the scores, which the softmax
+    ignores: sum_j dK_j = 0 per head (per document with a mask).  Rows of P sum to 1:
+    sum_j dV_j = sum_i dO_i."""
+    B, H, T, d = 2, 2, 37, 5
+    q, k, v, do = (rnd((B, H, T, d), 30 + s) for s in range(4))
+    dq, dk, dv = bwd(q, k, v, do, 0.45)
+    np.testing.assert_allclose(dk.sum(2), 0.0, atol=1e-12)
+    np.testing.assert_allclose(dv.sum(2), do.sum(2), atol=1e-12)
+    doc = inputs.random_doc_start(B, T, 5, 4, 15).numpy()
+    dq, dk, dv = bwd(q, k, v, do, 0.45, doc)
+    for b in range(B):
+        for s in np.unique(doc[b]):
+            e = s + int(np.sum(doc[b] == s))
+            np.testing.assert_allclose(dk[b, :, s:e].sum(1), 0.0, atol=1e-12)
+            np.testing.assert_allclose(dv[b, :, s:e].sum(1), do[b, :, s:e].sum(1), atol=1e-12)
+
+
+def test_linear_in_values():
+    """V -> a V scales O, dQ, dK by a and leaves LSE and dV unchanged."""
+    B, H, T, d = 1, 2, 19, 3
+    q, k, v, do = (rnd((B, H, T, d), 40 + s) for s in range(4))
+    a = -2.5
+    o1, l1 = fwd(q, k, v, 0.7)
+    o2, l2 = fwd(q, k, a * v, 0.7)
+    np.testing.assert_allclose(o2, a * o1, atol=1e-13)
+    np.testing.assert_array_equal(l1, l2)
+    g1 = bwd(q, k, v, do, 0.7)
+    g2 = bwd(q, k, a * v, do, 0.7)
+    np.testing.assert_allclose(g2[0], a * g1[0], atol=1e-12)
+    np.testing.assert_allclose(g2[1], a * g1[1], atol=1e-12)
+    np.testing.assert_allclose(g2[2], g1[2], atol=1e-13)
+
+
+def test_documents_equal_independent_slices():
+    """Document-causal attention on a packed row equals plain causal attention run on each
+    document slice on its own (forward and backward)."""
+    B, H, T, d = 2, 2, 45, 4
+    q, k, v, do = (rnd((B, H, T, d), 50 + s) for s in range(4))
+    doc = inputs.random_doc_start(B, T, 9, 5, 14).numpy()
+    o, lse = fwd(q, k, v, 0.55, doc)
+    dq, dk, dv = bwd(q, k, v, do, 0.55, doc)
+    for b in range(B):
+        for s in np.unique(doc[b]):
+            e = s + int(np.sum(doc[b] == s))
+            sl = (slice(b, b + 1), slice(None), slice(s, e))
+            oo, ll = fwd(q[sl], k[sl], v[sl], 0.55)
+            np.testing.assert_allclose(o[sl], oo, atol=1e-14)
+            np.testing.assert_allclose(lse[b:b + 1, :, s:e], ll, atol=1e-14)
+            gq, gk, gv = bwd(q[sl], k[sl], v[sl], do[sl], 0.55)
+            np.testing.assert_allclose(dq[sl], gq, atol=1e-13)
+            np.testing.assert_allclose(dk[sl], gk, atol=1e-13)
+            np.testing.assert_allclose(dv[sl], gv, atol=1e-13)
+
+
+# --------------------------------------------------------- numerical derivative
+
+@pytest.mark.parametrize("T,d", [(1, 2), (2, 2), (3, 4), (5, 2), (8, 4)])
+@pytest.mark.parametrize("with_doc", [False, True])
+def test_central_finite_differences(T, d, with_doc):
+    """dQ, dK, dV against central differences of L = sum(dO * O), h = 1e-6, in fp64."""
+    B, H = 1, 2
+    q, k, v, do = (rnd((B, H, T, d), 60 + 7 * T + d + s) for s in range(4))
+    scale = 1 / math.sqrt(d)
+    doc = inputs.random_doc_start(B, T, T, 1, 3).numpy() if with_doc else None
+    grads = bwd(q, k, v, do, scale, doc)
+    h = 1e-6
+    for which, g in enumerate(grads):
+        num = np.zeros_like(g)
+        for idx in np.ndindex(*g.shape):
+            args = [q, k, v]
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            lp = np.sum(do * fwd(*plus, scale, doc)[0])
+            lm = np.sum(do * fwd(*minus, scale, doc)[0])
+            num[idx] = (lp - lm) / (2 * h)
+        err = np.linalg.norm(num - g) / max(np.linalg.norm(num), 1e-30)
+        if np.linalg.norm(num) < 1e-12:
+            assert np.max(np.abs(g)) < 1e-9
+        else:
+            assert err <= 1e-6, (which, err)
+
+
+# ------------------------------------------------ independent library routine
+
+def torch_reference(q, k, v, do, scale, doc=None):
+    """torch CPU float64 SDPA + autograd: an implementation that shares nothing with the oracle."""
+    tq, tk, tv = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+    T = q.shape[2]
+    if doc is None:
+        o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=scale)
+    else:
+        i = torch.arange(T).view(T, 1)
+        j = torch.arange(T).view(1, T)
+        ds = torch.tensor(doc, dtype=torch.int64)  # [B,T]
+        mask = (j <= i) & (j >= ds.view(-1, T, 1))  # [B,T,T]
+        o = torch.nn.functional.scaled_dot_product_attention(
+            tq, tk, tv, attn_mask=mask.unsqueeze(1), scale=scale)
+    # LSE by the textbook formula on the same masked scores
+    s = torch.einsum("bhic,bhjc->bhij", tq.detach(), tk.detach()) * scale
+    i = torch.arange(T).view(T, 1)
+    j = torch.arange(T).view(1, T)
+    vis = (j <= i) if doc is None else ((j <= i) & (j >= torch.tensor(doc, dtype=torch.int64).view(-1, 1, T, 1)))
+    lse = torch.logsumexp(s.masked_fill(~vis, float("-inf")), dim=-1)
+    o.backward(torch.tensor(do, dtype=torch.float64))
+    return (o.detach().numpy(), lse.numpy(), tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy())
+
+
+@pytest.mark.parametrize("B,H,T,d,with_doc", [
+    (1, 4, 64, 32, False),     # the tiny GPT head shape
+    (1, 2, 130, 64, False),    # ragged length
+    (2, 1, 200, 128, True),    # documents, d = 128
+])
+def test_against_torch_sdpa_fp64(B, H, T, d, with_doc):
+    q, k, v, do = (t.to(torch.float64).numpy() for t in inputs.make_qkvdo(B, H, T, d, 77))
+    scale = inputs.fp32_scale(d)
+    doc = inputs.random_doc_start(B, T, 8, 20, 90).numpy() if with_doc else None
+    o, lse = fwd(q, k, v, scale, doc)
+    dq, dk, dv = bwd(q, k, v, do, scale, doc)
+    ro, rl, rq, rk, rv = torch_reference(q, k, v, do, scale, doc)
+    for a, b in ((o, ro), (lse, rl), (dq, rq), (dk, rk), (dv, rv)):
+        assert np.max(np.abs(a - b)) <= 1e-10
