@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark: causal attention forward + backward, bf16, TFLOP/s on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+forward (O, LSE), then backward (delta, dK/dV, dQ), all through the C ABI of
+libcausalattn on one CUDA stream.  The default workload is B=4 H=16 T=2048
+d=128 with the full causal mask.
+
+FLOP convention (algorithmic, visible (query, key) pairs only, diagonal
+included; pairs = B*H*T*(T+1)/2 for the causal mask):
+  forward 4*d*pairs, backward 10*d*pairs, step 14*d*pairs.
+
+Timing: W untimed warm-up steps, then exactly K steps between CUDA events on
+the launching stream, bracketed by barrier + synchronize; the inputs (Q, K, V,
+dO = 134 MB, plus O = 34 MB) exceed the 126 MB L2, so L2 is not flushed.
+Multi-GPU (torchrun): independent replicas, one per GPU, no data-path
+collective; value = all ranks' FLOPs / max over ranks of the timed region.
+
+`--impl reference` times the CPU fp64 oracle (the only other program on the
+pages' path) on the host cores, on bounded per-step samples of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "causal attention fwd+bwd TFLOP/s (bf16) and % of B200 dense peak, 1 GPU"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.md")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wide_d128")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"],
+                "hbm": p["hbm_gbs"], "source": "measured"}
+    return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_self_attention_mha_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    text = open(PROFILE_TRAFFIC).read()
+    m = re.search(r"source_hash:\s*(\w+)", text)
+    if not m or m.group(1) != kernel_source_hash():
+        return None
+    m = re.search(rf"^\|\s*{re.escape(kernel)}\s*\|\s*{re.escape(workload)}\s*\|\s*([0-9.eE+]+)\s*\|",
+                  text, re.M)
+    return float(m.group(1)) if m else None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms in the background."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 - 1 <= r[0] <= t1 + 1] or rows
+        if not inside:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in inside for n, v in zip(names, r[3][1:]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_sample(w, n_heads: int, rows: int = 0, data=None):
+    """Oracle fwd+bwd on the first n_heads (b, h) pairs of the workload, restricted to the first
+    `rows` query positions (0 = all T).  Causality makes a row prefix a self-contained
+    problem: query rows < R only see keys < R.  Returns (seconds, algorithmic flops)."""
+    import numpy as np
+    import torch
+    import oracle
+    from causal_self_attention_mha_b200 import inputs
+    q, k, v, do, doc = data if data is not None else inputs.make_workload(w)
+    R = rows or w.T
+    def pick(t):
+        return t.reshape(w.B * w.H, w.T, w.d)[:n_heads, :R].reshape(n_heads, 1, R, w.d).to(torch.float64).numpy()
+    qs, ks, vs, dos = (pick(t) for t in (q, k, v, do))
+    docs = None
+    pairs = 0
+    if doc is not None:
+        docs = np.stack([doc[i // w.H, :R].numpy() for i in range(n_heads)]).astype(np.int32)
+        for i in range(n_heads):
+            pairs += inputs.visible_pairs(1, 1, R, torch.from_numpy(docs[i:i + 1]))
+    else:
+        pairs = n_heads * R * (R + 1) // 2
+    t0 = time.perf_counter()
+    oracle.attention_forward(qs, ks, vs, w.scale, docs)
+    oracle.attention_backward(qs, ks, vs, dos, w.scale, docs)
+    dt = time.perf_counter() - t0
+    return dt, 14.0 * w.d * pairs
+
+
+def run_reference(args, w, rank: int):
+    """The oracle, as it stands, on the host cores: rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    from causal_self_attention_mha_b200 import inputs
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    n_heads = min(w.B * w.H, cores)
+    data = inputs.make_workload(w)
+    # size each step so that warm-up + timed steps stay within ~150 s of CPU time
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    R = min(w.T, 256)
+    dt, _ = oracle_sample(w, n_heads, R, data)
+    while R < w.T and dt * (min(w.T, 2 * R) / R) ** 3 < budget:
+        R = min(w.T, 2 * R)
+        dt, _ = oracle_sample(w, n_heads, R, data)
+    for _ in range(args.warmup):
+        oracle_sample(w, n_heads, R, data)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, flops = oracle_sample(w, n_heads, R, data)
+        times.append(dt)
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    sample = (f"fwd+bwd of {n_heads} of {w.B * w.H} heads, query/key prefix {R} of T={w.T} "
+              f"(d={w.d}) per step; CPU {cpu_model()}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic: seeded N(0,1) bf16 Q,K,V,dO",
+        "config": workload_config(w, "single host process (OpenMP over heads)"),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, parallelism):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} d={w.d}, "
+                        f"{'document-causal' if w.doc_packed else 'causal'} mask",
+            "B": w.B, "H": w.H, "T": w.T, "d": w.d, "seq_len": w.T,
+            "mask": "document-causal" if w.doc_packed else "causal",
+            "parallelism": parallelism,
+            "l2": "not flushed: inputs Q,K,V,dO (+O) exceed the 126 MB L2"}
+
+
+def main():
+    args = parse()
+    import torch
+    from causal_self_attention_mha_b200 import inputs
+
+    w = inputs.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    import torch.distributed as dist
+    from causal_self_attention_mha_b200 import abi
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    q, k, v, do, doc = inputs.make_workload(w)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    docd = doc.to(dev) if doc is not None else None
+    B, H, T, d = w.B, w.H, w.T, w.d
+    o = torch.empty_like(qd)
+    lse = torch.empty(B, H, T, device=dev, dtype=torch.float32)
+    delta = torch.empty_like(lse)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(qd), torch.empty_like(qd)
+    pairs = inputs.visible_pairs(B, H, T, doc)
+    step_flops = 14.0 * d * pairs
+    stream = torch.cuda.Stream(device=dev)
+    kernels = ["attn_fwd", "attn_bwd_delta", "attn_bwd_dkdv", "attn_bwd_dq"]
+    n_ev = 5
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        abi.gpt_attn_fwd(qd, kd, vd, o, lse, w.scale, docd, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        abi.gpt_attn_bwd_preprocess(o, dod, delta, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        abi.gpt_attn_bwd_dkdv(qd, kd, vd, dod, lse, delta, dk, dv, w.scale, docd, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        abi.gpt_attn_bwd_dq(qd, kd, vd, dod, lse, delta, dq, w.scale, docd, stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    torch.cuda.synchronize(dev)
+    if abi.gpt_attn_device_status(clear=True) != 0:
+        raise RuntimeError("a kernel reported a wait timeout during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    time.sleep(0.5)  # let the sampler start before the timed region
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(events[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    elapsed_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    per_kernel_ms = [0.0] * len(kernels)
+    for ev in events:
+        for j in range(len(kernels)):
+            per_kernel_ms[j] += ev[j].elapsed_time(ev[j + 1])
+    per_kernel_ms = [x / args.steps for x in per_kernel_ms]
+    status = abi.gpt_attn_device_status(clear=True)
+
+    # ---------------------------------------------- end to end, host buffers
+    step_host = abi.HostStep(B, H, T, d, dev)
+    step_host.set_doc_offsets(doc)
+    pin = lambda t: t.pin_memory()
+    qh, kh, vh, doh = (pin(t) for t in (q, k, v, do))
+    outs = {n: torch.empty(B, H, T, d, dtype=torch.bfloat16).pin_memory() for n in ("o", "dq", "dk", "dv")}
+    outs["lse"] = torch.empty(B, H, T, dtype=torch.float32).pin_memory()
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            step_host.run(qh, kh, vh, doh, outs, w.scale, stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.e2e_steps):
+        step_host.run(qh, kh, vh, doh, outs, w.scale, stream)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e_start.elapsed_time(e_end) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    barrier()
+
+    if rank == 0:
+        pk = peaks()
+        ms_per_step = elapsed_ms / args.steps
+        value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+        fwd_flops, bwd_flops = 4.0 * d * pairs, 10.0 * d * pairs
+        fwd_ms = per_kernel_ms[0]
+        bwd_ms = sum(per_kernel_ms[1:])
+        # roofline of the dominant kernel (largest share of the step)
+        kflops = {"attn_fwd": 4.0 * d * pairs, "attn_bwd_dkdv": 8.0 * d * pairs,
+                  "attn_bwd_dq": 6.0 * d * pairs}
+        kbytes = {"attn_bwd_delta": 2.0 * B * H * T * d * 2 + 4.0 * B * H * T}
+        j = max(range(len(kernels)), key=lambda i: per_kernel_ms[i])
+        name = kernels[j]
+        timed_s = elapsed_ms * 1e-3
+        peak_kind = "burst" if timed_s < 2.0 else "sustained"
+        if name in kflops:
+            peak = pk["bf16"] if peak_kind == "burst" else pk["bf16_sustained"]
+            achieved = kflops[name] / (per_kernel_ms[j] * 1e-3) / 1e12
+            roof = {"kernel": name, "bound": "tensor", "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak,
+                    "peak_source": f"{pk['source']} ({peak_kind} bf16 GEMM)"}
+        else:
+            achieved = kbytes[name] / (per_kernel_ms[j] * 1e-3) / 1e9
+            roof = {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": pk["hbm"],
+                    "unit": "GB/s", "frac": achieved / pk["hbm"], "peak_source": pk["source"]}
+        roof["traffic"] = recorded_traffic(name, w.name)
+        peak_step = pk["bf16"] if peak_kind == "burst" else pk["bf16_sustained"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) bf16 Q,K,V,dO",
+            "config": workload_config(w, f"replicas x{world}" if world > 1 else "single GPU"),
+            "pct_of_peak": 100.0 * (value / world) / peak_step,
+            "peak_tflops": peak_step,
+            "fwd_tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12,
+            "bwd_tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,
+            "kernel_ms": dict(zip(kernels, per_kernel_ms)),
+            "roofline": roof,
+            "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": step_host.h2d_bytes(),
+                    "d2h_bytes_per_step": step_host.d2h_bytes(), "ms_per_step": e2e_ms},
+            "gpu_launches": len(kernels) * args.steps,
+            "clocks": clocks,
+            "device_status": status,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            cores = len(os.sched_getaffinity(0))
+            oracle.set_threads(cores)
+            n_heads = min(B * H, cores)
+            dt, fl = oracle_sample(w, n_heads)
+            line["cpu_baseline"] = {
+                "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "seconds": dt,
+                "sample": f"fwd+bwd of {n_heads} of {B * H} heads (full T={T}, d={d}), "
+                          f"CPU {cpu_model()}"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,297 @@
+"""ctypes binding of libcausalattn (include/causalattn.h).
+
+Argument marshalling only: every function here checks that the torch tensors
+it is given have the layout the C ABI documents (contiguous bf16 [B,H,T,d] on
+the current CUDA device, fp32/int32 side arrays), passes their device
+pointers, sizes and the current CUDA stream through the C ABI, and turns a
+non-zero status into an exception.  All arithmetic happens in the library's
+CUDA kernels.  There is no CPU fallback: if the library is missing or cannot
+be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcausalattn.so")
+
+GPT_ATTN_OK = 0
+GPT_ATTN_ERR_NULL_PTR = 1
+GPT_ATTN_ERR_BAD_SHAPE = 2
+GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM = 3
+GPT_ATTN_ERR_MISALIGNED = 4
+GPT_ATTN_ERR_BAD_DOC_OFFSETS = 5
+GPT_ATTN_ERR_NO_DEVICE = 6
+GPT_ATTN_ERR_UNSUPPORTED_ARCH = 7
+GPT_ATTN_ERR_LAUNCH = 8
+GPT_ATTN_ERR_DEVICE_TIMEOUT = 9
+GPT_ATTN_ERR_NOT_IMPLEMENTED = 10
+GPT_ATTN_ERR_BAD_SCALE = 11
+GPT_ATTN_ERR_TOO_LARGE = 12
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+# name -> (argtypes, restype); mirrors include/causalattn.h
+SIGNATURES = {
+    "gpt_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
+    "gpt_attn_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
+    "gpt_attn_bwd_preprocess": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
+    "gpt_attn_bwd_dkdv": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
+    "gpt_attn_bwd_dq": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
+    "gpt_attn_check_doc_offsets": ([_vp, _i, _i, _vp], _i),
+    "gpt_attn_device_status": ([ctypes.POINTER(ctypes.c_uint), _i], _i),
+    "gpt_attn_selftest_wait_timeout": ([ctypes.c_uint64, _vp], _i),
+    "gpt_attn_strerror": ([_i], ctypes.c_char_p),
+    "gpt_attn_version": ([], _i),
+}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: status {status} ({strerror(status)})")
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libcausalattn.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None or path is not None:
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(
+                f"libcausalattn.so not found at {p}; build it with "
+                "`python -m causal_self_attention_mha_b200.build`")
+        lib = ctypes.CDLL(p)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        if path is not None:
+            return lib
+        _lib = lib
+    return _lib
+
+
+def strerror(status: int) -> str:
+    try:
+        return load().gpt_attn_strerror(int(status)).decode()
+    except Exception:  # the library itself may be what failed to load
+        return "unknown"
+
+
+def version() -> int:
+    return int(load().gpt_attn_version())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(fn: str, status: int) -> None:
+    if status != GPT_ATTN_OK:
+        raise AttnError(fn, status)
+
+
+def _bhtd(name: str, t: torch.Tensor, ref: Optional[torch.Tensor] = None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B,H,T,d] tensor")
+    if ref is not None and (t.shape != ref.shape or t.device != ref.device):
+        raise ValueError(f"{name} must match q: {tuple(ref.shape)} on {ref.device}")
+    return tuple(t.shape)
+
+
+def _side(name: str, t: torch.Tensor, shape, dtype) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+
+
+def _doc_ptr(doc, B, T):
+    if doc is None:
+        return None
+    _side("doc_offsets", doc, (B, T), torch.int32)
+    return doc.data_ptr()
+
+
+def gpt_attn_fwd(q, k, v, o, lse, scale: float, doc_offsets=None, stream=None) -> None:
+    B, H, T, d = _bhtd("q", q)
+    _bhtd("k", k, q)
+    _bhtd("v", v, q)
+    _bhtd("o", o, q)
+    _side("lse", lse, (B, H, T), torch.float32)
+    _check("gpt_attn_fwd", load().gpt_attn_fwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, d,
+        float(scale), _doc_ptr(doc_offsets, B, T), _stream(stream)))
+
+
+def gpt_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, scale: float, doc_offsets=None,
+                 stream=None) -> None:
+    B, H, T, d = _bhtd("q", q)
+    for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _bhtd(name, t, q)
+    _side("lse", lse, (B, H, T), torch.float32)
+    _side("delta_ws", delta_ws, (B, H, T), torch.float32)
+    _check("gpt_attn_bwd", load().gpt_attn_bwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), delta_ws.data_ptr(), B, H, T, d, float(scale),
+        _doc_ptr(doc_offsets, B, T), _stream(stream)))
+
+
+def gpt_attn_bwd_preprocess(o, dout, delta, stream=None) -> None:
+    B, H, T, d = _bhtd("o", o)
+    _bhtd("dout", dout, o)
+    _side("delta", delta, (B, H, T), torch.float32)
+    _check("gpt_attn_bwd_preprocess", load().gpt_attn_bwd_preprocess(
+        o.data_ptr(), dout.data_ptr(), delta.data_ptr(), B, H, T, d, _stream(stream)))
+
+
+def gpt_attn_bwd_dkdv(q, k, v, dout, lse, delta, dk, dv, scale: float, doc_offsets=None,
+                      stream=None) -> None:
+    B, H, T, d = _bhtd("q", q)
+    for name, t in (("k", k), ("v", v), ("dout", dout), ("dk", dk), ("dv", dv)):
+        _bhtd(name, t, q)
+    _side("lse", lse, (B, H, T), torch.float32)
+    _side("delta", delta, (B, H, T), torch.float32)
+    _check("gpt_attn_bwd_dkdv", load().gpt_attn_bwd_dkdv(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), lse.data_ptr(), delta.data_ptr(),
+        dk.data_ptr(), dv.data_ptr(), B, H, T, d, float(scale), _doc_ptr(doc_offsets, B, T),
+        _stream(stream)))
+
+
+def gpt_attn_bwd_dq(q, k, v, dout, lse, delta, dq, scale: float, doc_offsets=None,
+                    stream=None) -> None:
+    B, H, T, d = _bhtd("q", q)
+    for name, t in (("k", k), ("v", v), ("dout", dout), ("dq", dq)):
+        _bhtd(name, t, q)
+    _side("lse", lse, (B, H, T), torch.float32)
+    _side("delta", delta, (B, H, T), torch.float32)
+    _check("gpt_attn_bwd_dq", load().gpt_attn_bwd_dq(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), lse.data_ptr(), delta.data_ptr(),
+        dq.data_ptr(), B, H, T, d, float(scale), _doc_ptr(doc_offsets, B, T), _stream(stream)))
+
+
+def gpt_attn_check_doc_offsets(doc_offsets, stream=None) -> bool:
+    """True when the [B,T] int32 device array is a valid document-start array."""
+    if not isinstance(doc_offsets, torch.Tensor) or doc_offsets.dim() != 2:
+        raise ValueError("doc_offsets must be a [B,T] tensor")
+    B, T = doc_offsets.shape
+    _side("doc_offsets", doc_offsets, (B, T), torch.int32)
+    s = load().gpt_attn_check_doc_offsets(doc_offsets.data_ptr(), B, T, _stream(stream))
+    if s == GPT_ATTN_ERR_BAD_DOC_OFFSETS:
+        return False
+    _check("gpt_attn_check_doc_offsets", s)
+    return True
+
+
+def gpt_attn_device_status(clear: bool = False) -> int:
+    out = ctypes.c_uint(0)
+    _check("gpt_attn_device_status", load().gpt_attn_device_status(ctypes.byref(out), int(clear)))
+    return int(out.value)
+
+
+def gpt_attn_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
+    """Runs the bounded-wait self-test; returns the raw status (DEVICE_TIMEOUT expected)."""
+    return int(load().gpt_attn_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+# ------------------------------------------------------------ conveniences
+
+def attention_forward(q, k, v, scale: Optional[float] = None, doc_offsets=None, stream=None):
+    """Allocates O [B,H,T,d] bf16 and LSE [B,H,T] fp32 and runs gpt_attn_fwd."""
+    B, H, T, d = _bhtd("q", q)
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, T, device=q.device, dtype=torch.float32)
+    gpt_attn_fwd(q, k, v, o, lse, scale, doc_offsets, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, scale: Optional[float] = None, doc_offsets=None,
+                       stream=None):
+    """Allocates dQ, dK, dV and the delta workspace and runs gpt_attn_bwd."""
+    B, H, T, d = _bhtd("q", q)
+    if scale is None:
+        scale = d ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    delta = torch.empty(B, H, T, device=q.device, dtype=torch.float32)
+    gpt_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta, scale, doc_offsets, stream)
+    return dq, dk, dv
+
+
+class CausalSelfAttentionFunction(torch.autograd.Function):
+    """torch.autograd wrapper: y = attention(q, k, v) with the library's fwd/bwd kernels."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale, doc_offsets):
+        o, lse = attention_forward(q, k, v, scale, doc_offsets)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.scale, ctx.doc = scale, doc_offsets
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = attention_backward(q, k, v, o, lse, dout.contiguous(), ctx.scale, ctx.doc)
+        return dq, dk, dv, None, None
+
+
+def causal_attention(q, k, v, scale: Optional[float] = None, doc_offsets=None):
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    return CausalSelfAttentionFunction.apply(q, k, v, scale, doc_offsets)
+
+
+class HostStep:
+    """Forward + backward on pinned HOST tensors: copies the step's inputs to the
+    device, runs gpt_attn_fwd and gpt_attn_bwd, and copies O, LSE, dQ, dK, dV back
+    into caller-provided pinned host tensors, all on one stream.  The device
+    buffers are allocated once, here, by torch."""
+
+    def __init__(self, B: int, H: int, T: int, d: int, device="cuda"):
+        dev = torch.device(device)
+        bf = dict(device=dev, dtype=torch.bfloat16)
+        self.q, self.k, self.v, self.do, self.o, self.dq, self.dk, self.dv = (
+            torch.empty(B, H, T, d, **bf) for _ in range(8))
+        self.lse = torch.empty(B, H, T, device=dev, dtype=torch.float32)
+        self.delta = torch.empty(B, H, T, device=dev, dtype=torch.float32)
+        self.doc = None
+        self.shape = (B, H, T, d)
+
+    def set_doc_offsets(self, doc_host):
+        self.doc = None if doc_host is None else doc_host.to(self.q.device).contiguous()
+
+    def h2d_bytes(self) -> int:
+        return 4 * self.q.numel() * 2
+
+    def d2h_bytes(self) -> int:
+        return 4 * self.q.numel() * 2 + self.lse.numel() * 4
+
+    def run(self, q_h, k_h, v_h, do_h, out_h, scale: float, stream=None) -> None:
+        """out_h: dict with pinned host tensors 'o', 'lse', 'dq', 'dk', 'dv'.  Asynchronous."""
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            for dst, src in ((self.q, q_h), (self.k, k_h), (self.v, v_h), (self.do, do_h)):
+                dst.copy_(src, non_blocking=True)
+            gpt_attn_fwd(self.q, self.k, self.v, self.o, self.lse, scale, self.doc, s)
+            gpt_attn_bwd(self.q, self.k, self.v, self.o, self.do, self.lse, self.dq, self.dk,
+                         self.dv, self.delta, scale, self.doc, s)
+            for name in ("o", "lse", "dq", "dk", "dv"):
+                out_h[name].copy_(getattr(self, name), non_blocking=True)

@@ -1,0 +1,416 @@
+// causalattn.cu -- host side of libcausalattn: the C ABI declared in
+// include/causalattn.h (argument validation, TMA descriptor encoding,
+// per-device setup, kernel launches, status reporting) plus the small
+// utility kernels (document-offset validator, wait-timeout self-test).
+// The attention kernels themselves live in fwd.cuh and bwd.cuh.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/causalattn.h"
+#include "bwd.cuh"
+#include "fwd.cuh"
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------ validation
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(int B, int H, int T, int d) {
+  if (B < 1 || H < 1 || T < 1) return GPT_ATTN_ERR_BAD_SHAPE;
+  if (d != 32 && d != 64 && d != 128) return GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM;
+  const int64_t elems = (int64_t)B * H * T * d;
+  if (elems > (int64_t)INT32_MAX) return GPT_ATTN_ERR_TOO_LARGE;
+  return GPT_ATTN_OK;
+}
+
+int check_scale(float scale) {
+  if (!std::isfinite(scale) || !(scale > 0.f)) return GPT_ATTN_ERR_BAD_SCALE;
+  return GPT_ATTN_OK;
+}
+
+// ----------------------------------------------------------- device setup
+std::mutex g_mu;
+std::atomic<int> g_dev_state[kMaxDevices];  // 0 unknown, 1 ready, 2 wrong arch, 3 setup failed
+
+template <int D>
+cudaError_t set_smem_attrs() {
+  cudaError_t e;
+  e = cudaFuncSetAttribute(ca::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           ca::FwdLayout<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(ca::attn_bwd_dkdv_kernel<D>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DkdvLayout<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(ca::attn_bwd_dq_kernel<D>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DqLayout<D>::SMEM);
+}
+
+int ensure_device() {
+  int count = 0;
+  if (cudaGetDeviceCount(&count) != cudaSuccess || count < 1) {
+    cudaGetLastError();
+    return GPT_ATTN_ERR_NO_DEVICE;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return GPT_ATTN_ERR_NO_DEVICE;
+  }
+  int st = g_dev_state[dev].load(std::memory_order_acquire);
+  if (st == 0) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    st = g_dev_state[dev].load(std::memory_order_relaxed);
+    if (st == 0) {
+      int major = 0, minor = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return GPT_ATTN_ERR_NO_DEVICE;
+      }
+      if (major != 10 || minor != 0) {
+        st = 2;
+      } else if (set_smem_attrs<32>() != cudaSuccess || set_smem_attrs<64>() != cudaSuccess ||
+                 set_smem_attrs<128>() != cudaSuccess) {
+        cudaGetLastError();
+        st = 3;
+      } else {
+        st = 1;
+      }
+      g_dev_state[dev].store(st, std::memory_order_release);
+    }
+  }
+  if (st == 1) return GPT_ATTN_OK;
+  if (st == 2) return GPT_ATTN_ERR_UNSUPPORTED_ARCH;
+  return GPT_ATTN_ERR_LAUNCH;
+}
+
+// ------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// A [B*H, T, d] bf16 tensor viewed as 3-D (d innermost), boxes of
+// (swizzle width, 128 rows, 1 head); rows past T read as zero.
+template <int D>
+bool make_map(CUtensorMap* m, const void* base, int BH, int T) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  using Tl = ca::Tile<D>;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
+  cuuint32_t box[3] = {(cuuint32_t)Tl::BOX_COLS, (cuuint32_t)ca::kRows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   Tl::SW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_LAUNCH;
+}
+
+// ------------------------------------------------------------- launchers
+template <int D>
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
+             float scale, const int32_t* doc, cudaStream_t st) {
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map<D>(&mq, q, BH, T) || !make_map<D>(&mk, k, BH, T) || !make_map<D>(&mv, v, BH, T))
+    return GPT_ATTN_ERR_LAUNCH;
+  ca::FwdParams p;
+  p.doc = doc;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.H = H;
+  p.T = T;
+  p.BH = BH;
+  p.n_qt = (T + ca::kRows - 1) / ca::kRows;
+  p.scale_log2 = scale * ca::kLog2e;
+  p.wait_limit_ns = kWaitLimitNs;
+  const unsigned grid = (unsigned)p.n_qt * (unsigned)BH;
+  ca::attn_fwd_kernel<D><<<grid, ca::FwdLayout<D>::THREADS, ca::FwdLayout<D>::SMEM, st>>>(mq, mk,
+                                                                                         mv, p);
+  return launch_status();
+}
+
+template <int D>
+int delta_impl(const void* o, const void* dout, float* delta, int B, int H, int T,
+               cudaStream_t st) {
+  const long rows = (long)B * H * T;
+  const long threads = rows * (D / 8);
+  long blocks = (threads + 255) / 256;
+  if (blocks > 148L * 16) blocks = 148L * 16;
+  ca::attn_bwd_delta_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
+  return launch_status();
+}
+
+template <int D>
+int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const void* dout,
+                   const float* lse, const float* delta, void* g0, void* g1, int B, int H, int T,
+                   float scale, const int32_t* doc, cudaStream_t st) {
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map<D>(&mq, q, BH, T) || !make_map<D>(&mk, k, BH, T) || !make_map<D>(&mv, v, BH, T) ||
+      !make_map<D>(&mdo, dout, BH, T))
+    return GPT_ATTN_ERR_LAUNCH;
+  ca::BwdParams p;
+  p.doc = doc;
+  p.lse = lse;
+  p.delta = delta;
+  p.g0 = static_cast<__nv_bfloat16*>(g0);
+  p.g1 = static_cast<__nv_bfloat16*>(g1);
+  p.H = H;
+  p.T = T;
+  p.BH = BH;
+  p.n_t = (T + ca::kRows - 1) / ca::kRows;
+  p.scale = scale;
+  p.scale_log2 = scale * ca::kLog2e;
+  p.wait_limit_ns = kWaitLimitNs;
+  const unsigned grid = (unsigned)p.n_t * (unsigned)BH;
+  if (dkdv)
+    ca::attn_bwd_dkdv_kernel<D>
+        <<<grid, ca::DkdvLayout<D>::THREADS, ca::DkdvLayout<D>::SMEM, st>>>(mq, mk, mv, mdo, p);
+  else
+    ca::attn_bwd_dq_kernel<D>
+        <<<grid, ca::DqLayout<D>::THREADS, ca::DqLayout<D>::SMEM, st>>>(mq, mk, mv, mdo, p);
+  return launch_status();
+}
+
+// -------------------------------------------------------- utility kernels
+__device__ int g_doc_bad;
+
+__global__ void check_doc_kernel(const int32_t* doc, int B, int T) {
+  const long n = (long)B * T;
+  for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long)gridDim.x * blockDim.x) {
+    const int i = (int)(e % T);
+    const int v = doc[e];
+    const bool ok = (i == 0) ? (v == 0) : (v == i || v == doc[e - 1]);
+    if (!ok) atomicOr(&g_doc_bad, 1);
+  }
+}
+
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    ca::mbar_init(ca::smem_u32(&bar), 1);
+    ca::fence_barrier_init();
+    const ca::Guard g{&abort_flag, limit_ns};
+    // nothing ever arrives on `bar`: the wait must give up and report
+    ca::wait_bounded(ca::smem_u32(&bar), 0, g, 14);
+  }
+}
+
+int common_checks(int B, int H, int T, int d) { return check_shape(B, H, T, d); }
+
+}  // namespace
+
+// ======================================================================== ABI
+extern "C" {
+
+int gpt_attn_version(void) { return GPT_ATTN_ABI_VERSION; }
+
+const char* gpt_attn_strerror(int s) {
+  switch (s) {
+    case GPT_ATTN_OK: return "ok";
+    case GPT_ATTN_ERR_NULL_PTR: return "a required pointer is NULL";
+    case GPT_ATTN_ERR_BAD_SHAPE: return "B, H and T must be >= 1";
+    case GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM: return "head dim d must be 32, 64 or 128";
+    case GPT_ATTN_ERR_MISALIGNED: return "bf16 tensors need 16-byte alignment, fp32/int32 arrays 4-byte";
+    case GPT_ATTN_ERR_BAD_DOC_OFFSETS: return "doc_offsets is not a valid document-start array";
+    case GPT_ATTN_ERR_NO_DEVICE: return "no usable CUDA device";
+    case GPT_ATTN_ERR_UNSUPPORTED_ARCH: return "current device is not sm_100 (B200)";
+    case GPT_ATTN_ERR_LAUNCH: return "CUDA launch or setup failed";
+    case GPT_ATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case GPT_ATTN_ERR_NOT_IMPLEMENTED: return "not implemented";
+    case GPT_ATTN_ERR_BAD_SCALE: return "scale must be finite and > 0";
+    case GPT_ATTN_ERR_TOO_LARGE: return "tensor too large (B*H*T*d must be < 2^31)";
+    default: return "unknown status";
+  }
+}
+
+int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int T, int d, float scale, const int32_t* doc_offsets, void* stream) {
+  if (!q || !k || !v || !o || !lse) return GPT_ATTN_ERR_NULL_PTR;
+  int s = common_checks(B, H, T, d);
+  if (s) return s;
+  if ((s = check_scale(scale))) return s;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(doc_offsets, 4))
+    return GPT_ATTN_ERR_MISALIGNED;
+  if ((s = ensure_device())) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 32: return fwd_impl<32>(q, k, v, o, lse, B, H, T, scale, doc_offsets, st);
+    case 64: return fwd_impl<64>(q, k, v, o, lse, B, H, T, scale, doc_offsets, st);
+    default: return fwd_impl<128>(q, k, v, o, lse, B, H, T, scale, doc_offsets, st);
+  }
+}
+
+int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B, int H, int T,
+                            int d, void* stream) {
+  if (!o || !dout || !delta) return GPT_ATTN_ERR_NULL_PTR;
+  int s = common_checks(B, H, T, d);
+  if (s) return s;
+  if (!aligned(o, 16) || !aligned(dout, 16) || !aligned(delta, 4)) return GPT_ATTN_ERR_MISALIGNED;
+  if ((s = ensure_device())) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 32: return delta_impl<32>(o, dout, delta, B, H, T, st);
+    case 64: return delta_impl<64>(o, dout, delta, B, H, T, st);
+    default: return delta_impl<128>(o, dout, delta, B, H, T, st);
+  }
+}
+
+static int bwd_step(bool dkdv, const void* q, const void* k, const void* v, const void* dout,
+                    const float* lse, const float* delta, void* g0, void* g1, int B, int H, int T,
+                    int d, float scale, const int32_t* doc, void* stream) {
+  if (!q || !k || !v || !dout || !lse || !delta || !g0 || (dkdv && !g1))
+    return GPT_ATTN_ERR_NULL_PTR;
+  int s = common_checks(B, H, T, d);
+  if (s) return s;
+  if ((s = check_scale(scale))) return s;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) ||
+      !aligned(g0, 16) || (dkdv && !aligned(g1, 16)) || !aligned(lse, 4) || !aligned(delta, 4) ||
+      !aligned(doc, 4))
+    return GPT_ATTN_ERR_MISALIGNED;
+  if ((s = ensure_device())) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 32: return bwd_tiled_impl<32>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, st);
+    case 64: return bwd_tiled_impl<64>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, st);
+    default: return bwd_tiled_impl<128>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, st);
+  }
+}
+
+int gpt_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
+                      const float* lse, const float* delta, void* dk, void* dv, int B, int H,
+                      int T, int d, float scale, const int32_t* doc_offsets, void* stream) {
+  return bwd_step(true, q, k, v, dout, lse, delta, dk, dv, B, H, T, d, scale, doc_offsets, stream);
+}
+
+int gpt_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
+                    const float* lse, const float* delta, void* dq, int B, int H, int T, int d,
+                    float scale, const int32_t* doc_offsets, void* stream) {
+  return bwd_step(false, q, k, v, dout, lse, delta, dq, nullptr, B, H, T, d, scale, doc_offsets,
+                  stream);
+}
+
+int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, float* delta_ws, int B, int H,
+                 int T, int d, float scale, const int32_t* doc_offsets, void* stream) {
+  // validate everything before the first launch, so an error never leaves a partial backward
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !delta_ws)
+    return GPT_ATTN_ERR_NULL_PTR;
+  int s = common_checks(B, H, T, d);
+  if (s) return s;
+  if ((s = check_scale(scale))) return s;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(delta_ws, 4) || !aligned(doc_offsets, 4))
+    return GPT_ATTN_ERR_MISALIGNED;
+  if ((s = ensure_device())) return s;
+  if ((s = gpt_attn_bwd_preprocess(o, dout, delta_ws, B, H, T, d, stream))) return s;
+  if ((s = gpt_attn_bwd_dkdv(q, k, v, dout, lse, delta_ws, dk, dv, B, H, T, d, scale, doc_offsets,
+                             stream)))
+    return s;
+  return gpt_attn_bwd_dq(q, k, v, dout, lse, delta_ws, dq, B, H, T, d, scale, doc_offsets, stream);
+}
+
+int gpt_attn_check_doc_offsets(const int32_t* doc_offsets, int B, int T, void* stream) {
+  if (!doc_offsets) return GPT_ATTN_ERR_NULL_PTR;
+  if (B < 1 || T < 1) return GPT_ATTN_ERR_BAD_SHAPE;
+  if ((int64_t)B * T > (int64_t)INT32_MAX) return GPT_ATTN_ERR_TOO_LARGE;
+  if (!aligned(doc_offsets, 4)) return GPT_ATTN_ERR_MISALIGNED;
+  int s = ensure_device();
+  if (s) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_doc_bad, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return GPT_ATTN_ERR_LAUNCH;
+  }
+  long blocks = ((long)B * T + 255) / 256;
+  if (blocks > 148L * 8) blocks = 148L * 8;
+  check_doc_kernel<<<(unsigned)blocks, 256, 0, st>>>(doc_offsets, B, T);
+  if ((s = launch_status())) return s;
+  int bad = 0;
+  if (cudaMemcpyFromSymbolAsync(&bad, g_doc_bad, sizeof(int), 0, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return GPT_ATTN_ERR_LAUNCH;
+  }
+  return bad ? GPT_ATTN_ERR_BAD_DOC_OFFSETS : GPT_ATTN_OK;
+}
+
+int gpt_attn_device_status(unsigned int* out, int clear) {
+  if (!out) return GPT_ATTN_ERR_NULL_PTR;
+  int s = ensure_device();
+  if (s) return s;
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpyFromSymbol(out, ca::g_status, sizeof(unsigned)) != cudaSuccess) {
+    cudaGetLastError();
+    return GPT_ATTN_ERR_LAUNCH;
+  }
+  if (clear) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(ca::g_status, &zero, sizeof(unsigned)) != cudaSuccess) {
+      cudaGetLastError();
+      return GPT_ATTN_ERR_LAUNCH;
+    }
+  }
+  return GPT_ATTN_OK;
+}
+
+int gpt_attn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  int s = ensure_device();
+  if (s) return s;
+  unsigned before = 0;
+  if ((s = gpt_attn_device_status(&before, 1))) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns);
+  if ((s = launch_status())) return s;
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return GPT_ATTN_ERR_LAUNCH;
+  }
+  unsigned after = 0;
+  if ((s = gpt_attn_device_status(&after, 1))) return s;
+  return (after & ca::kStatusTimeout) ? GPT_ATTN_ERR_DEVICE_TIMEOUT : GPT_ATTN_OK;
+}
+
+}  // extern "C"

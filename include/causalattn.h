@@ -1,0 +1,149 @@
+/*
+ * causalattn.h -- C ABI of libcausalattn: multi-head causal scaled-dot-product
+ * self-attention, forward and backward, on NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For every batch b and head h, with Q, K, V, dO slices of
+ * shape [T, d]:
+ *     S   = scale * Q K^T                      (scale is normally 1/sqrt(d))
+ *     S_ij = -inf  where j > i                 (causal mask, diagonal kept)
+ *     P   = softmax(S) along each row
+ *     O   = P V,      LSE_i = log sum_j exp(S_ij)   (natural log)
+ * as written in "Stanford CS336 walkthrough" (lmnt.cn), section 5.1 model.py,
+ * CausalSelfAttention.forward (q @ k^T * 1/sqrt(k.size(-1)), masked_fill of
+ * the upper triangle with -inf, softmax, att @ v), section 3.3 of the same
+ * page (masked positions get weight 0 after the softmax), and the
+ * torch.tril(ones) mask buffer of "Train Your Own LLM from Scratch"
+ * (fishgap.com), section 1, which keeps the diagonal.  Attention dropout is
+ * the identity (p = 0.0 in every configuration the pages print).
+ *
+ * The backward is the gradient of that forward for loss.backward() (CS336
+ * walkthrough, section 5.2 train.py):
+ *     dV = P^T dO,  dP = dO V^T,  delta_i = sum_c dO_ic O_ic,
+ *     dS = P o (dP - delta),  dQ = scale dS K,  dK = scale dS^T Q.
+ *
+ * Document mask (optional).  BOS-aligned best-fit packing puts several
+ * documents in one row ("How to build an LLM by hand", agmtopy.github.io,
+ * section 5.5).  Reading: a token attends only to earlier tokens of its own
+ * document.  doc_offsets is an int32 device array [B, T]; entry [b, i] is the
+ * first position of the document that holds position i.  Position i attends
+ * to j iff doc_offsets[b, i] <= j <= i.  Valid arrays have doc_offsets[b,0] =
+ * 0 and each entry equal to i (a new document) or to the previous entry.
+ * NULL means plain causal attention.
+ *
+ * Layouts.  q, k, v, o, dout, dq, dk, dv: contiguous bf16 [B, H, T, d]
+ * (d fastest), the layout of the pages' .view(B, T, H, C//H).transpose(1, 2).
+ * lse, delta: contiguous fp32 [B, H, T].
+ *
+ * Ownership.  Every pointer is caller-owned DEVICE memory on the current CUDA
+ * device.  The library allocates no memory; it keeps no state besides
+ * per-device attribute caches and one device-side status word.
+ *
+ * Asynchrony.  Calls validate their arguments, enqueue kernels on `stream`
+ * (a cudaStream_t; NULL = the legacy default stream) and return.  Outputs are
+ * valid once the stream has reached that point.  Inputs are not modified.
+ * dq, dk, dv, o, lse, delta are fully overwritten, never accumulated into.
+ *
+ * Errors.  Every call returns a gpt_attn_status.  Nothing aborts, throws or
+ * exits across this boundary.  Arguments are checked before any CUDA call, so
+ * argument errors are reported even on a machine without a GPU.  A launch
+ * failure returns GPT_ATTN_ERR_LAUNCH.  Kernels never wait without bound: a
+ * wait that exceeds its limit (2 s) makes the kernel record the event in the
+ * device status word (read it with gpt_attn_device_status) and exit early,
+ * leaving the outputs unspecified.  An invalid doc_offsets array yields
+ * unspecified output values but never an out-of-bounds access.
+ *
+ * Limits.  d in {32, 64, 128}; T >= 1 (any T: tiles past T are masked);
+ * B, H >= 1 with B*H*T*d < 2^31 elements per tensor; scale finite and > 0;
+ * the bf16 tensors 16-byte aligned, lse/delta/doc_offsets 4-byte aligned.
+ */
+#ifndef CAUSALATTN_H
+#define CAUSALATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPT_ATTN_ABI_VERSION 1
+
+typedef enum {
+  GPT_ATTN_OK = 0,
+  GPT_ATTN_ERR_NULL_PTR = 1,              /* a required pointer is NULL */
+  GPT_ATTN_ERR_BAD_SHAPE = 2,             /* B, H or T < 1 */
+  GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM = 3,  /* d not in {32, 64, 128} */
+  GPT_ATTN_ERR_MISALIGNED = 4,            /* a pointer breaks the alignment rule above */
+  GPT_ATTN_ERR_BAD_DOC_OFFSETS = 5,       /* gpt_attn_check_doc_offsets found an invalid entry */
+  GPT_ATTN_ERR_NO_DEVICE = 6,             /* no usable CUDA device */
+  GPT_ATTN_ERR_UNSUPPORTED_ARCH = 7,      /* current device is not sm_100 (B200) */
+  GPT_ATTN_ERR_LAUNCH = 8,                /* a CUDA call or kernel launch failed */
+  GPT_ATTN_ERR_DEVICE_TIMEOUT = 9,        /* a kernel gave up on a bounded wait */
+  GPT_ATTN_ERR_NOT_IMPLEMENTED = 10,
+  GPT_ATTN_ERR_BAD_SCALE = 11,            /* scale not finite or <= 0 */
+  GPT_ATTN_ERR_TOO_LARGE = 12             /* a tensor exceeds 2^31 - 1 elements */
+} gpt_attn_status;
+
+/*
+ * Forward.  Reads q, k, v [B,H,T,d]; writes o [B,H,T,d] and lse [B,H,T].
+ */
+int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int T, int d, float scale, const int32_t* doc_offsets, void* stream);
+
+/*
+ * Backward.  Reads q, k, v, o, dout [B,H,T,d] and lse [B,H,T] (the forward's
+ * outputs); writes dq, dk, dv [B,H,T,d].  delta_ws is a caller-provided fp32
+ * [B,H,T] workspace that receives delta = rowsum(dout o o).  Equivalent to
+ * gpt_attn_bwd_preprocess, then gpt_attn_bwd_dkdv, then gpt_attn_bwd_dq.
+ */
+int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, float* delta_ws, int B, int H,
+                 int T, int d, float scale, const int32_t* doc_offsets, void* stream);
+
+/* Backward step 1: delta[b,h,i] = sum_c dout[b,h,i,c] * o[b,h,i,c] (fp32). */
+int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B, int H, int T,
+                            int d, void* stream);
+
+/* Backward step 2: dk, dv [B,H,T,d] from q, k, v, dout, lse and delta. */
+int gpt_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
+                      const float* lse, const float* delta, void* dk, void* dv, int B, int H,
+                      int T, int d, float scale, const int32_t* doc_offsets, void* stream);
+
+/* Backward step 3: dq [B,H,T,d] from q, k, v, dout, lse and delta. */
+int gpt_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
+                    const float* lse, const float* delta, void* dq, int B, int H, int T, int d,
+                    float scale, const int32_t* doc_offsets, void* stream);
+
+/*
+ * Checks a doc_offsets array on the device against the validity rule above.
+ * Synchronises `stream`.  Returns GPT_ATTN_OK or GPT_ATTN_ERR_BAD_DOC_OFFSETS.
+ */
+int gpt_attn_check_doc_offsets(const int32_t* doc_offsets, int B, int T, void* stream);
+
+/*
+ * Reads (and, if clear != 0, resets) the device status word of the current
+ * device: 0 when no kernel has given up on a wait, otherwise bit 31 plus one
+ * bit per wait site.  Synchronises the device.  Returns GPT_ATTN_OK, or an
+ * error status if the device cannot be read.
+ */
+int gpt_attn_device_status(unsigned int* out, int clear);
+
+/*
+ * Failure-detection self-test: launches one kernel that waits, with the given
+ * limit in nanoseconds, on a barrier nothing ever signals.  The kernel must
+ * give up, record the timeout and exit.  Synchronises `stream`, clears the
+ * status word again and returns GPT_ATTN_ERR_DEVICE_TIMEOUT when the timeout
+ * was detected and reported (the expected outcome), GPT_ATTN_OK if it was not.
+ */
+int gpt_attn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gpt_attn_strerror(int status);
+
+/* GPT_ATTN_ABI_VERSION of the loaded library. */
+int gpt_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CAUSALATTN_H */

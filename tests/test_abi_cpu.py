@@ -1,0 +1,104 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments before making any CUDA call."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+import torch
+
+from causal_self_attention_mha_b200 import abi, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "causalattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return abi.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gpt_attn_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "gpt_attn_fwd" in names and "gpt_attn_bwd" in names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in abi.SIGNATURES, f"binding lacks {n}"
+
+
+def test_version_and_strerror(lib):
+    assert lib.gpt_attn_version() == 1
+    for s in range(0, 13):
+        msg = lib.gpt_attn_strerror(s)
+        assert isinstance(msg, bytes) and len(msg) > 0
+    assert lib.gpt_attn_strerror(999) == b"unknown status"
+
+
+# fake, never-dereferenced, 16-byte aligned addresses: validation must reject before use
+P = [0x10000 + 0x100 * i for i in range(12)]
+
+
+def fwd(lib, q=P[0], k=P[1], v=P[2], o=P[3], lse=P[4], B=1, H=2, T=64, d=64, scale=0.125, doc=None):
+    return lib.gpt_attn_fwd(q, k, v, o, lse, B, H, T, d, scale, doc, None)
+
+
+def test_fwd_argument_errors(lib):
+    assert fwd(lib, q=None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert fwd(lib, lse=None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert fwd(lib, B=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    assert fwd(lib, T=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    assert fwd(lib, H=-1) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    for d in (16, 48, 96, 256):
+        assert fwd(lib, d=d) == abi.GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM
+    for s in (0.0, -1.0, math.inf, math.nan):
+        assert fwd(lib, scale=s) == abi.GPT_ATTN_ERR_BAD_SCALE
+    assert fwd(lib, q=P[0] + 8) == abi.GPT_ATTN_ERR_MISALIGNED
+    assert fwd(lib, o=P[3] + 2) == abi.GPT_ATTN_ERR_MISALIGNED
+    assert fwd(lib, lse=P[4] + 2) == abi.GPT_ATTN_ERR_MISALIGNED
+    assert fwd(lib, doc=P[5] + 1) == abi.GPT_ATTN_ERR_MISALIGNED
+    assert fwd(lib, B=1 << 12, H=1 << 12, T=1 << 10, d=128) == abi.GPT_ATTN_ERR_TOO_LARGE
+
+
+def test_bwd_argument_errors(lib):
+    def bwd(**kw):
+        a = dict(q=P[0], k=P[1], v=P[2], o=P[3], do=P[4], lse=P[5], dq=P[6], dk=P[7], dv=P[8],
+                 delta=P[9], B=1, H=2, T=64, d=64, scale=0.125, doc=None)
+        a.update(kw)
+        return lib.gpt_attn_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"],
+                                a["dv"], a["delta"], a["B"], a["H"], a["T"], a["d"], a["scale"],
+                                a["doc"], None)
+    for name in ("q", "k", "v", "o", "do", "lse", "dq", "dk", "dv", "delta"):
+        assert bwd(**{name: None}) == abi.GPT_ATTN_ERR_NULL_PTR, name
+    assert bwd(T=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    assert bwd(d=80) == abi.GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM
+    assert bwd(scale=-0.5) == abi.GPT_ATTN_ERR_BAD_SCALE
+    assert bwd(dk=P[7] + 4) == abi.GPT_ATTN_ERR_MISALIGNED
+    assert lib.gpt_attn_bwd_preprocess(P[0], None, P[2], 1, 1, 8, 32, None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert lib.gpt_attn_bwd_dkdv(P[0], P[1], P[2], P[3], P[4], P[5], P[6], None, 1, 1, 8, 32, 0.1,
+                                 None, None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert lib.gpt_attn_bwd_dq(P[0], P[1], P[2], P[3], P[4], P[5], P[6], 1, 1, 8, 40, 0.1,
+                               None, None) == abi.GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM
+    assert lib.gpt_attn_check_doc_offsets(None, 1, 8, None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert lib.gpt_attn_check_doc_offsets(P[0], 0, 8, None) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    out = ctypes.c_uint(0)
+    assert lib.gpt_attn_device_status(None, 0) == abi.GPT_ATTN_ERR_NULL_PTR
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_valid_arguments_without_a_gpu_report_no_device(lib):
+    assert fwd(lib) == abi.GPT_ATTN_ERR_NO_DEVICE
+    assert lib.gpt_attn_selftest_wait_timeout(1000, None) == abi.GPT_ATTN_ERR_NO_DEVICE
+
+
+def test_binding_rejects_host_tensors(lib):
+    q = torch.zeros(1, 1, 8, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        abi.gpt_attn_fwd(q, q, q, q, torch.zeros(1, 1, 8), 0.1)

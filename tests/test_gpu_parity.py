@@ -1,0 +1,218 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU fp64 oracle, on
+the same seeded bf16 inputs.
+
+Tolerances (bf16 inputs, fp32 accumulation, bf16 outputs):
+  O    max |gpu - oracle|                       <= 1e-2
+  LSE  max |gpu - oracle|                       <= 1e-3
+  dQ, dK, dV  ||gpu - oracle||_2 / ||oracle||_2  <= 2e-2   (per tensor; ||oracle|| floored
+              at 1e-3 RMS so that exactly-zero gradients are judged in absolute terms)
+The full-size workloads run in the same launch configuration the benchmark
+times; for the two T = 2048, d = 128 workloads the explicit-Jacobian oracle
+backward (O(T^3) per head) is evaluated on a spread of sampled heads (every
+head when CAUSALATTN_ORACLE_ALL_HEADS=1), the forward on every head.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from causal_self_attention_mha_b200 import abi, inputs
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL, GRAD_TOL = 1e-2, 1e-3, 2e-2
+
+
+def run_gpu(q, k, v, do, doc, scale):
+    dev = torch.device("cuda:0")
+    q, k, v, do = (t.to(dev).contiguous() for t in (q, k, v, do))
+    docd = doc.to(dev).contiguous() if doc is not None else None
+    o, lse = abi.attention_forward(q, k, v, scale, docd)
+    dq, dk, dv = abi.attention_backward(q, k, v, o, lse, do, scale, docd)
+    torch.cuda.synchronize()
+    return [t.cpu() for t in (o, lse, dq, dk, dv)]
+
+
+def oracle_heads(q, k, v, do, doc, scale, heads, with_grad=True):
+    """Oracle outputs for the listed (b, h) pairs: dict (b,h) -> (o, lse, dq, dk, dv)."""
+    out = {}
+    for b, h in heads:
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        ds = doc[b:b + 1] if doc is not None else None
+        o, lse = oracle.attention_forward(sl(q), sl(k), sl(v), scale, ds)
+        g = oracle.attention_backward(sl(q), sl(k), sl(v), sl(do), scale, ds) if with_grad else None
+        out[(b, h)] = (o, lse, g)
+    return out
+
+
+def rel_l2(a, b):
+    """||a - b|| / ||b||, with ||b|| floored at an RMS of 1e-3 per element: where the exact
+    gradient is zero (T = 1, uniform V) the GPU's fp32 rounding residue is judged absolutely."""
+    floor = 1e-3 * np.sqrt(b.size)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), floor))
+
+
+def compare(gpu, q, k, v, do, doc, scale, grad_heads=None, label=""):
+    """Forward on every head (one oracle call); backward on grad_heads (None = all)."""
+    o_g, lse_g, dq_g, dk_g, dv_g = (t.to(torch.float64).numpy() for t in gpu)
+    B, H = q.shape[:2]
+    o_r, lse_r = oracle.attention_forward(q, k, v, scale, doc)
+    err_o = float(np.max(np.abs(o_g - o_r)))
+    err_l = float(np.max(np.abs(lse_g - lse_r)))
+    if grad_heads is None:
+        dq_r, dk_r, dv_r = oracle.attention_backward(q, k, v, do, scale, doc)
+        sel = (slice(None), slice(None))
+        errs = [rel_l2(g[sel], r) for g, r in ((dq_g, dq_r), (dk_g, dk_r), (dv_g, dv_r))]
+    else:
+        ref = oracle_heads(q, k, v, do, doc, scale, grad_heads)
+        errs = []
+        for i, g in enumerate((dq_g, dk_g, dv_g)):
+            gs = np.concatenate([g[b, h].ravel() for b, h in grad_heads])
+            rs = np.concatenate([ref[(b, h)][2][i].ravel() for b, h in grad_heads])
+            errs.append(rel_l2(gs, rs))
+    print(f"{label}: O maxabs {err_o:.3e}  LSE maxabs {err_l:.3e}  "
+          f"dQ {errs[0]:.3e} dK {errs[1]:.3e} dV {errs[2]:.3e}")
+    assert np.all(np.isfinite(o_g)) and np.all(np.isfinite(lse_g))
+    assert err_o <= O_TOL, (label, "O", err_o)
+    assert err_l <= LSE_TOL, (label, "LSE", err_l)
+    for name, e in zip(("dQ", "dK", "dV"), errs):
+        assert e <= GRAD_TOL, (label, name, e)
+    return err_o, err_l, errs
+
+
+def no_device_timeouts():
+    st = abi.gpt_attn_device_status(clear=True)
+    assert st == 0, f"device status word {st:#x}: a kernel gave up on a wait"
+
+
+# ------------------------------------------------------------ full workloads
+
+def sampled_heads(B, H, n=8):
+    idx = np.linspace(0, B * H - 1, n).round().astype(int)
+    return sorted({(int(i) // H, int(i) % H) for i in idx})
+
+
+@pytest.mark.parametrize("name", list(inputs.WORKLOADS))
+def test_workload_parity(name, cuda_device):
+    w = inputs.WORKLOADS[name]
+    q, k, v, do, doc = inputs.make_workload(w)
+    gpu = run_gpu(q, k, v, do, doc, w.scale)
+    heads = None
+    if w.T >= 2048 and os.environ.get("CAUSALATTN_ORACLE_ALL_HEADS") != "1":
+        heads = sampled_heads(w.B, w.H)
+    compare(gpu, q, k, v, do, doc, w.scale, heads, label=name)
+    no_device_timeouts()
+
+
+# ------------------------------------------------- tails, tiny and odd shapes
+
+@pytest.mark.parametrize("T", [1, 2, 17, 63, 64, 65, 127, 128, 129, 200, 255, 257, 300])
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_ragged_lengths(T, d, cuda_device):
+    B, H = 1, 2
+    q, k, v, do = inputs.make_qkvdo(B, H, T, d, 1000 + T + d)
+    scale = inputs.fp32_scale(d)
+    compare(run_gpu(q, k, v, do, None, scale), q, k, v, do, None, scale, label=f"T{T} d{d}")
+    no_device_timeouts()
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("lo,hi", [(1, 4), (5, 40), (60, 300)])
+def test_document_masks(d, lo, hi, cuda_device):
+    B, H, T = 2, 2, 389
+    q, k, v, do = inputs.make_qkvdo(B, H, T, d, 7 * lo + d)
+    doc = inputs.random_doc_start(B, T, lo + hi, lo, hi)
+    scale = inputs.fp32_scale(d)
+    compare(run_gpu(q, k, v, do, doc, scale), q, k, v, do, doc, scale, label=f"doc[{lo},{hi}] d{d}")
+    no_device_timeouts()
+
+
+def test_many_tiles_one_head(cuda_device):
+    B, H, T, d = 1, 1, 4096, 64
+    q, k, v, do = inputs.make_qkvdo(B, H, T, d, 4242)
+    scale = inputs.fp32_scale(d)
+    compare(run_gpu(q, k, v, do, None, scale), q, k, v, do, None, scale, label="T4096")
+
+
+def test_other_scale(cuda_device):
+    """The scale is an argument: a non-default value must be honoured end to end."""
+    B, H, T, d = 1, 2, 150, 64
+    q, k, v, do = inputs.make_qkvdo(B, H, T, d, 31)
+    compare(run_gpu(q, k, v, do, None, 0.3), q, k, v, do, None, 0.3, label="scale0.3")
+
+
+# ------------------------------------------------------------- properties
+
+def test_deterministic(cuda_device):
+    w = inputs.WORKLOADS["gpt2_small"]
+    q, k, v, do, doc = inputs.make_workload(w)
+    a = run_gpu(q, k, v, do, doc, w.scale)
+    b = run_gpu(q, k, v, do, doc, w.scale)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_uniform_values_on_gpu(cuda_device):
+    """All value rows equal: every output row equals that row (up to its bf16 rounding)."""
+    B, H, T, d = 1, 2, 300, 64
+    q, k, _, do = inputs.make_qkvdo(B, H, T, d, 5)
+    u = torch.randn(d, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    v = u.expand(B, H, T, d).contiguous()
+    o, lse, dq, dk, dv = run_gpu(q, k, v, do, None, inputs.fp32_scale(d))
+    exact = torch.eq(o, v).double().mean().item()
+    print(f"uniform V: {exact:.4%} of O elements bit-equal to V")
+    assert (o.float() - v.float()).abs().max() <= O_TOL
+    assert dq.abs().max() < 2e-2 and dk.abs().max() < 2e-2
+
+
+def test_autograd_wrapper(cuda_device):
+    B, H, T, d = 1, 2, 96, 32
+    q, k, v, do = inputs.make_qkvdo(B, H, T, d, 9)
+    dev = torch.device("cuda:0")
+    tq, tk, tv = (t.to(dev).requires_grad_(True) for t in (q, k, v))
+    o = abi.causal_attention(tq, tk, tv)
+    o.backward(do.to(dev))
+    gpu = [o.detach().cpu(), torch.zeros(B, H, T), tq.grad.cpu(), tk.grad.cpu(), tv.grad.cpu()]
+    o_r, _ = oracle.attention_forward(q, k, v, inputs.fp32_scale(d))
+    assert np.max(np.abs(gpu[0].double().numpy() - o_r)) <= O_TOL
+    g = oracle.attention_backward(q, k, v, do, inputs.fp32_scale(d))
+    for a, r in zip(gpu[2:], g):
+        assert rel_l2(a.double().numpy(), r) <= GRAD_TOL
+
+
+# ------------------------------------------------------- errors and faults
+
+def test_doc_offsets_validator(cuda_device):
+    dev = torch.device("cuda:0")
+    good = inputs.random_doc_start(3, 500, 2, 10, 90).to(dev)
+    assert abi.gpt_attn_check_doc_offsets(good)
+    bad = good.clone()
+    bad[1, 37] = 40  # points past its own position
+    assert not abi.gpt_attn_check_doc_offsets(bad)
+    bad = good.clone()
+    bad[2, 0] = 1
+    assert not abi.gpt_attn_check_doc_offsets(bad)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
+    """A wait on a barrier nobody signals gives up after its limit, reports through the status
+    word, and leaves the CUDA context usable."""
+    assert abi.gpt_attn_selftest_wait_timeout(2_000_000) == abi.GPT_ATTN_ERR_DEVICE_TIMEOUT
+    assert abi.gpt_attn_device_status() == 0
+    B, H, T, d = 1, 1, 130, 64
+    q, k, v, do = inputs.make_qkvdo(B, H, T, d, 77)
+    compare(run_gpu(q, k, v, do, None, 0.125), q, k, v, do, None, 0.125, label="after-timeout")
+
+
+def test_gpu_argument_errors(cuda_device):
+    q = torch.zeros(1, 1, 64, 48, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(1, 1, 64, device="cuda")
+    with pytest.raises(abi.AttnError) as e:
+        abi.gpt_attn_fwd(q, q, q, q, lse, 0.1)
+    assert e.value.status == abi.GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM
+    q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(abi.AttnError) as e:
+        abi.gpt_attn_fwd(q, q, q, q, lse, float("nan"))
+    assert e.value.status == abi.GPT_ATTN_ERR_BAD_SCALE
