@@ -190,7 +190,9 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int ds = p.doc ? p.doc[(size_t)b * T + (row < T ? row : T - 1)] : 0;
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    // l: sum of the fp32 weights (for the LSE); lr: sum of the bf16-rounded weights that the
+    // PV MMA actually multiplies (for normalising O, so its weights sum to one exactly)
+    float m = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
     for (int it = 0; it < n; ++it) {
       const int j = kv_lo + it;
@@ -238,6 +240,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (grow) {
         l *= alpha;
+        lr *= alpha;
         m = m_new;
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
@@ -247,8 +250,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2(x[32 * c + 2 * e] - mu), p1 = ex2(x[32 * c + 2 * e + 1] - mu);
-          l += p0 + p1;  // the row sum (and so the LSE) uses the unrounded weights
-          pk[e] = pack_bf16(p0, p1);
+          const uint32_t v = pack_bf16(p0, p1);
+          l += p0 + p1;
+          lr += bf16_lo(v) + bf16_hi(v);
+          pk[e] = v;
         }
         tmem_st16(tS + 16u * c, pk);
       }
@@ -260,7 +265,7 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ epilogue
     if (ok && wait_bounded_warp(o_done, (n - 1) & 1, g, 9)) {
       tc_fence_after();
-      const float inv = 1.0f / l;
+      const float inv = 1.0f / lr;
       const uint32_t tO = tmem + lane_off + 256u;
       __nv_bfloat16* orow = p.o + ((size_t)bh * T + row) * D;
 #pragma unroll
