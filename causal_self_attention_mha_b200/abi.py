@@ -44,6 +44,7 @@ SIGNATURES = {
     "gpt_attn_bwd_preprocess": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "gpt_attn_bwd_dkdv": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_bwd_dq": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
+    "gpt_attn_bwd_static_ws": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_check_doc_offsets": ([_vp, _i, _i, _vp], _i),
     "gpt_attn_device_status": ([ctypes.POINTER(ctypes.c_uint), _i], _i),
     "gpt_attn_selftest_wait_timeout": ([ctypes.c_uint64, _vp], _i),
@@ -151,6 +152,20 @@ def gpt_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, scale: float, doc_
     _check("gpt_attn_bwd", load().gpt_attn_bwd(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), delta_ws.data_ptr(), B, H, T, d, float(scale),
+        _doc_ptr(doc_offsets, B, T), _stream(stream)))
+
+
+def gpt_attn_bwd_static_ws(q, k, v, o, dout, lse, dq, dk, dv, scale: float, doc_offsets=None,
+                           stream=None) -> None:
+    """gpt_attn_bwd without a caller workspace: for callers that cannot allocate device memory
+    (the delta scratch is a fixed 2^20-row array inside the library; calls share it)."""
+    B, H, T, d = _bhtd("q", q)
+    for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _bhtd(name, t, q)
+    _side("lse", lse, (B, H, T), torch.float32)
+    _check("gpt_attn_bwd_static_ws", load().gpt_attn_bwd_static_ws(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T, d, float(scale),
         _doc_ptr(doc_offsets, B, T), _stream(stream)))
 
 

@@ -414,3 +414,66 @@ int gpt_attn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
 }
 
 }  // extern "C"
+
+// ============================================ backward without caller scratch
+// For callers that cannot allocate device memory (see gpt_attn_bwd_static_ws in
+// include/causalattn.h): the delta workspace lives in this file-scope device
+// array instead of a caller buffer.  Every GPU that loads the library holds it
+// (4 MiB) until the process exits.
+
+namespace {
+
+constexpr long kStaticWsRows = 1L << 20;  // == GPT_ATTN_STATIC_WS_MAX_ROWS
+
+static __device__ __align__(256) float g_static_delta[kStaticWsRows];
+
+std::mutex g_static_mu;
+float* g_static_delta_ptr[kMaxDevices];  // device address per device, set once
+
+// Device address of g_static_delta on the current device.  In host code the
+// symbol's name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, once per device, with that device current.
+int static_delta_ptr(float** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return GPT_ATTN_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_delta_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_delta) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return GPT_ATTN_ERR_LAUNCH;
+    }
+    g_static_delta_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_static_delta_ptr[dev];
+  return GPT_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int gpt_attn_bwd_static_ws(const void* q, const void* k, const void* v, const void* o,
+                                      const void* dout, const float* lse, void* dq, void* dk,
+                                      void* dv, int B, int H, int T, int d, float scale,
+                                      const int32_t* doc_offsets, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return GPT_ATTN_ERR_NULL_PTR;
+  int s = common_checks(B, H, T, d);
+  if (s) return s;
+  if ((int64_t)B * H * T > (int64_t)kStaticWsRows) return GPT_ATTN_ERR_TOO_LARGE;
+  if ((s = check_scale(scale))) return s;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(doc_offsets, 4))
+    return GPT_ATTN_ERR_MISALIGNED;
+  if ((s = ensure_device())) return s;
+  float* delta = nullptr;
+  if ((s = static_delta_ptr(&delta))) return s;
+  // delta is fully rewritten by the first step, so nothing needs clearing first
+  if ((s = gpt_attn_bwd_preprocess(o, dout, delta, B, H, T, d, stream))) return s;
+  if ((s = gpt_attn_bwd_dkdv(q, k, v, dout, lse, delta, dk, dv, B, H, T, d, scale, doc_offsets,
+                             stream)))
+    return s;
+  return gpt_attn_bwd_dq(q, k, v, dout, lse, delta, dq, B, H, T, d, scale, doc_offsets, stream);
+}

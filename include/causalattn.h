@@ -114,6 +114,32 @@ int gpt_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dou
                     float scale, const int32_t* doc_offsets, void* stream);
 
 /*
+ * Backward for callers that cannot allocate device memory -- code running
+ * under a framework's caching allocator that owns the whole device, inside a
+ * plugin host that lends out only its own tensors, or in a real-time loop
+ * where allocation is forbidden, so that no workspace can be created.  Same
+ * arguments and results as gpt_attn_bwd minus delta_ws: the delta workspace
+ * is a file-scope device array inside the library,
+ * GPT_ATTN_STATIC_WS_MAX_ROWS floats (4 MiB), which every GPU that loads the
+ * library holds until the process exits.  (The pages have no counterpart to
+ * this entry point; it only changes where the scratch lives.)
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - Returns GPT_ATTN_ERR_TOO_LARGE when B*H*T > GPT_ATTN_STATIC_WS_MAX_ROWS.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents
+ *     (delta is rewritten in full by every call, so nothing needs clearing):
+ *     calls whose work overlaps on the GPU -- two streams, two threads --
+ *     race on it and must be serialised by the caller.
+ */
+#define GPT_ATTN_STATIC_WS_MAX_ROWS (1L << 20)
+int gpt_attn_bwd_static_ws(const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                           int B, int H, int T, int d, float scale, const int32_t* doc_offsets,
+                           void* stream);
+
+/*
  * Checks a doc_offsets array on the device against the validity rule above.
  * Synchronises `stream`.  Returns GPT_ATTN_OK or GPT_ATTN_ERR_BAD_DOC_OFFSETS.
  */
