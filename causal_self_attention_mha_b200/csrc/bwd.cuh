@@ -62,10 +62,30 @@ struct BwdParams {
   uint64_t wait_limit_ns;
 };
 
+
+// Store 16 fp32 values (one TMEM x16 chunk of a row), times `mul`, as 16 bf16 to global.
+__device__ __forceinline__ void store16_bf16(__nv_bfloat16* dst, const uint32_t (&r)[16], float mul) {
+  uint32_t pk[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    pk[e] = pack_bf16(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+
+// Both tiled backward kernels walk the other operand in 64-row halves of its
+// 128-row tiles (N = 64 for the S / dP products).  Half g uses TMEM "set"
+// g % 2: its S (or S^T) in columns [128*set, +64) and dP (or dP^T) in
+// [128*set + 64, +64), so the MMAs of half g+1 run while the 8 element-wise
+// warps work on half g.  Element-wise warp w owns TMEM lanes 32*(w%4).. and
+// columns 32*(w/4).. of each half; it writes its bf16 P / dS (16 packed
+// columns) over the first half of the fp32 columns it has just read.
+
 // ------------------------------------------------------------------ dK/dV
 template <int D>
 struct DkdvLayout {
-  static constexpr int ST = (D == 128) ? 2 : 3;   // Q/dO ring depth
+  static constexpr int ST = (D == 128) ? 2 : 3;   // Q/dO ring depth (128-row tiles)
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + Tile<D>::BYTES;
   static constexpr int Q_OFF = V_OFF + Tile<D>::BYTES;             // + s * BYTES
@@ -73,17 +93,18 @@ struct DkdvLayout {
   static constexpr int VEC_OFF = DO_OFF + ST * Tile<D>::BYTES;     // per stage: lse2, delta, dsq
   static constexpr int VEC_STAGE = 3 * kRows * 4;
   static constexpr int BAR_OFF = VEC_OFF + ST * VEC_STAGE;
-  // barriers: kv_full | q_full[ST] | q_empty[ST] | st_full | pds_full | acc_done | drain
-  static constexpr int NBAR = 1 + 2 * ST + 4;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem slot, abort flag, q-tile range
+  // barriers: kv_full | q_full[ST] | q_empty[ST] | st_full[2] | pds_full[2] | set_free[2] | acc_done | drain
+  static constexpr int NBAR = 1 + 2 * ST + 6 + 2;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem slot, abort flag, query-tile range
   static constexpr int BYTES = MISC_OFF + 32;
   static constexpr int SMEM = BYTES + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int COMPUTE_WARPS = 8;
+  static constexpr int THREADS = (COMPUTE_WARPS + 2) * 32;
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
@@ -91,6 +112,7 @@ __global__ void __launch_bounds__(192, 1)
   using Tl = Tile<D>;
   using L = DkdvLayout<D>;
   constexpr int ST = L::ST;
+  constexpr int kProducerWarp = L::COMPUTE_WARPS, kMmaWarp = L::COMPUTE_WARPS + 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* gsm;
   const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
@@ -102,10 +124,11 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t kv_full = bar0;
   auto q_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto q_empty = [&](int s) { return bar0 + 8u * (1 + ST + s); };
-  const uint32_t st_full = bar0 + 8u * (1 + 2 * ST);
-  const uint32_t pds_full = bar0 + 8u * (2 + 2 * ST);
-  const uint32_t acc_done = bar0 + 8u * (3 + 2 * ST);
-  const uint32_t drain = bar0 + 8u * (4 + 2 * ST);
+  auto st_full = [&](int b) { return bar0 + 8u * (1 + 2 * ST + b); };
+  auto pds_full = [&](int b) { return bar0 + 8u * (3 + 2 * ST + b); };
+  auto set_free = [&](int b) { return bar0 + 8u * (5 + 2 * ST + b); };
+  const uint32_t acc_done = bar0 + 8u * (7 + 2 * ST);
+  const uint32_t drain = bar0 + 8u * (8 + 2 * ST);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
   int* range = reinterpret_cast<int*>(gsm + L::MISC_OFF + 8);
@@ -139,14 +162,17 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(q_full(s), 32);
       mbar_init(q_empty(s), 1);
     }
-    mbar_init(st_full, 1);
-    mbar_init(pds_full, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(st_full(i), 1);
+      mbar_init(pds_full(i), L::COMPUTE_WARPS);
+      mbar_init(set_free(i), 1);
+    }
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -155,11 +181,12 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int i_lo = range[0];
-  const int n = range[1] - i_lo + 1;
+  const int n = range[1] - i_lo + 1;   // query tiles
+  const int nh = 2 * n;                // query halves
   const Guard g{abort_flag, p.wait_limit_ns};
-  const uint32_t tST = tmem, tDPT = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
+  const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -181,12 +208,12 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int k = 0; k < kRows / 32; ++k) {
         const int rl = lane + 32 * k, r = r0 + rl;
-        if (r < T) {
-          lse2[rl] = p.lse[(size_t)bh * T + r] * kLog2e;
-          dl[rl] = p.delta[(size_t)bh * T + r];
+        if (r < T) {  // stored negated: -LSE*log2(e) and -delta
+          lse2[rl] = -p.lse[(size_t)bh * T + r] * kLog2e;
+          dl[rl] = -p.delta[(size_t)bh * T + r];
           dsq[rl] = p.doc ? p.doc[(size_t)b * T + r] : 0;
         } else {  // rows past the end: no key is visible
-          lse2[rl] = INFINITY;
+          lse2[rl] = -INFINITY;
           dl[rl] = 0.f;
           dsq[rl] = 0x7fffffff;
         }
@@ -207,35 +234,48 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false);  // S^T, dP^T: M = keys, N = queries
-      constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);     // dV, dK: N = d, B is MN-major
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, false);  // S^T, dP^T: M = keys, N = 64 queries
+      constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);    // dV, dK: N = d, B is MN-major
+      // dV += P^T dO and dK += dS^T Q for query half gp (K = 64 queries, 4 MMA-K steps)
+      auto issue_grad = [&](int gp) -> bool {
+        const int bp = gp & 1, sp = (gp >> 1) % ST;
+        if (!wait_bounded(pds_full(bp), (gp >> 1) & 1, g, 5)) return false;
+        tc_fence_after();
+        const uint32_t tset = tmem + 128u * bp;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tdV, tset + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sdO(sp), 4 * bp + kk), kIdG,
+                 (gp > 0 || kk > 0));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tdK, tset + 64u + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sQ(sp), 4 * bp + kk),
+                 kIdG, (gp > 0 || kk > 0));
+        tc_commit(set_free(bp));
+        if (bp == 1) tc_commit(q_empty(sp));
+        return true;
+      };
       bool ok = wait_bounded(kv_full, 0, g, 2);
-      for (int it = 0; ok && it < n; ++it) {
-        const int s = it % ST;
-        if (!wait_bounded(q_full(s), (it / ST) & 1, g, 3)) break;
-        // S^T / dP^T overwrite the P^T / dS^T that the previous dV / dK MMAs read
-        if (it > 0 && !wait_bounded(q_empty((it - 1) % ST), ((it - 1) / ST) & 1, g, 4)) break;
+      for (int gh = 0; ok && gh < nh; ++gh) {
+        const int it = gh >> 1, h = gh & 1, s = it % ST;
+        if (h == 0 && !wait_bounded(q_full(s), (it / ST) & 1, g, 3)) break;
+        // set h is reused: the dV / dK MMAs of half gh-2 must have finished reading it
+        if (gh >= 2 && !wait_bounded(set_free(h), ((gh - 2) >> 1) & 1, g, 4)) break;
         tc_fence_after();
+        const uint32_t tset = tmem + 128u * h;
+        const uint32_t off = (uint32_t)(64 * h * Tl::SW);  // query rows 64h.. of the stage tile
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tST, desc_k<D>(sK, kk), desc_k<D>(sQ(s), kk), kIdS, kk > 0);
+          mma_ss(tset, desc_k<D>(sK, kk), desc_k<D>(sQ(s) + off, kk), kIdS, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tDPT, desc_k<D>(sV, kk), desc_k<D>(sdO(s), kk), kIdS, kk > 0);
-        tc_commit(st_full);
-        if (!wait_bounded(pds_full, it & 1, g, 5)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)
-          mma_ts(tdV, tST + 8u * kk, desc_mn<D>(sdO(s), kk), kIdG, (it > 0 || kk > 0));
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)
-          mma_ts(tdK, tDPT + 8u * kk, desc_mn<D>(sQ(s), kk), kIdG, (it > 0 || kk > 0));
-        tc_commit(q_empty(s));
+          mma_ss(tset + 64u, desc_k<D>(sV, kk), desc_k<D>(sdO(s) + off, kk), kIdS, kk > 0);
+        tc_commit(st_full(h));
+        if (gh >= 1 && !issue_grad(gh - 1)) { ok = false; break; }
       }
+      if (ok) issue_grad(nh - 1);
       tc_commit(acc_done);
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
@@ -243,80 +283,91 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ------------------------------------------- P^T / dS^T (thread = key row)
-    const int t = threadIdx.x;
-    const int c = k0 + t;  // key position owned by this thread
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int qd = warp & 3, cs = warp >> 2;
+    const int c = k0 + qd * 32 + lane;  // key position owned by this thread
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2(sl2, sl2);
     bool ok = true;
-    for (int it = 0; it < n; ++it) {
-      const int s = it % ST;
-      const int i = i_lo + it;
-      const int r0 = i * kRows;
-      if (!wait_bounded_warp(st_full, it & 1, g, 6)) { ok = false; break; }
+    for (int gh = 0; gh < nh; ++gh) {
+      const int it = gh >> 1, h = gh & 1, s = it % ST;
+      if (!wait_bounded_warp(st_full(h), (gh >> 1) & 1, g, 6)) { ok = false; break; }
       if (!wait_bounded_warp(q_full(s), (it / ST) & 1, g, 7)) { ok = false; break; }
       tc_fence_after();
       const float* lse2 = vec + s * 3 * kRows;
       const float* dl = lse2 + kRows;
       const int* dsq = reinterpret_cast<const int*>(dl + kRows);
-      // no mask needed when every query row of the tile is strictly below this key
-      // and its document starts at or before it
-      const bool full = (i > jt) && (dsq[kRows - 1] <= c);
+      const int rb = 64 * h + 32 * cs;           // first query row (within the tile) of my columns
+      const int r0 = (i_lo + it) * kRows + rb;   // its position
+      const uint32_t tS = tmem + lane_off + 128u * h + 32u * cs;
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tS, sr);
+      tmem_ld32(tS + 64u, dr);
+      tc_wait_ld();
+      reg_fence(sr);
+      reg_fence(dr);
+      // no mask needed when all my query rows are at or below this key and their
+      // documents start at or before it (dsq is nondecreasing; huge past T)
+      if (!((r0 >= c) && (dsq[rb + 31] <= c))) {
+        const int4* ds4 = reinterpret_cast<const int4*>(dsq + rb);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tST + lane_off + 32u * cc, sr);
-        tmem_ld32(tDPT + lane_off + 32u * cc, dr);
-        tc_wait_ld();
-        reg_fence(sr);
-        reg_fence(dr);
-        uint32_t pk[16], dk[16];
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const int4 dv4 = ds4[q4];
+          const int dsv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int rl = 32 * cc + 2 * e + h;
-            float pr = ex2(__uint_as_float(sr[2 * e + h]) * sl2 - lse2[rl]);
-            if (!full) {
-              const int r = r0 + rl;
-              if (c > r || c < dsq[rl]) pr = 0.f;
-            }
-            pv[h] = pr;
-            dv[h] = pr * (__uint_as_float(dr[2 * e + h]) - dl[rl]);
+          for (int k = 0; k < 4; ++k) {
+            const int e = 4 * q4 + k;
+            if (c > r0 + e || c < dsv[k]) sr[e] = 0xFF800000u;  // -inf: weight 0
           }
-          pk[e] = pack_bf16(pv[0], pv[1]);
-          dk[e] = pack_bf16(dv[0], dv[1]);
         }
-        tmem_st16(tST + lane_off + 16u * cc, pk);
-        tmem_st16(tDPT + lane_off + 16u * cc, dk);
       }
+      const float4* l4 = reinterpret_cast<const float4*>(lse2 + rb);  // -LSE*log2(e)
+      const float4* d4 = reinterpret_cast<const float4*>(dl + rb);    // -delta
+      uint32_t pk[16], dk[16];
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 lv = l4[q4], dv4 = d4[q4];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int e = 4 * q4 + 2 * h2;
+          const uint64_t nl = h2 ? f2(lv.z, lv.w) : f2(lv.x, lv.y);
+          const uint64_t nd = h2 ? f2(dv4.z, dv4.w) : f2(dv4.x, dv4.y);
+          // P^T = exp2(S^T * scale * log2e - LSE * log2e);  dS^T = P^T * (dP^T - delta)
+          const float2 x = f2split(ffma2(f2u(sr[e], sr[e + 1]), sl2x2, nl));
+          const float p0 = ex2(x.x), p1 = ex2(x.y);
+          const float2 dd = f2split(fmul2(f2(p0, p1), fadd2(f2u(dr[e], dr[e + 1]), nd)));
+          pk[e >> 1] = pack_bf16(p0, p1);
+          dk[e >> 1] = pack_bf16(dd.x, dd.y);
+        }
+      }
+      tmem_st16(tS, pk);
+      tmem_st16(tS + 64u, dk);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(pds_full);
+      if (lane == 0) mbar_arrive(pds_full(h));
     }
     if (ok && wait_bounded_warp(acc_done, 0, g, 8)) {
       tc_fence_after();
       __nv_bfloat16* dk_row = p.g0 + ((size_t)bh * T + c) * D;
       __nv_bfloat16* dv_row = p.g1 + ((size_t)bh * T + c) * D;
+      // 16-column jobs over (dV, dK), split between the two warps that share these lanes
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tdV + lane_off + 32u * cc, r);
+      for (int j = cs; j < 2 * (D / 16); j += 2) {
+        const bool is_k = j >= D / 16;
+        const int col = 16 * (is_k ? j - D / 16 : j);
+        uint32_t r[16];
+        tmem_ld16((is_k ? tdK : tdV) + lane_off + col, r);
         tc_wait_ld();
-        reg_fence(r);
-        if (c < T) store_row_chunk_bf16(dv_row + 32 * cc, r, 1.0f);
-        tmem_ld32(tdK + lane_off + 32u * cc, r);
-        tc_wait_ld();
-        reg_fence(r);
-        if (c < T) store_row_chunk_bf16(dk_row + 32 * cc, r, p.scale);
+        reg_fence16(r);
+        if (c < T) store16_bf16((is_k ? dk_row : dv_row) + col, r, is_k ? p.scale : 1.0f);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
@@ -325,29 +376,31 @@ __global__ void __launch_bounds__(192, 1)
 // --------------------------------------------------------------------- dQ
 template <int D>
 struct DqLayout {
-  static constexpr int ST = (D == 128) ? 2 : 3;   // K/V ring depth
+  static constexpr int ST = (D == 128) ? 2 : 3;   // K/V ring depth (128-row tiles)
   static constexpr int Q_OFF = 0;
   static constexpr int DO_OFF = Q_OFF + Tile<D>::BYTES;
   static constexpr int K_OFF = DO_OFF + Tile<D>::BYTES;           // + s * BYTES
   static constexpr int V_OFF = K_OFF + ST * Tile<D>::BYTES;       // + s * BYTES
   static constexpr int BAR_OFF = V_OFF + ST * Tile<D>::BYTES;
-  // barriers: qdo_full | kv_full[ST] | kv_empty[ST] | s_full | ds_full | acc_done | drain
-  static constexpr int NBAR = 1 + 2 * ST + 4;
+  // barriers: qdo_full | kv_full[ST] | kv_empty[ST] | s_full[2] | ds_full[2] | set_free[2] | acc_done | drain
+  static constexpr int NBAR = 1 + 2 * ST + 6 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int COMPUTE_WARPS = 8;
+  static constexpr int THREADS = (COMPUTE_WARPS + 2) * 32;
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmdO, const BwdParams p) {
   using Tl = Tile<D>;
   using L = DqLayout<D>;
   constexpr int ST = L::ST;
+  constexpr int kProducerWarp = L::COMPUTE_WARPS, kMmaWarp = L::COMPUTE_WARPS + 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* gsm;
   const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
@@ -358,10 +411,11 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t qdo_full = bar0;
   auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
   auto kv_empty = [&](int s) { return bar0 + 8u * (1 + ST + s); };
-  const uint32_t s_full = bar0 + 8u * (1 + 2 * ST);
-  const uint32_t ds_full = bar0 + 8u * (2 + 2 * ST);
-  const uint32_t acc_done = bar0 + 8u * (3 + 2 * ST);
-  const uint32_t drain = bar0 + 8u * (4 + 2 * ST);
+  auto s_full = [&](int b) { return bar0 + 8u * (1 + 2 * ST + b); };
+  auto ds_full = [&](int b) { return bar0 + 8u * (3 + 2 * ST + b); };
+  auto set_free = [&](int b) { return bar0 + 8u * (5 + 2 * ST + b); };
+  const uint32_t acc_done = bar0 + 8u * (7 + 2 * ST);
+  const uint32_t drain = bar0 + 8u * (8 + 2 * ST);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -376,7 +430,8 @@ __global__ void __launch_bounds__(192, 1)
     kv_lo = p.doc[(size_t)b * T + q0] / kRows;
     kv_lo = kv_lo < 0 ? 0 : (kv_lo > qt ? qt : kv_lo);
   }
-  const int n = qt - kv_lo + 1;
+  const int n = qt - kv_lo + 1;   // key tiles
+  const int nh = 2 * n;           // key halves
 
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
@@ -384,14 +439,17 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(ds_full, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full(i), 1);
+      mbar_init(ds_full(i), L::COMPUTE_WARPS);
+      mbar_init(set_free(i), 1);
+    }
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -400,9 +458,9 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, p.wait_limit_ns};
-  const uint32_t tS = tmem, tDP = tmem + 128, tdQ = tmem + 256;
+  const uint32_t tdQ = tmem + 256;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -429,97 +487,108 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, false);  // S, dP: M = queries, N = 64 keys
+      constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);    // dQ: N = d, B (K) is MN-major
+      auto issue_grad = [&](int gp) -> bool {
+        const int bp = gp & 1, sp = (gp >> 1) % ST;
+        if (!wait_bounded(ds_full(bp), (gp >> 1) & 1, g, 5)) return false;
+        tc_fence_after();
+        const uint32_t tset = tmem + 128u * bp;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tdQ, tset + 64u + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sK(sp), 4 * bp + kk),
+                 kIdG, (gp > 0 || kk > 0));
+        tc_commit(set_free(bp));
+        if (bp == 1) tc_commit(kv_empty(sp));
+        return true;
+      };
       bool ok = wait_bounded(qdo_full, 0, g, 2);
-      for (int it = 0; ok && it < n; ++it) {
-        const int s = it % ST;
-        if (!wait_bounded(kv_full(s), (it / ST) & 1, g, 3)) break;
-        // S / dP overwrite the dS that the previous dQ MMA read
-        if (it > 0 && !wait_bounded(kv_empty((it - 1) % ST), ((it - 1) / ST) & 1, g, 4)) break;
+      for (int gh = 0; ok && gh < nh; ++gh) {
+        const int it = gh >> 1, h = gh & 1, s = it % ST;
+        if (h == 0 && !wait_bounded(kv_full(s), (it / ST) & 1, g, 3)) break;
+        // set h is reused: the dQ MMAs of half gh-2 must have finished reading it
+        if (gh >= 2 && !wait_bounded(set_free(h), ((gh - 2) >> 1) & 1, g, 4)) break;
         tc_fence_after();
+        const uint32_t tset = tmem + 128u * h;
+        const uint32_t off = (uint32_t)(64 * h * Tl::SW);  // key rows 64h.. of the stage tile
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tS, desc_k<D>(sQ, kk), desc_k<D>(sK(s), kk), kIdS, kk > 0);
+          mma_ss(tset, desc_k<D>(sQ, kk), desc_k<D>(sK(s) + off, kk), kIdS, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tDP, desc_k<D>(sdO, kk), desc_k<D>(sV(s), kk), kIdS, kk > 0);
-        tc_commit(s_full);
-        if (!wait_bounded(ds_full, it & 1, g, 5)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)
-          mma_ts(tdQ, tDP + 8u * kk, desc_mn<D>(sK(s), kk), kIdG, (it > 0 || kk > 0));
-        tc_commit(kv_empty(s));
+          mma_ss(tset + 64u, desc_k<D>(sdO, kk), desc_k<D>(sV(s) + off, kk), kIdS, kk > 0);
+        tc_commit(s_full(h));
+        if (gh >= 1 && !issue_grad(gh - 1)) { ok = false; break; }
       }
+      if (ok) issue_grad(nh - 1);
       tc_commit(acc_done);
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
     }
     __syncwarp();
   } else {
-    const int t = threadIdx.x;
-    const int r = q0 + t;  // query position owned by this thread
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int qd = warp & 3, cs = warp >> 2;
+    const int r = q0 + qd * 32 + lane;  // query position owned by this thread
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const float sl2 = p.scale_log2;
-    const float lse2 = (r < T) ? p.lse[(size_t)bh * T + r] * kLog2e : INFINITY;
-    const float dlt = (r < T) ? p.delta[(size_t)bh * T + r] : 0.f;
+    // rows past T: -LSE = -inf makes every weight zero
+    const float nlse2 = (r < T) ? -p.lse[(size_t)bh * T + r] * kLog2e : -INFINITY;
+    const float ndlt = (r < T) ? -p.delta[(size_t)bh * T + r] : 0.f;
     const int ds = p.doc ? p.doc[(size_t)b * T + (r < T ? r : T - 1)] : 0;
+    const uint64_t sl2x2 = f2(sl2, sl2), nlse2x2 = f2(nlse2, nlse2), ndltx2 = f2(ndlt, ndlt);
     bool ok = true;
-    for (int it = 0; it < n; ++it) {
-      const int j = kv_lo + it;
-      if (!wait_bounded_warp(s_full, it & 1, g, 6)) { ok = false; break; }
+    for (int gh = 0; gh < nh; ++gh) {
+      const int it = gh >> 1, h = gh & 1;
+      if (!wait_bounded_warp(s_full(h), (gh >> 1) & 1, g, 6)) { ok = false; break; }
       tc_fence_after();
-      const bool full = (j < qt) && (j * kRows >= ds);
+      const int c0 = (kv_lo + it) * kRows + 64 * h + 32 * cs;  // first key of my columns
+      const uint32_t tS = tmem + lane_off + 128u * h + 32u * cs;
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tS, sr);
+      tmem_ld32(tS + 64u, dr);
+      tc_wait_ld();
+      reg_fence(sr);
+      reg_fence(dr);
+      if (!((c0 + 31 <= r) && (c0 >= ds))) {
+        const int hi = r - c0, lo = ds - c0;  // visible keys: e in [lo, hi]
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tS + lane_off + 32u * cc, sr);
-        tmem_ld32(tDP + lane_off + 32u * cc, dr);
-        tc_wait_ld();
-        reg_fence(sr);
-        reg_fence(dr);
-        uint32_t dk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float dv[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float pr = ex2(__uint_as_float(sr[2 * e + h]) * sl2 - lse2);
-            if (!full) {
-              const int col = j * kRows + 32 * cc + 2 * e + h;
-              if (col > r || col < ds) pr = 0.f;
-            }
-            dv[h] = pr * (__uint_as_float(dr[2 * e + h]) - dlt);
-          }
-          dk[e] = pack_bf16(dv[0], dv[1]);
-        }
-        tmem_st16(tDP + lane_off + 16u * cc, dk);
+        for (int e = 0; e < 32; ++e)
+          if (e > hi || e < lo) sr[e] = 0xFF800000u;  // -inf: weight 0
       }
+      uint32_t dk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        // P = exp2(S * scale * log2e - LSE * log2e);  dS = P * (dP - delta)
+        const float2 x = f2split(ffma2(f2u(sr[2 * e], sr[2 * e + 1]), sl2x2, nlse2x2));
+        const uint64_t p2 = f2(ex2(x.x), ex2(x.y));
+        const float2 d = f2split(fmul2(p2, fadd2(f2u(dr[2 * e], dr[2 * e + 1]), ndltx2)));
+        dk[e] = pack_bf16(d.x, d.y);
+      }
+      tmem_st16(tS + 64u, dk);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
+      if (lane == 0) mbar_arrive(ds_full(h));
     }
     if (ok && wait_bounded_warp(acc_done, 0, g, 8)) {
       tc_fence_after();
       __nv_bfloat16* dq_row = p.g0 + ((size_t)bh * T + r) * D;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tdQ + lane_off + 32u * cc, v);
+      for (int j = cs; j < D / 16; j += 2) {
+        uint32_t v[16];
+        tmem_ld16(tdQ + lane_off + 16u * j, v);
         tc_wait_ld();
-        reg_fence(v);
-        if (r < T) store_row_chunk_bf16(dq_row + 32 * cc, v, p.scale);
+        reg_fence16(v);
+        if (r < T) store16_bf16(dq_row + 16 * j, v, p.scale);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
