@@ -50,6 +50,7 @@ SIGNATURES = {
     "gpt_attn_selftest_wait_timeout": ([ctypes.c_uint64, _vp], _i),
     "gpt_attn_strerror": ([_i], ctypes.c_char_p),
     "gpt_attn_version": ([], _i),
+    "gpt_attn_last_cuda_error": ([], ctypes.c_char_p),
 }
 
 _lib = None
@@ -58,7 +59,13 @@ _lib = None
 class AttnError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: status {status} ({strerror(status)})")
+        detail = ""
+        if status == GPT_ATTN_ERR_LAUNCH:
+            try:
+                detail = ": " + load().gpt_attn_last_cuda_error().decode()
+            except Exception:
+                pass
+        super().__init__(f"{fn} failed: status {status} ({strerror(status)}{detail})")
 
 
 def load(path: Optional[str] = None) -> ctypes.CDLL:

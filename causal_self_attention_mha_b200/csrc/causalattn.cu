@@ -40,6 +40,7 @@ int check_scale(float scale) {
 // ----------------------------------------------------------- device setup
 std::mutex g_mu;
 std::atomic<int> g_dev_state[kMaxDevices];  // 0 unknown, 1 ready, 2 wrong arch, 3 setup failed
+int g_sm_count[kMaxDevices];                // multiprocessors per device (persistent grids)
 
 template <int D>
 cudaError_t set_smem_attrs() {
@@ -76,6 +77,9 @@ int ensure_device() {
         cudaGetLastError();
         return GPT_ATTN_ERR_NO_DEVICE;
       }
+      int sms = 0;
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      g_sm_count[dev] = sms > 0 ? sms : 148;
       if (major != 10 || minor != 0) {
         st = 2;
       } else if (set_smem_attrs<32>() != cudaSuccess || set_smem_attrs<64>() != cudaSuccess ||
@@ -133,9 +137,19 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int T) {
   return r == CUDA_SUCCESS;
 }
 
+int sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return (dev >= 0 && dev < kMaxDevices && g_sm_count[dev] > 0) ? g_sm_count[dev] : 148;
+}
+
+thread_local const char* t_last_cuda_error = "no error";
+
 int launch_status() {
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? GPT_ATTN_OK : GPT_ATTN_ERR_LAUNCH;
+  if (e == cudaSuccess) return GPT_ATTN_OK;
+  t_last_cuda_error = cudaGetErrorString(e);
+  return GPT_ATTN_ERR_LAUNCH;
 }
 
 // ------------------------------------------------------------- launchers
@@ -154,9 +168,13 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.T = T;
   p.BH = BH;
   p.n_qt = (T + ca::kRows - 1) / ca::kRows;
+  p.n_pairs = (p.n_qt + 1) / 2;
+  p.n_items = p.n_pairs * BH;
   p.scale_log2 = scale * ca::kLog2e;
   p.wait_limit_ns = kWaitLimitNs;
-  const unsigned grid = (unsigned)p.n_qt * (unsigned)BH;
+  // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int sms = sm_count();
+  const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
   ca::attn_fwd_kernel<D><<<grid, ca::FwdLayout<D>::THREADS, ca::FwdLayout<D>::SMEM, st>>>(mq, mk,
                                                                                          mv, p);
   return launch_status();
@@ -241,6 +259,8 @@ int common_checks(int B, int H, int T, int d) { return check_shape(B, H, T, d); 
 extern "C" {
 
 int gpt_attn_version(void) { return GPT_ATTN_ABI_VERSION; }
+
+const char* gpt_attn_last_cuda_error(void) { return t_last_cuda_error; }
 
 const char* gpt_attn_strerror(int s) {
   switch (s) {

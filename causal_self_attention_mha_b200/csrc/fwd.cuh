@@ -1,6 +1,6 @@
 // fwd.cuh -- causal attention forward on sm_100a.
 //
-// Computes, for one head and one 128-row query tile per CTA,
+// Computes, for every head and 128-row query tile,
 //   S = scale * Q K^T  (upper triangle and other documents masked to -inf),
 //   P = softmax(S) row-wise,  O = P V,  LSE = log sum exp(S)  (natural log)
 // as in "Stanford CS336 walkthrough" (lmnt.cn), section 5.1 model.py,
@@ -8,24 +8,33 @@
 // the softmax).  The softmax is evaluated online over 128-column key tiles
 // (running max m and sums, in base 2), so the T x T matrix never exists.
 //
-// Warp roles (320 threads):
-//   warps 0-7  softmax.  Warp w owns TMEM lanes 32*(w%4).. (32 query rows) and
-//              key half kh = w/4 of every key tile (64 keys).  Each half keeps
-//              its own running max, sums and O accumulator, so a row is never
-//              exchanged between threads inside the loop; the two halves are
-//              merged once, in the epilogue.
-//   warp 8     TMA producer: Q once, then K/V tiles through an ST-stage ring
-//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
-// TMEM (512 columns): S double buffer at columns 0 and 128 (each key half's P,
-// as packed bf16, overwrites the first 32 of its own 64 S columns); O for key
-// half 0 at column 256, for key half 1 at 256 + D.
+// Persistent kernel: one CTA per SM walks work items w = blockIdx.x,
+// blockIdx.x + gridDim.x, ...  An item is a PAIR of adjacent 128-row query
+// tiles (A = 2m, B = 2m+1) of one head, so every K/V tile brought on chip
+// serves 256 query rows.  Items are numbered heaviest first.  All roles walk
+// the same item / key-tile sequence; the K/V rings run on across items.
 //
-// Per key tile j the MMA issuer runs S_{j+1} = Q K_{j+1}^T while the softmax
-// warps turn S_j into P_j; then O_h += P_j,h V_j,h for both halves, with P read
-// straight from TMEM.  O_h is rescaled in TMEM only when its row max grows by
-// more than 2^8.  Normalisation uses the sum of the bf16-rounded weights the
-// MMA actually multiplied (the weights of each output row sum to one); the LSE
-// uses the sum of the fp32 weights.
+// Warp roles (384 threads = three warpgroups):
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: one thread per
+//              query row (= TMEM lane), so row max and sums are in-thread
+//   warp 8     TMA producer: lane 0 loads Q_A, Q_B and the K ring, lane 1 the V ring
+//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 idle
+// Registers: launched at 168 per thread; the third warpgroup drops to 88 and
+// the two softmax warpgroups rise to 208 (2*128*208 + 128*88 = 384*168), room
+// for a whole 128-column row of S in registers.
+// TMEM (512 columns): S_A at 0, S_B at 128 (P, packed bf16, overwrites the
+// first 64 columns of its own S), O_A at 256, O_B at 256 + D.
+//
+// MMA order per key tile j: PV_A(j-1), S_A(j), PV_B(j-1), S_B(j).  Each tile's
+// chain alternates softmax and MMA; the two chains run half a period apart,
+// so the tensor pipe works on one tile while the other tile's softmax runs.
+// S_X(j) overwrites P_X(j-1) only after PV_X(j-1) in the same in-order MMA
+// stream.  A K slot is released once both S MMAs that read it are done, a V
+// slot after its last PV.  O_X is rescaled in TMEM only when a row max grows
+// by more than 2^8.  Normalisation uses the sum of the bf16-rounded weights
+// the MMA actually multiplied (the weights of each output row sum to one);
+// the LSE uses the sum of the fp32 weights.
 #pragma once
 
 #include "tiles.cuh"
@@ -36,80 +45,112 @@ struct FwdParams {
   const int32_t* doc;     // [B, T] document start of each position, or nullptr
   __nv_bfloat16* o;       // [B, H, T, D]
   float* lse;             // [B, H, T]
-  int H, T, BH, n_qt;
+  int H, T, BH, n_qt, n_pairs, n_items;
   float scale_log2;       // scale * log2(e)
   uint64_t wait_limit_ns;
 };
 
 template <int D>
 struct FwdLayout {
-  static constexpr int ST = (D == 128) ? 2 : 3;             // K/V ring depth
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + Tile<D>::BYTES;
-  static constexpr int V_OFF = K_OFF + ST * Tile<D>::BYTES;
-  static constexpr int RED_OFF = V_OFF + ST * Tile<D>::BYTES;  // [2 halves][3][128] floats
-  static constexpr int BAR_OFF = RED_OFF + 2 * 3 * kRows * 4;
-  // barriers: q_full | k_full[ST] | v_full[ST] | kv_empty[ST] | s_full[2] | p_full[2] | o_done | drain
-  static constexpr int NBAR = 1 + 3 * ST + 2 + 2 + 2;
+  static constexpr int STK = (D == 128) ? 2 : 4;            // K ring depth
+  static constexpr int STV = (D == 128) ? 2 : 3;            // V ring depth
+  static constexpr int Q_OFF = 0;                            // Q_A, Q_B
+  static constexpr int K_OFF = Q_OFF + 2 * Tile<D>::BYTES;
+  static constexpr int V_OFF = K_OFF + STK * Tile<D>::BYTES;
+  static constexpr int BAR_OFF = V_OFF + STV * Tile<D>::BYTES;
+  // barriers: q_full[2] q_empty[2] k_full[STK] k_empty[STK] v_full[STV] v_empty[STV]
+  //           s_full[2] p_full[2] o_done[2] o_free[2] drain
+  static constexpr int NBAR = 4 + 2 * STK + 2 * STV + 8 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;       // tmem base slot, abort flag
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;                  // + alignment slack
   static constexpr int SOFTMAX_WARPS = 8;
-  static constexpr int THREADS = (SOFTMAX_WARPS + 2) * 32;
+  static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
+// One work item: query tiles A = 2*pm and B = 2*pm + 1 of head bh.
+struct FwdItem {
+  int bh, b;
+  int qt[2];       // query tile of A and B
+  bool hasB;       // B lies (at least partly) inside T
+  int j_lo, j_hi;  // key tiles streamed for the pair
+  int lo[2];       // first key tile each of A / B needs (A: j_lo; B: >= j_lo)
+  int hi[2];       // last key tile each needs (its diagonal)
+};
+
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
+  FwdItem I;
+  const int pm = p.n_pairs - 1 - w / p.BH;  // heaviest pairs first
+  I.bh = w % p.BH;
+  I.b = I.bh / p.H;
+  I.qt[0] = 2 * pm;
+  I.qt[1] = 2 * pm + 1;
+  I.hasB = I.qt[1] < p.n_qt;
+  for (int x = 0; x < 2; ++x) {
+    int lo = 0;
+    if (p.doc && (x == 0 || I.hasB)) {
+      lo = p.doc[(size_t)I.b * p.T + I.qt[x] * kRows] / kRows;
+      lo = lo < 0 ? 0 : (lo > I.qt[x] ? I.qt[x] : lo);
+    }
+    I.lo[x] = lo;
+    I.hi[x] = I.qt[x];
+  }
+  if (I.lo[1] < I.lo[0]) I.lo[1] = I.lo[0];
+  I.j_lo = I.lo[0];
+  I.j_hi = I.hasB ? I.hi[1] : I.hi[0];
+  return I;
+}
+
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using Tl = Tile<D>;
   using L = FwdLayout<D>;
-  constexpr int ST = L::ST;
+  constexpr int STK = L::STK, STV = L::STV;
   constexpr int kProducerWarp = L::SOFTMAX_WARPS, kMmaWarp = L::SOFTMAX_WARPS + 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* gsm;
   const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
   const uint32_t sQ = sbase + L::Q_OFF, sK = sbase + L::K_OFF, sV = sbase + L::V_OFF;
-  float* red = reinterpret_cast<float*>(gsm + L::RED_OFF);
   const uint32_t bar0 = sbase + L::BAR_OFF;
-  const uint32_t q_full = bar0;
-  auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto v_full = [&](int s) { return bar0 + 8u * (1 + ST + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + 2 * ST + s); };
-  auto s_full = [&](int b) { return bar0 + 8u * (1 + 3 * ST + b); };
-  auto p_full = [&](int b) { return bar0 + 8u * (3 + 3 * ST + b); };
-  const uint32_t o_done = bar0 + 8u * (5 + 3 * ST);
-  const uint32_t drain = bar0 + 8u * (6 + 3 * ST);
+  auto q_full = [&](int x) { return bar0 + 8u * x; };
+  auto q_empty = [&](int x) { return bar0 + 8u * (2 + x); };
+  auto k_full = [&](int s) { return bar0 + 8u * (4 + s); };
+  auto k_empty = [&](int s) { return bar0 + 8u * (4 + STK + s); };
+  auto v_full = [&](int s) { return bar0 + 8u * (4 + 2 * STK + s); };
+  auto v_empty = [&](int s) { return bar0 + 8u * (4 + 2 * STK + STV + s); };
+  const uint32_t xb = bar0 + 8u * (4 + 2 * STK + 2 * STV);
+  auto s_full = [&](int x) { return xb + 8u * x; };
+  auto p_full = [&](int x) { return xb + 8u * (2 + x); };
+  auto o_done = [&](int x) { return xb + 8u * (4 + x); };
+  auto o_free = [&](int x) { return xb + 8u * (6 + x); };
+  const uint32_t drain = xb + 8u * 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.T;
-  // Work item: heaviest query tiles (most key tiles) are launched first.
-  const int qt = p.n_qt - 1 - (int)(blockIdx.x / p.BH);
-  const int bh = (int)(blockIdx.x % p.BH);
-  const int b = bh / p.H;
-  const int q0 = qt * kRows;
-  int kv_lo = 0;
-  if (p.doc) {
-    kv_lo = p.doc[(size_t)b * T + q0] / kRows;
-    kv_lo = kv_lo < 0 ? 0 : (kv_lo > qt ? qt : kv_lo);
-  }
-  const int n = qt - kv_lo + 1;  // key tiles to visit (>= 1)
+  const int w0 = blockIdx.x, dw = gridDim.x;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < ST; ++s) {
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(q_full(x), 1);
+      mbar_init(q_empty(x), 1);
+      mbar_init(s_full(x), 1);
+      mbar_init(p_full(x), 4);
+      mbar_init(o_done(x), 1);
+      mbar_init(o_free(x), 4);
+    }
+    for (int s = 0; s < STK; ++s) {
       mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+    }
+    for (int s = 0; s < STV; ++s) {
       mbar_init(v_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(v_empty(s), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full(i), 1);
-      mbar_init(p_full(i), L::SOFTMAX_WARPS);
-    }
-    mbar_init(o_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -123,33 +164,60 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, p.wait_limit_ns};
-
+  if (warp >= L::SOFTMAX_WARPS) {
+    // third warpgroup: give registers to the softmax warpgroups, then specialise
+    regs_shrink<88>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0) {  // Q_A, Q_B and the K ring
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, Tl::BYTES);
-      load_tile<D>(sQ, &tmQ, q0, bh, q_full);
-      int it = 0;
-      for (; it < n; ++it) {
-        const int s = it % ST, u = it / ST;
-        if (u > 0 && !wait_bounded(kv_empty(s), (u - 1) & 1, g, 1)) break;
-        const int row = (kv_lo + it) * kRows;
-        mbar_arrive_expect_tx(k_full(s), Tl::BYTES);
-        load_tile<D>(sK + s * Tl::BYTES, &tmK, row, bh, k_full(s));
-        mbar_arrive_expect_tx(v_full(s), Tl::BYTES);
-        load_tile<D>(sV + s * Tl::BYTES, &tmV, row, bh, v_full(s));
+      int nq[2] = {0, 0};  // Q loads issued into buffer A / B
+      int gk = 0;          // K loads issued
+      bool ok = true;
+      for (int w = w0; ok && w < p.n_items; w += dw) {
+        const FwdItem I = fwd_item(p, w);
+        for (int x = 0; x < 2; ++x) {
+          if (x == 1 && !I.hasB) continue;
+          if (nq[x] >= 1 && !wait_bounded(q_empty(x), (nq[x] - 1) & 1, g, 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(q_full(x), Tl::BYTES);
+          load_tile<D>(sQ + x * Tl::BYTES, &tmQ, I.qt[x] * kRows, I.bh, q_full(x));
+          ++nq[x];
+        }
+        for (int j = I.j_lo; ok && j <= I.j_hi; ++j) {
+          const int s = gk % STK, u = gk / STK;
+          if (u > 0 && !wait_bounded(k_empty(s), (u - 1) & 1, g, 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(k_full(s), Tl::BYTES);
+          load_tile<D>(sK + s * Tl::BYTES, &tmK, j * kRows, I.bh, k_full(s));
+          ++gk;
+        }
       }
       if (*abort_flag) {  // let every copy already issued land before the CTA exits
-        drain_wait(q_full, 0, p.wait_limit_ns);
-        for (int s = 0; s < ST; ++s) {
-          const int cnt = it > s ? (it - s + ST - 1) / ST : 0;
-          if (cnt > 0) {
-            drain_wait(k_full(s), (cnt - 1) & 1, p.wait_limit_ns);
-            drain_wait(v_full(s), (cnt - 1) & 1, p.wait_limit_ns);
-          }
+        for (int x = 0; x < 2; ++x)
+          if (nq[x] > 0) drain_wait(q_full(x), (nq[x] - 1) & 1, p.wait_limit_ns);
+        for (int s = 0; s < STK; ++s) {
+          const int cnt = gk > s ? (gk - s + STK - 1) / STK : 0;
+          if (cnt > 0) drain_wait(k_full(s), (cnt - 1) & 1, p.wait_limit_ns);
+        }
+      }
+    } else if (lane == 1) {  // the V ring
+      tma_prefetch_desc(&tmV);
+      int gv = 0;
+      bool ok = true;
+      for (int w = w0; ok && w < p.n_items; w += dw) {
+        const FwdItem I = fwd_item(p, w);
+        for (int j = I.j_lo; j <= I.j_hi; ++j) {
+          const int s = gv % STV, u = gv / STV;
+          if (u > 0 && !wait_bounded(v_empty(s), (u - 1) & 1, g, 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(v_full(s), Tl::BYTES);
+          load_tile<D>(sV + s * Tl::BYTES, &tmV, j * kRows, I.bh, v_full(s));
+          ++gv;
+        }
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < STV; ++s) {
+          const int cnt = gv > s ? (gv - s + STV - 1) / STV : 0;
+          if (cnt > 0) drain_wait(v_full(s), (cnt - 1) & 1, p.wait_limit_ns);
         }
       }
     }
@@ -159,194 +227,200 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t kIdO = idesc_bf16_f32(128, D, true);
-      auto issue_s = [&](int it) -> bool {
-        const int s = it % ST;
-        if (!wait_bounded(k_full(s), (it / ST) & 1, g, 3)) return false;
+      int nq[2] = {0, 0};   // items started per query tile slot (q_full phases)
+      int tx[2] = {0, 0};   // S MMAs issued per slot (s_full / p_full / o_done phases)
+      int gk = 0, gv = 0;   // key tiles consumed from the K / V rings
+      bool ok = true;
+      // pending PV of slot x: its global tile index, V slot, "first of item", "last user of V"
+      int pend_t[2] = {-1, -1}, pend_v[2] = {0, 0};
+      bool pend_first[2] = {false, false}, pend_rel[2] = {false, false};
+      auto issue_pv = [&](int x) -> bool {
+        const int tp = pend_t[x];
+        if (pend_first[x] && nq[x] >= 2 && !wait_bounded(o_free(x), (nq[x] - 2) & 1, g, 4))
+          return false;  // the previous item's epilogue must have read O_x
+        if (!wait_bounded(p_full(x), tp & 1, g, 5)) return false;
+        const int sv = pend_v[x] % STV;
+        if (!wait_bounded(v_full(sv), (pend_v[x] / STV) & 1, g, 6)) return false;
         tc_fence_after();
-        const uint32_t tS = tmem + 128u * (it & 1);
+        const uint32_t sVs = sV + sv * Tl::BYTES;
+        const uint32_t tP = tmem + 128u * x, tO = tmem + 256u + x * D;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tS, desc_k<D>(sQ, kk), desc_k<D>(sK + s * Tl::BYTES, kk), kIdS, kk > 0);
-        tc_commit(s_full(it & 1));
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          mma_ts(tO, tP + 8u * kk, desc_mn<D>(sVs, kk), kIdO, (!pend_first[x] || kk > 0));
+        tc_commit(o_done(x));
+        if (pend_rel[x]) tc_commit(v_empty(sv));
+        pend_t[x] = -1;
         return true;
       };
-      bool ok = wait_bounded(q_full, 0, g, 2) && issue_s(0);
-      for (int it = 0; ok && it < n; ++it) {
-        const int s = it % ST, bb = it & 1;
-        if (it + 1 < n) {
-          // S_{it+1} reuses the TMEM buffer that held P_{it-1}: PV_{it-1} must be done with it.
-          if (it >= 1 && !wait_bounded(o_done, (it - 1) & 1, g, 4)) break;
-          if (!issue_s(it + 1)) break;
+      for (int w = w0; ok && w < p.n_items; w += dw) {
+        const FwdItem I = fwd_item(p, w);
+        for (int x = 0; x < 2; ++x) {
+          if (x == 1 && !I.hasB) continue;
+          if (!wait_bounded(q_full(x), nq[x] & 1, g, 2)) { ok = false; break; }
+          ++nq[x];
         }
-        if (!wait_bounded(p_full(bb), (it >> 1) & 1, g, 5)) break;
-        if (!wait_bounded(v_full(s), (it / ST) & 1, g, 6)) break;
-        tc_fence_after();
-        const uint32_t tP = tmem + 128u * bb;
-        const uint32_t sVs = sV + s * Tl::BYTES;
+        for (int j = I.j_lo; ok && j <= I.j_hi; ++j, ++gk, ++gv) {
+          const int sk = gk % STK;
+          if (!wait_bounded(k_full(sk), (gk / STK) & 1, g, 3)) { ok = false; break; }
+          const bool actB = I.hasB && j >= I.lo[1] && j <= I.hi[1];
+          // slot x: the pending PV of x (previous key tile), then S_x for this key tile
+          auto step = [&](int x, bool act) -> bool {
+            if (pend_t[x] >= 0 && !issue_pv(x)) return false;
+            if (!act) return true;
+            tc_fence_after();
+            const uint32_t tS = tmem + 128u * x;
 #pragma unroll
-        for (int kh = 0; kh < 2; ++kh)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + 256u + kh * D, tP + 64u * kh + 8u * kk, desc_mn<D>(sVs, 4 * kh + kk),
-                   kIdO, (it > 0 || kk > 0));
-        tc_commit(o_done);
-        tc_commit(kv_empty(s));
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tS, desc_k<D>(sQ + x * Tl::BYTES, kk), desc_k<D>(sK + sk * Tl::BYTES, kk),
+                     kIdS, kk > 0);
+            tc_commit(s_full(x));
+            if (j == I.hi[x]) tc_commit(q_empty(x));  // last S of this query tile
+            pend_t[x] = tx[x]++;
+            pend_v[x] = gv;
+            pend_first[x] = (j == I.lo[x]);
+            pend_rel[x] = (x == 1) || !actB;  // the last PV to read V_j releases it
+            return true;
+          };
+          if (!step(0, j <= I.hi[0]) || !step(1, actB)) { ok = false; break; }
+          tc_commit(k_empty(sk));
+        }
+        if (ok && pend_t[0] >= 0 && !issue_pv(0)) ok = false;
+        if (ok && pend_t[1] >= 0 && !issue_pv(1)) ok = false;
       }
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
     }
     __syncwarp();
+  }
   } else {
+    regs_grow<208>();
     // ------------------------------------------------------ softmax warps
-    const int qd = warp & 3, kh = warp >> 2;
-    const int rl = qd * 32 + lane;  // row within the tile == TMEM lane
-    const int row = q0 + rl;
-    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    const uint32_t tO = tmem + lane_off + 256u + kh * D;
-    const int ds = p.doc ? p.doc[(size_t)b * T + (row < T ? row : T - 1)] : 0;
+    const int x = warp >> 2;             // 0: tile A, 1: tile B
+    const int rl = (warp & 3) * 32 + lane;  // row within the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + 128u * x;
+    const uint32_t tO = tmem + lane_off + 256u + x * D;
     const float sl2 = p.scale_log2;
-    // acc_l: sum of the fp32 weights (for the LSE); acc_lr: sum of the bf16-rounded weights
-    // the PV MMA actually multiplies (for normalising O).  Four packed fp32 pairs each, so
-    // the additions form independent chains.
-    float m = -INFINITY;
-    uint64_t acc_l[4], acc_lr[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc_l[i] = acc_lr[i] = f2(0.f, 0.f);
     const uint64_t sl2x2 = f2(sl2, sl2);
     bool ok = true;
-    for (int it = 0; it < n; ++it) {
-      const int bb = it & 1;
-      const int c0 = (kv_lo + it) * kRows + 64 * kh;  // first key of this thread's half
-      const uint32_t tS = tmem + lane_off + 128u * bb + 64u * kh;
-      if (!wait_bounded_warp(s_full(bb), (it >> 1) & 1, g, 7)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tS, sr[0]);
-      tmem_ld32(tS + 32u, sr[1]);
-      tc_wait_ld();
-      reg_fence(sr[0]);
-      reg_fence(sr[1]);
-      // mask only where needed: keys past the row, or before the row's document
-      if (!((c0 + 63 <= row) && (c0 >= ds))) {
-        const int hi = row - c0, lo = ds - c0;  // visible keys: e in [lo, hi]
+    int t = 0;   // tiles processed by this slot (s_full / p_full / o_done phases)
+    for (int w = w0; w < p.n_items; w += dw) {
+      const FwdItem I = fwd_item(p, w);
+      if (x == 1 && !I.hasB) continue;
+      const int row = I.qt[x] * kRows + rl;
+      const int ds = p.doc ? p.doc[(size_t)I.b * T + (row < T ? row : T - 1)] : 0;
+      float m = -INFINITY;
+      // acc_l: sum of the fp32 weights (for the LSE); acc_lr: sum of the bf16-rounded weights
+      // the PV MMA actually multiplies (for normalising O).  Packed pairs, independent chains.
+      uint64_t acc_l[4], acc_lr[4];
 #pragma unroll
-        for (int e = 0; e < 64; ++e)
-          if (e > hi || e < lo) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf
-      }
-      // row max of the raw scores (scale > 0 commutes with max), four independent chains
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int e = 0; e < 64; e += 8)
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          mx4[q] = fmax3(mx4[q], __uint_as_float(sr[(e + 2 * q) >> 5][(e + 2 * q) & 31]),
-                         __uint_as_float(sr[(e + 2 * q + 1) >> 5][(e + 2 * q + 1) & 31]));
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
-      const float m_new = fmaxf(m, mx);
-      const bool grow = m_new > m + 8.0f;  // also true the first time this half sees a key
-      const float alpha = grow ? ex2(m - m_new) : 1.0f;
-      if (it > 0 && __any_sync(0xffffffffu, grow)) {
-        // rescale this half's running O: PV_{it-1} must have landed first
-        if (!wait_bounded_warp(o_done, (it - 1) & 1, g, 8)) { ok = false; break; }
+      for (int i = 0; i < 4; ++i) acc_l[i] = acc_lr[i] = f2(0.f, 0.f);
+      const int n = I.hi[x] - I.lo[x] + 1;
+      const int t_last = t + n - 1;
+      for (int it = 0; ok && it < n; ++it, ++t) {
+        const int c0 = (I.lo[x] + it) * kRows;  // first key of the tile
+        if (!wait_bounded_warp(s_full(x), t & 1, g, 8)) { ok = false; break; }
+        // s_full(t) also means PV(t-1) has completed: O_x may be read and rescaled
         tc_fence_after();
-        const uint64_t a2 = f2(alpha, alpha);
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32u * c, sr[c]);
+        tc_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+        if (!((c0 + kRows - 1 <= row) && (c0 >= ds))) {
+          const int hi = row - c0, lo = ds - c0;  // visible keys: e in [lo, hi]
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (e > hi || e < lo) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf
+        }
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int e = 0; e < 128; e += 8)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mx4[q] = fmax3(mx4[q], __uint_as_float(sr[(e + 2 * q) >> 5][(e + 2 * q) & 31]),
+                           __uint_as_float(sr[(e + 2 * q + 1) >> 5][(e + 2 * q + 1) & 31]));
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+        const float m_new = fmaxf(m, mx);
+        const bool grow = m_new > m + 8.0f;  // also true the first time a row sees a key
+        const float alpha = grow ? ex2(m - m_new) : 1.0f;
+        if (it > 0 && __any_sync(0xffffffffu, grow)) {
+          const uint64_t a2 = f2(alpha, alpha);
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld16(tO + 16u * c, r);
+            tc_wait_ld();
+            reg_fence16(r);
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const float2 y = f2split(fmul2(f2u(r[e], r[e + 1]), a2));
+              r[e] = __float_as_uint(y.x);
+              r[e + 1] = __float_as_uint(y.y);
+            }
+            tmem_st16(tO + 16u * c, r);
+          }
+        }
+        if (grow) {
+          const uint64_t a2 = f2(alpha, alpha);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc_l[i] = fmul2(acc_l[i], a2);
+            acc_lr[i] = fmul2(acc_lr[i], a2);
+          }
+          m = m_new;
+        }
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        const uint64_t nmu2 = f2(-mu, -mu);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 xx = f2split(ffma2(f2u(sr[c][2 * e], sr[c][2 * e + 1]), sl2x2, nmu2));
+            const float p0 = ex2(xx.x), p1 = ex2(xx.y);
+            const uint32_t v = pack_bf16(p0, p1);
+            acc_l[e & 3] = fadd2(acc_l[e & 3], f2(p0, p1));
+            acc_lr[e & 3] = fadd2(acc_lr[e & 3], bf16x2_to_f2(v));
+            pk[e] = v;
+          }
+          tmem_st16(tS + 16u * c, pk);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(x));
+      }
+      t = t_last + 1;
+      // ---------------------------------------------------------- epilogue
+      if (ok && wait_bounded_warp(o_done(x), t_last & 1, g, 10)) {
+        tc_fence_after();
+        float l = 0.f, lr = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 a = f2split(acc_l[i]), bq = f2split(acc_lr[i]);
+          l += a.x + a.y;
+          lr += bq.x + bq.y;
+        }
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        if (row < T) p.lse[(size_t)I.bh * T + row] = (mu + lg2(l)) * kLn2;
+        const float inv = 1.0f / lr;
+        __nv_bfloat16* orow = p.o + ((size_t)I.bh * T + row) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
           tmem_ld32(tO + 32u * c, r);
           tc_wait_ld();
           reg_fence(r);
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float2 y = f2split(fmul2(f2u(r[e], r[e + 1]), a2));
-            r[e] = __float_as_uint(y.x);
-            r[e + 1] = __float_as_uint(y.y);
-          }
-          tmem_st32(tO + 32u * c, r);
+          if (row < T) store_row_chunk_bf16(orow + 32 * c, r, inv);
         }
-      }
-      if (grow) {
-        const uint64_t a2 = f2(alpha, alpha);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc_l[i] = fmul2(acc_l[i], a2);
-          acc_lr[i] = fmul2(acc_lr[i], a2);
-        }
-        m = m_new;
-      }
-      const float mu = (m == -INFINITY) ? 0.f : m;
-      const uint64_t nmu2 = f2(-mu, -mu);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 x = f2split(ffma2(f2u(sr[c][2 * e], sr[c][2 * e + 1]), sl2x2, nmu2));
-          const float p0 = ex2(x.x), p1 = ex2(x.y);
-          const uint32_t v = pack_bf16(p0, p1);
-          acc_l[e & 3] = fadd2(acc_l[e & 3], f2(p0, p1));
-          acc_lr[e & 3] = fadd2(acc_lr[e & 3], bf16x2_to_f2(v));
-          pk[e] = v;
-        }
-        tmem_st16(tS + 16u * c, pk);
-      }
-      tc_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(bb));
-    }
-    float l = 0.f, lr = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 a = f2split(acc_l[i]), bq = f2split(acc_lr[i]);
-      l += a.x + a.y;
-      lr += bq.x + bq.y;
-    }
-    // ------------------------------------------------------------ epilogue
-    ok = ok && wait_bounded_warp(o_done, (n - 1) & 1, g, 9);
-    red[(kh * 3 + 0) * kRows + rl] = m;
-    red[(kh * 3 + 1) * kRows + rl] = lr;
-    red[(kh * 3 + 2) * kRows + rl] = l;
-    named_barrier(1, L::SOFTMAX_WARPS * 32);  // every softmax thread reaches this exactly once
-    if (ok) {
-      tc_fence_after();
-      const int oh = kh ^ 1;
-      const float mo = red[(oh * 3 + 0) * kRows + rl];
-      const float lro = red[(oh * 3 + 1) * kRows + rl];
-      const float lo = red[(oh * 3 + 2) * kRows + rl];
-      float M = fmaxf(m, mo);
-      if (M == -INFINITY) M = 0.f;
-      const float a_self = ex2(m - M), a_oth = ex2(mo - M);
-      const float LR = lr * a_self + lro * a_oth;
-      const float LX = l * a_self + lo * a_oth;
-      if (kh == 0 && row < T) p.lse[(size_t)bh * T + row] = (M + lg2(LX)) * kLn2;
-      const float inv = 1.0f / LR;
-      const float w0 = (kh == 0 ? a_self : a_oth) * inv;  // weight of O_half0
-      const float w1 = (kh == 0 ? a_oth : a_self) * inv;  // weight of O_half1
-      const uint32_t tO0 = tmem + lane_off + 256u, tO1 = tO0 + D;
-      __nv_bfloat16* orow = p.o + ((size_t)bh * T + row) * D;
-      // this thread writes output columns [kh*D/2, (kh+1)*D/2)
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        const int col = kh * (D / 2) + 16 * c;
-        uint32_t r0[16], r1[16];
-        tmem_ld16(tO0 + col, r0);
-        tmem_ld16(tO1 + col, r1);
-        tc_wait_ld();
-        reg_fence16(r0);
-        reg_fence16(r1);
-        uint32_t pk[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float y0 = __uint_as_float(r0[2 * e]) * w0 + __uint_as_float(r1[2 * e]) * w1;
-          const float y1 = __uint_as_float(r0[2 * e + 1]) * w0 + __uint_as_float(r1[2 * e + 1]) * w1;
-          pk[e] = pack_bf16(y0, y1);
-        }
-        if (row < T) {
-          uint4* d4 = reinterpret_cast<uint4*>(orow + col);
-          d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
+        // O_x has been read: the next item's first PV may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_free(x));
+      } else {
+        ok = false;
       }
     }
   }

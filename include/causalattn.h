@@ -168,6 +168,12 @@ const char* gpt_attn_strerror(int status);
 /* GPT_ATTN_ABI_VERSION of the loaded library. */
 int gpt_attn_version(void);
 
+/*
+ * Text of the CUDA error behind the most recent GPT_ATTN_ERR_LAUNCH returned on
+ * the calling thread ("no error" if none).  Static string, never NULL.
+ */
+const char* gpt_attn_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif
