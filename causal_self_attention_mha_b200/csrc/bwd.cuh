@@ -57,6 +57,7 @@ struct BwdParams {
   __nv_bfloat16* g0;      // dK (dkdv kernel) or dQ (dq kernel)   [B, H, T, D]
   __nv_bfloat16* g1;      // dV (dkdv kernel) or unused
   int H, T, BH, n_t;      // n_t = number of 128-row tiles along T
+  int n_items;            // n_t * BH work items (one 128-row tile of one head each)
   float scale;            // softmax scale (1/sqrt(d))
   float scale_log2;       // scale * log2(e)
   uint64_t wait_limit_ns;
@@ -74,13 +75,19 @@ __device__ __forceinline__ void store16_bf16(__nv_bfloat16* dst, const uint32_t 
   d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
-// Both tiled backward kernels walk the other operand in 64-row halves of its
-// 128-row tiles (N = 64 for the S / dP products).  Half g uses TMEM "set"
-// g % 2: its S (or S^T) in columns [128*set, +64) and dP (or dP^T) in
-// [128*set + 64, +64), so the MMAs of half g+1 run while the 8 element-wise
-// warps work on half g.  Element-wise warp w owns TMEM lanes 32*(w%4).. and
-// columns 32*(w/4).. of each half; it writes its bf16 P / dS (16 packed
-// columns) over the first half of the fp32 columns it has just read.
+// Both tiled backward kernels are persistent: one CTA per SM walks work items
+// w = blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest first) and streams the
+// other operand in 64-row halves of its 128-row tiles (N = 64 for the S / dP
+// products).  Half g uses TMEM "set" g % 2: its S (or S^T) in columns
+// [128*set, +64) and dP (or dP^T) in [128*set + 64, +64), so the MMAs of half
+// g+1 run while the 8 element-wise warps work on half g.  A set is reused two
+// halves later by the next S / dP MMAs, which the single in-order MMA stream
+// issues after the gradient MMAs that read it.  Element-wise warp w owns TMEM
+// lanes 32*(w%4).. and columns 32*(w/4).. of each half; it writes its bf16 P /
+// dS (16 packed columns) over the first half of the fp32 columns it has just
+// read.  At an item boundary the gradient accumulators are handed over with
+// acc_done (MMA -> epilogue) and acc_free (epilogue -> next item's first
+// gradient MMA).
 
 // ------------------------------------------------------------------ dK/dV
 template <int D>
@@ -90,18 +97,47 @@ struct DkdvLayout {
   static constexpr int V_OFF = K_OFF + Tile<D>::BYTES;
   static constexpr int Q_OFF = V_OFF + Tile<D>::BYTES;             // + s * BYTES
   static constexpr int DO_OFF = Q_OFF + ST * Tile<D>::BYTES;       // + s * BYTES
-  static constexpr int VEC_OFF = DO_OFF + ST * Tile<D>::BYTES;     // per stage: lse2, delta, dsq
+  static constexpr int VEC_OFF = DO_OFF + ST * Tile<D>::BYTES;     // per stage: -lse2, -delta, dsq
   static constexpr int VEC_STAGE = 3 * kRows * 4;
   static constexpr int BAR_OFF = VEC_OFF + ST * VEC_STAGE;
-  // barriers: kv_full | q_full[ST] | q_empty[ST] | st_full[2] | pds_full[2] | set_free[2] | acc_done | drain
-  static constexpr int NBAR = 1 + 2 * ST + 6 + 2;
-  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem slot, abort flag, query-tile range
-  static constexpr int BYTES = MISC_OFF + 32;
+  // barriers: kv_full kv_empty | q_full[ST] q_empty[ST] | st_full[2] pds_full[2] | acc_done acc_free drain
+  static constexpr int NBAR = 2 + 2 * ST + 4 + 3;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem slot, abort flag
+  static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
   static constexpr int COMPUTE_WARPS = 8;
   static constexpr int THREADS = (COMPUTE_WARPS + 2) * 32;
   static constexpr uint32_t TMEM_COLS = 512;
 };
+
+struct DkdvItem {
+  int jt, bh, b, k0, i_lo, n;  // key tile, head, batch, first key row, query tiles [i_lo, i_lo+n)
+};
+
+// Key tiles near the start of the sequence see the most query tiles: they come first.
+__device__ __forceinline__ DkdvItem dkdv_item(const BwdParams& p, int w) {
+  DkdvItem I;
+  I.jt = w / p.BH;
+  I.bh = w % p.BH;
+  I.b = I.bh / p.H;
+  I.k0 = I.jt * kRows;
+  I.i_lo = I.jt;
+  int i_hi = p.n_t - 1;
+  if (p.doc) {
+    // last query row that can see the last key row of this tile: end of its document - 1
+    const int32_t* drow = p.doc + (size_t)I.b * p.T;
+    const int c_last = (I.k0 + kRows - 1 < p.T) ? I.k0 + kRows - 1 : p.T - 1;
+    int lo = c_last + 1, hi = p.T;  // first r in (c_last, T) with drow[r] > c_last, else T
+    while (lo < hi) {
+      const int mid = lo + ((hi - lo) >> 1);
+      if (drow[mid] > c_last) hi = mid; else lo = mid + 1;
+    }
+    i_hi = (lo - 1) / kRows;
+    i_hi = i_hi < I.jt ? I.jt : (i_hi > p.n_t - 1 ? p.n_t - 1 : i_hi);
+  }
+  I.n = i_hi - I.i_lo + 1;
+  return I;
+}
 
 template <int D>
 __global__ void __launch_bounds__(320, 1)
@@ -121,43 +157,24 @@ __global__ void __launch_bounds__(320, 1)
   auto sdO = [&](int s) { return sbase + L::DO_OFF + s * Tl::BYTES; };
   float* vec = reinterpret_cast<float*>(gsm + L::VEC_OFF);   // [ST][3][128]
   const uint32_t bar0 = sbase + L::BAR_OFF;
-  const uint32_t kv_full = bar0;
-  auto q_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto q_empty = [&](int s) { return bar0 + 8u * (1 + ST + s); };
-  auto st_full = [&](int b) { return bar0 + 8u * (1 + 2 * ST + b); };
-  auto pds_full = [&](int b) { return bar0 + 8u * (3 + 2 * ST + b); };
-  auto set_free = [&](int b) { return bar0 + 8u * (5 + 2 * ST + b); };
-  const uint32_t acc_done = bar0 + 8u * (7 + 2 * ST);
+  const uint32_t kv_full = bar0, kv_empty = bar0 + 8u;
+  auto q_full = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto q_empty = [&](int s) { return bar0 + 8u * (2 + ST + s); };
+  auto st_full = [&](int b) { return bar0 + 8u * (2 + 2 * ST + b); };
+  auto pds_full = [&](int b) { return bar0 + 8u * (4 + 2 * ST + b); };
+  const uint32_t acc_done = bar0 + 8u * (6 + 2 * ST);
+  const uint32_t acc_free = bar0 + 8u * (7 + 2 * ST);
   const uint32_t drain = bar0 + 8u * (8 + 2 * ST);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
-  int* range = reinterpret_cast<int*>(gsm + L::MISC_OFF + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.T;
-  // Work item: key tiles near the start of the sequence see the most query tiles; launch them first.
-  const int jt = (int)(blockIdx.x / p.BH);
-  const int bh = (int)(blockIdx.x % p.BH);
-  const int b = bh / p.H;
-  const int k0 = jt * kRows;
+  const int w0 = blockIdx.x, dw = gridDim.x;
 
   if (threadIdx.x == 0) {
-    int i_hi = p.n_t - 1;
-    if (p.doc) {
-      // last query row that can see the last key row of this tile: end of its document - 1
-      const int32_t* drow = p.doc + (size_t)b * T;
-      const int c_last = (k0 + kRows - 1 < T) ? k0 + kRows - 1 : T - 1;
-      int lo = c_last + 1, hi = T;  // first r in (c_last, T) with drow[r] > c_last, else T
-      while (lo < hi) {
-        const int mid = lo + ((hi - lo) >> 1);
-        if (drow[mid] > c_last) hi = mid; else lo = mid + 1;
-      }
-      i_hi = (lo - 1) / kRows;
-      i_hi = i_hi < jt ? jt : (i_hi > p.n_t - 1 ? p.n_t - 1 : i_hi);
-    }
-    range[0] = jt;
-    range[1] = i_hi;
     mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
     for (int s = 0; s < ST; ++s) {
       mbar_init(q_full(s), 32);
       mbar_init(q_empty(s), 1);
@@ -165,9 +182,9 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(st_full(i), 1);
       mbar_init(pds_full(i), L::COMPUTE_WARPS);
-      mbar_init(set_free(i), 1);
     }
     mbar_init(acc_done, 1);
+    mbar_init(acc_free, L::COMPUTE_WARPS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -180,9 +197,6 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int i_lo = range[0];
-  const int n = range[1] - i_lo + 1;   // query tiles
-  const int nh = 2 * n;                // query halves
   const Guard g{abort_flag, p.wait_limit_ns};
   const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D;
 
@@ -193,43 +207,55 @@ __global__ void __launch_bounds__(320, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
-      mbar_arrive_expect_tx(kv_full, 2 * Tl::BYTES);
-      load_tile<D>(sK, &tmK, k0, bh, kv_full);
-      load_tile<D>(sV, &tmV, k0, bh, kv_full);
     }
-    int it = 0;
-    for (; it < n; ++it) {
-      const int s = it % ST, u = it / ST;
-      if (u > 0 && !wait_bounded_warp(q_empty(s), (u - 1) & 1, g, 1)) break;
-      const int r0 = (i_lo + it) * kRows;
-      float* lse2 = vec + s * 3 * kRows;
-      float* dl = lse2 + kRows;
-      int* dsq = reinterpret_cast<int*>(dl + kRows);
-#pragma unroll
-      for (int k = 0; k < kRows / 32; ++k) {
-        const int rl = lane + 32 * k, r = r0 + rl;
-        if (r < T) {  // stored negated: -LSE*log2(e) and -delta
-          lse2[rl] = -p.lse[(size_t)bh * T + r] * kLog2e;
-          dl[rl] = -p.delta[(size_t)bh * T + r];
-          dsq[rl] = p.doc ? p.doc[(size_t)b * T + r] : 0;
-        } else {  // rows past the end: no key is visible
-          lse2[rl] = -INFINITY;
-          dl[rl] = 0.f;
-          dsq[rl] = 0x7fffffff;
-        }
-      }
+    int li = 0, gq = 0;  // items whose K/V were loaded, query tiles loaded
+    bool ok = true;
+    for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
+      const DkdvItem I = dkdv_item(p, w);
+      // K/V of this item: the previous item's last S^T / dP^T MMAs must be done with them
+      if (li >= 1 && !wait_bounded_warp(kv_empty, (li - 1) & 1, g, 1)) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(q_full(s), 2 * Tl::BYTES);
-        load_tile<D>(sQ(s), &tmQ, r0, bh, q_full(s));
-        load_tile<D>(sdO(s), &tmdO, r0, bh, q_full(s));
-      } else {
-        mbar_arrive(q_full(s));
+        mbar_arrive_expect_tx(kv_full, 2 * Tl::BYTES);
+        load_tile<D>(sK, &tmK, I.k0, I.bh, kv_full);
+        load_tile<D>(sV, &tmV, I.k0, I.bh, kv_full);
+      }
+      ++li;
+      for (int it = 0; it < I.n; ++it) {
+        const int s = gq % ST, u = gq / ST;
+        if (u > 0 && !wait_bounded_warp(q_empty(s), (u - 1) & 1, g, 1)) { ok = false; break; }
+        const int r0 = (I.i_lo + it) * kRows;
+        float* lse2 = vec + s * 3 * kRows;
+        float* dl = lse2 + kRows;
+        int* dsq = reinterpret_cast<int*>(dl + kRows);
+#pragma unroll
+        for (int k = 0; k < kRows / 32; ++k) {
+          const int rl = lane + 32 * k, r = r0 + rl;
+          if (r < T) {  // stored negated: -LSE*log2(e) and -delta
+            lse2[rl] = -p.lse[(size_t)I.bh * T + r] * kLog2e;
+            dl[rl] = -p.delta[(size_t)I.bh * T + r];
+            dsq[rl] = p.doc ? p.doc[(size_t)I.b * T + r] : 0;
+          } else {  // rows past the end: no key is visible
+            lse2[rl] = -INFINITY;
+            dl[rl] = 0.f;
+            dsq[rl] = 0x7fffffff;
+          }
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full(s), 2 * Tl::BYTES);
+          load_tile<D>(sQ(s), &tmQ, r0, I.bh, q_full(s));
+          load_tile<D>(sdO(s), &tmdO, r0, I.bh, q_full(s));
+        } else {
+          mbar_arrive(q_full(s));
+        }
+        ++gq;
       }
     }
-    if (lane == 0 && *abort_flag) {
-      drain_wait(kv_full, 0, p.wait_limit_ns);
+    if (lane == 0 && *abort_flag) {  // let every copy already issued land before the CTA exits
+      if (li > 0) drain_wait(kv_full, (li - 1) & 1, p.wait_limit_ns);
       for (int s = 0; s < ST; ++s) {
-        const int cnt = it > s ? (it - s + ST - 1) / ST : 0;
+        const int cnt = gq > s ? (gq - s + ST - 1) / ST : 0;
         if (cnt > 0) drain_wait(q_full(s), (cnt - 1) & 1, p.wait_limit_ns);
       }
     }
@@ -239,44 +265,61 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, false);  // S^T, dP^T: M = keys, N = 64 queries
       constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);    // dV, dK: N = d, B is MN-major
-      // dV += P^T dO and dK += dS^T Q for query half gp (K = 64 queries, 4 MMA-K steps)
-      auto issue_grad = [&](int gp) -> bool {
-        const int bp = gp & 1, sp = (gp >> 1) % ST;
+      int li = 0, gq = 0, gh = 0;  // items, query tiles, query halves consumed
+      // dV += P^T dO and dK += dS^T Q for global half gp (K = 64 queries, 4 MMA-K steps);
+      // `first`: first half of its item (accumulators start from zero)
+      auto issue_grad = [&](int gp, int sp, bool first) -> bool {
+        const int bp = gp & 1;
+        // the first gradient MMA of an item overwrites dV / dK: the previous epilogue must be done
+        if (first && li >= 2 && !wait_bounded(acc_free, (li - 2) & 1, g, 4)) return false;
         if (!wait_bounded(pds_full(bp), (gp >> 1) & 1, g, 5)) return false;
         tc_fence_after();
         const uint32_t tset = tmem + 128u * bp;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tdV, tset + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sdO(sp), 4 * bp + kk), kIdG,
-                 (gp > 0 || kk > 0));
+                 (!first || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tdK, tset + 64u + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sQ(sp), 4 * bp + kk),
-                 kIdG, (gp > 0 || kk > 0));
-        tc_commit(set_free(bp));
+                 kIdG, (!first || kk > 0));
         if (bp == 1) tc_commit(q_empty(sp));
         return true;
       };
-      bool ok = wait_bounded(kv_full, 0, g, 2);
-      for (int gh = 0; ok && gh < nh; ++gh) {
-        const int it = gh >> 1, h = gh & 1, s = it % ST;
-        if (h == 0 && !wait_bounded(q_full(s), (it / ST) & 1, g, 3)) break;
-        // set h is reused: the dV / dK MMAs of half gh-2 must have finished reading it
-        if (gh >= 2 && !wait_bounded(set_free(h), ((gh - 2) >> 1) & 1, g, 4)) break;
-        tc_fence_after();
-        const uint32_t tset = tmem + 128u * h;
-        const uint32_t off = (uint32_t)(64 * h * Tl::SW);  // query rows 64h.. of the stage tile
+      bool ok = true;
+      for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
+        const DkdvItem I = dkdv_item(p, w);
+        if (!wait_bounded(kv_full, li & 1, g, 2)) break;
+        ++li;
+        int prev_s = 0;
+        for (int it = 0; ok && it < I.n; ++it, ++gq) {
+          const int s = gq % ST;
+          if (!wait_bounded(q_full(s), (gq / ST) & 1, g, 3)) { ok = false; break; }
+          for (int h = 0; h < 2; ++h, ++gh) {
+            tc_fence_after();
+            const uint32_t tset = tmem + 128u * h;
+            const uint32_t off = (uint32_t)(64 * h * Tl::SW);  // query rows 64h.. of the stage tile
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tset, desc_k<D>(sK, kk), desc_k<D>(sQ(s) + off, kk), kIdS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tset, desc_k<D>(sK, kk), desc_k<D>(sQ(s) + off, kk), kIdS, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tset + 64u, desc_k<D>(sV, kk), desc_k<D>(sdO(s) + off, kk), kIdS, kk > 0);
-        tc_commit(st_full(h));
-        if (gh >= 1 && !issue_grad(gh - 1)) { ok = false; break; }
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tset + 64u, desc_k<D>(sV, kk), desc_k<D>(sdO(s) + off, kk), kIdS, kk > 0);
+            tc_commit(st_full(h));
+            if (it == I.n - 1 && h == 1) tc_commit(kv_empty);  // K, V of this item no longer read
+            if ((it > 0 || h > 0) && !issue_grad(gh - 1, h == 0 ? prev_s : s, it == 0 && h == 1)) {
+              ok = false;
+              break;
+            }
+          }
+          prev_s = s;
+        }
+        // the item's last half (never its first: that one was issued inside the loop)
+        if (ok && !issue_grad(gh - 1, prev_s, false)) ok = false;
+        if (ok) tc_commit(acc_done);
       }
-      if (ok) issue_grad(nh - 1);
-      tc_commit(acc_done);
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
     }
@@ -284,83 +327,99 @@ __global__ void __launch_bounds__(320, 1)
   } else {
     // ------------------------------------------- P^T / dS^T (thread = key row)
     const int qd = warp & 3, cs = warp >> 2;
-    const int c = k0 + qd * 32 + lane;  // key position owned by this thread
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2(sl2, sl2);
     bool ok = true;
-    for (int gh = 0; gh < nh; ++gh) {
-      const int it = gh >> 1, h = gh & 1, s = it % ST;
-      if (!wait_bounded_warp(st_full(h), (gh >> 1) & 1, g, 6)) { ok = false; break; }
-      if (!wait_bounded_warp(q_full(s), (it / ST) & 1, g, 7)) { ok = false; break; }
-      tc_fence_after();
-      const float* lse2 = vec + s * 3 * kRows;
-      const float* dl = lse2 + kRows;
-      const int* dsq = reinterpret_cast<const int*>(dl + kRows);
-      const int rb = 64 * h + 32 * cs;           // first query row (within the tile) of my columns
-      const int r0 = (i_lo + it) * kRows + rb;   // its position
-      const uint32_t tS = tmem + lane_off + 128u * h + 32u * cs;
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tS, sr);
-      tmem_ld32(tS + 64u, dr);
-      tc_wait_ld();
-      reg_fence(sr);
-      reg_fence(dr);
-      // no mask needed when all my query rows are at or below this key and their
-      // documents start at or before it (dsq is nondecreasing; huge past T)
-      if (!((r0 >= c) && (dsq[rb + 31] <= c))) {
-        const int4* ds4 = reinterpret_cast<const int4*>(dsq + rb);
+    int li = 0, gq = 0, gh = 0;
+    for (int k_ = 0; k_ * dw < p.n_items; ++k_, ++li) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
+      const DkdvItem I = dkdv_item(p, w);
+      const int c = I.k0 + qd * 32 + lane;  // key position owned by this thread
+      for (int it = 0; ok && it < I.n; ++it, ++gq) {
+        const int s = gq % ST;
+        for (int h = 0; h < 2; ++h, ++gh) {
+          if (!wait_bounded_warp(st_full(h), (gh >> 1) & 1, g, 6)) { ok = false; break; }
+          if (!wait_bounded_warp(q_full(s), (gq / ST) & 1, g, 7)) { ok = false; break; }
+          tc_fence_after();
+          const float* lse2 = vec + s * 3 * kRows;
+          const float* dl = lse2 + kRows;
+          const int* dsq = reinterpret_cast<const int*>(dl + kRows);
+          const int rb = 64 * h + 32 * cs;                 // first query row (in the tile) of my columns
+          const int r0 = (I.i_lo + it) * kRows + rb;       // its position
+          const uint32_t tS = tmem + lane_off + 128u * h + 32u * cs;
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tS, sr);
+          tmem_ld32(tS + 64u, dr);
+          tc_wait_ld();
+          reg_fence(sr);
+          reg_fence(dr);
+          // no mask needed when all my query rows are at or below this key and their
+          // documents start at or before it (dsq is nondecreasing; huge past T)
+          if (!((r0 >= c) && (dsq[rb + 31] <= c))) {
+            const int4* ds4 = reinterpret_cast<const int4*>(dsq + rb);
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const int4 dv4 = ds4[q4];
-          const int dsv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const int4 dv4 = ds4[q4];
+              const int dsv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int e = 4 * q4 + k;
-            if (c > r0 + e || c < dsv[k]) sr[e] = 0xFF800000u;  // -inf: weight 0
+              for (int k = 0; k < 4; ++k) {
+                const int e = 4 * q4 + k;
+                if (c > r0 + e || c < dsv[k]) sr[e] = 0xFF800000u;  // -inf: weight 0
+              }
+            }
           }
+          const float4* l4 = reinterpret_cast<const float4*>(lse2 + rb);  // -LSE*log2(e)
+          const float4* d4 = reinterpret_cast<const float4*>(dl + rb);    // -delta
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 lv = l4[q4], dv4 = d4[q4];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = 4 * q4 + 2 * h2;
+              const uint64_t nl = h2 ? f2(lv.z, lv.w) : f2(lv.x, lv.y);
+              const uint64_t nd = h2 ? f2(dv4.z, dv4.w) : f2(dv4.x, dv4.y);
+              // P^T = exp2(S^T * scale * log2e - LSE * log2e);  dS^T = P^T * (dP^T - delta)
+              const float2 x = f2split(ffma2(f2u(sr[e], sr[e + 1]), sl2x2, nl));
+              const float p0 = ex2(x.x), p1 = ex2(x.y);
+              const float2 dd = f2split(fmul2(f2(p0, p1), fadd2(f2u(dr[e], dr[e + 1]), nd)));
+              pk[e >> 1] = pack_bf16(p0, p1);
+              dk[e >> 1] = pack_bf16(dd.x, dd.y);
+            }
+          }
+          tmem_st16(tS, pk);
+          tmem_st16(tS + 64u, dk);
+          tc_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(pds_full(h));
         }
+        if (!ok) break;
       }
-      const float4* l4 = reinterpret_cast<const float4*>(lse2 + rb);  // -LSE*log2(e)
-      const float4* d4 = reinterpret_cast<const float4*>(dl + rb);    // -delta
-      uint32_t pk[16], dk[16];
+      // ---------------------------------------------------------- epilogue
+      if (ok && wait_bounded_warp(acc_done, li & 1, g, 8)) {
+        tc_fence_after();
+        __nv_bfloat16* dk_row = p.g0 + ((size_t)I.bh * T + c) * D;
+        __nv_bfloat16* dv_row = p.g1 + ((size_t)I.bh * T + c) * D;
+        // 16-column jobs over (dV, dK), split between the two warps that share these lanes
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 lv = l4[q4], dv4 = d4[q4];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int e = 4 * q4 + 2 * h2;
-          const uint64_t nl = h2 ? f2(lv.z, lv.w) : f2(lv.x, lv.y);
-          const uint64_t nd = h2 ? f2(dv4.z, dv4.w) : f2(dv4.x, dv4.y);
-          // P^T = exp2(S^T * scale * log2e - LSE * log2e);  dS^T = P^T * (dP^T - delta)
-          const float2 x = f2split(ffma2(f2u(sr[e], sr[e + 1]), sl2x2, nl));
-          const float p0 = ex2(x.x), p1 = ex2(x.y);
-          const float2 dd = f2split(fmul2(f2(p0, p1), fadd2(f2u(dr[e], dr[e + 1]), nd)));
-          pk[e >> 1] = pack_bf16(p0, p1);
-          dk[e >> 1] = pack_bf16(dd.x, dd.y);
+        for (int j = cs; j < 2 * (D / 16); j += 2) {
+          const bool is_k = j >= D / 16;
+          const int col = 16 * (is_k ? j - D / 16 : j);
+          uint32_t r[16];
+          tmem_ld16((is_k ? tdK : tdV) + lane_off + col, r);
+          tc_wait_ld();
+          reg_fence16(r);
+          if (c < T) store16_bf16((is_k ? dk_row : dv_row) + col, r, is_k ? p.scale : 1.0f);
         }
-      }
-      tmem_st16(tS, pk);
-      tmem_st16(tS + 64u, dk);
-      tc_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(pds_full(h));
-    }
-    if (ok && wait_bounded_warp(acc_done, 0, g, 8)) {
-      tc_fence_after();
-      __nv_bfloat16* dk_row = p.g0 + ((size_t)bh * T + c) * D;
-      __nv_bfloat16* dv_row = p.g1 + ((size_t)bh * T + c) * D;
-      // 16-column jobs over (dV, dK), split between the two warps that share these lanes
-#pragma unroll
-      for (int j = cs; j < 2 * (D / 16); j += 2) {
-        const bool is_k = j >= D / 16;
-        const int col = 16 * (is_k ? j - D / 16 : j);
-        uint32_t r[16];
-        tmem_ld16((is_k ? tdK : tdV) + lane_off + col, r);
-        tc_wait_ld();
-        reg_fence16(r);
-        if (c < T) store16_bf16((is_k ? dk_row : dv_row) + col, r, is_k ? p.scale : 1.0f);
+        // dV / dK have been read: the next item's first gradient MMA may overwrite them
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_free);
+      } else {
+        ok = false;
       }
     }
   }
@@ -374,23 +433,85 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // --------------------------------------------------------------------- dQ
+// Q and dO are the stationary operands of the dQ kernel: they are staged in
+// shared memory by TMA and then copied, once per item, into TMEM, so S = Q K^T
+// and dP = dO V^T run as TMEM-operand MMAs that read only the streamed K / V
+// half from shared memory.
 template <int D>
 struct DqLayout {
   static constexpr int ST = (D == 128) ? 2 : 3;   // K/V ring depth (128-row tiles)
-  static constexpr int Q_OFF = 0;
+  static constexpr int Q_OFF = 0;                  // Q, dO staging for the TMEM copy
   static constexpr int DO_OFF = Q_OFF + Tile<D>::BYTES;
   static constexpr int K_OFF = DO_OFF + Tile<D>::BYTES;           // + s * BYTES
   static constexpr int V_OFF = K_OFF + ST * Tile<D>::BYTES;       // + s * BYTES
   static constexpr int BAR_OFF = V_OFF + ST * Tile<D>::BYTES;
-  // barriers: qdo_full | kv_full[ST] | kv_empty[ST] | s_full[2] | ds_full[2] | set_free[2] | acc_done | drain
-  static constexpr int NBAR = 1 + 2 * ST + 6 + 2;
+  // barriers: qdo_full qdo_tmem | kv_full[ST] kv_empty[ST] | s_full[2] ds_full[2] | acc_done acc_free drain
+  static constexpr int NBAR = 2 + 2 * ST + 4 + 3;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
   static constexpr int COMPUTE_WARPS = 8;
   static constexpr int THREADS = (COMPUTE_WARPS + 2) * 32;
   static constexpr uint32_t TMEM_COLS = 512;
+  // TMEM columns: sets at 0 and 128, dQ at 256, Q at 256 + D, dO at 256 + 3D/2
+  static constexpr uint32_t T_DQ = 256, T_Q = 256 + D, T_DO = 256 + D + D / 2;
 };
+
+struct DqItem {
+  int qt, bh, b, q0, kv_lo, n;  // query tile, head, batch, first row, key tiles [kv_lo, kv_lo+n)
+};
+
+// Query tiles near the end of the sequence see the most key tiles: they come first.
+__device__ __forceinline__ DqItem dq_item(const BwdParams& p, int w) {
+  DqItem I;
+  I.qt = p.n_t - 1 - w / p.BH;
+  I.bh = w % p.BH;
+  I.b = I.bh / p.H;
+  I.q0 = I.qt * kRows;
+  I.kv_lo = 0;
+  if (p.doc) {
+    const int lo = p.doc[(size_t)I.b * p.T + I.q0] / kRows;
+    I.kv_lo = lo < 0 ? 0 : (lo > I.qt ? I.qt : lo);
+  }
+  I.n = I.qt - I.kv_lo + 1;
+  return I;
+}
+
+// Copy row `rl` of a TMA-swizzled 128-row tile from shared memory into TMEM
+// (this thread's lane) as packed bf16 pairs: D/2 columns starting at `taddr`.
+// The hardware swizzle puts 16-byte granule g of row r at g ^ (r & 7) (128-byte
+// rows) or g ^ ((r >> 1) & 3) (64-byte rows).
+template <int D>
+__device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int rl, uint32_t taddr) {
+  using Tl = Tile<D>;
+#pragma unroll
+  for (int c = 0; c < Tl::CHUNKS; ++c) {
+    const uint8_t* row = tile + c * Tl::CHUNK_BYTES + rl * Tl::SW;
+    if constexpr (Tl::SW == 128) {
+      uint32_t r[32];
+#pragma unroll
+      for (int gi = 0; gi < 8; ++gi) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + ((gi ^ (rl & 7)) * 16));
+        r[4 * gi] = v.x;
+        r[4 * gi + 1] = v.y;
+        r[4 * gi + 2] = v.z;
+        r[4 * gi + 3] = v.w;
+      }
+      tmem_st32(taddr + 32u * c, r);
+    } else {
+      uint32_t r[16];
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + ((gi ^ ((rl >> 1) & 3)) * 16));
+        r[4 * gi] = v.x;
+        r[4 * gi + 1] = v.y;
+        r[4 * gi + 2] = v.z;
+        r[4 * gi + 3] = v.w;
+      }
+      tmem_st16(taddr + 16u * c, r);
+    }
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(320, 1)
@@ -408,33 +529,24 @@ __global__ void __launch_bounds__(320, 1)
   auto sK = [&](int s) { return sbase + L::K_OFF + s * Tl::BYTES; };
   auto sV = [&](int s) { return sbase + L::V_OFF + s * Tl::BYTES; };
   const uint32_t bar0 = sbase + L::BAR_OFF;
-  const uint32_t qdo_full = bar0;
-  auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + ST + s); };
-  auto s_full = [&](int b) { return bar0 + 8u * (1 + 2 * ST + b); };
-  auto ds_full = [&](int b) { return bar0 + 8u * (3 + 2 * ST + b); };
-  auto set_free = [&](int b) { return bar0 + 8u * (5 + 2 * ST + b); };
-  const uint32_t acc_done = bar0 + 8u * (7 + 2 * ST);
+  const uint32_t qdo_full = bar0, qdo_tmem = bar0 + 8u;
+  auto kv_full = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + ST + s); };
+  auto s_full = [&](int b) { return bar0 + 8u * (2 + 2 * ST + b); };
+  auto ds_full = [&](int b) { return bar0 + 8u * (4 + 2 * ST + b); };
+  const uint32_t acc_done = bar0 + 8u * (6 + 2 * ST);
+  const uint32_t acc_free = bar0 + 8u * (7 + 2 * ST);
   const uint32_t drain = bar0 + 8u * (8 + 2 * ST);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.T;
-  const int qt = p.n_t - 1 - (int)(blockIdx.x / p.BH);
-  const int bh = (int)(blockIdx.x % p.BH);
-  const int b = bh / p.H;
-  const int q0 = qt * kRows;
-  int kv_lo = 0;
-  if (p.doc) {
-    kv_lo = p.doc[(size_t)b * T + q0] / kRows;
-    kv_lo = kv_lo < 0 ? 0 : (kv_lo > qt ? qt : kv_lo);
-  }
-  const int n = qt - kv_lo + 1;   // key tiles
-  const int nh = 2 * n;           // key halves
+  const int w0 = blockIdx.x, dw = gridDim.x;
 
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
+    mbar_init(qdo_tmem, L::COMPUTE_WARPS);
     for (int s = 0; s < ST; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
@@ -442,9 +554,9 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
       mbar_init(ds_full(i), L::COMPUTE_WARPS);
-      mbar_init(set_free(i), 1);
     }
     mbar_init(acc_done, 1);
+    mbar_init(acc_free, L::COMPUTE_WARPS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -458,30 +570,47 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, p.wait_limit_ns};
-  const uint32_t tdQ = tmem + 256;
+  const uint32_t tdQ = tmem + L::T_DQ, tQ = tmem + L::T_Q, tdO = tmem + L::T_DO;
 
   if (warp == kProducerWarp) {
-    if (lane == 0) {
+    if (lane == 0) {  // Q / dO staging, one pair per item
       tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmdO);
+      int li = 0;
+      for (int k_ = 0; k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
+        const DqItem I = dq_item(p, w);
+        // the previous item's Q / dO must have been copied into TMEM
+        if (li >= 1 && !wait_bounded(qdo_tmem, (li - 1) & 1, g, 1)) break;
+        mbar_arrive_expect_tx(qdo_full, 2 * Tl::BYTES);
+        load_tile<D>(sQ, &tmQ, I.q0, I.bh, qdo_full);
+        load_tile<D>(sdO, &tmdO, I.q0, I.bh, qdo_full);
+        ++li;
+      }
+      if (*abort_flag && li > 0) drain_wait(qdo_full, (li - 1) & 1, p.wait_limit_ns);
+    } else if (lane == 1) {  // the K/V ring
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      tma_prefetch_desc(&tmdO);
-      mbar_arrive_expect_tx(qdo_full, 2 * Tl::BYTES);
-      load_tile<D>(sQ, &tmQ, q0, bh, qdo_full);
-      load_tile<D>(sdO, &tmdO, q0, bh, qdo_full);
-      int it = 0;
-      for (; it < n; ++it) {
-        const int s = it % ST, u = it / ST;
-        if (u > 0 && !wait_bounded(kv_empty(s), (u - 1) & 1, g, 1)) break;
-        const int row = (kv_lo + it) * kRows;
-        mbar_arrive_expect_tx(kv_full(s), 2 * Tl::BYTES);
-        load_tile<D>(sK(s), &tmK, row, bh, kv_full(s));
-        load_tile<D>(sV(s), &tmV, row, bh, kv_full(s));
+      int gk = 0;
+      bool ok = true;
+      for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
+        const DqItem I = dq_item(p, w);
+        for (int it = 0; it < I.n; ++it) {
+          const int s = gk % ST, u = gk / ST;
+          if (u > 0 && !wait_bounded(kv_empty(s), (u - 1) & 1, g, 1)) { ok = false; break; }
+          const int row = (I.kv_lo + it) * kRows;
+          mbar_arrive_expect_tx(kv_full(s), 2 * Tl::BYTES);
+          load_tile<D>(sK(s), &tmK, row, I.bh, kv_full(s));
+          load_tile<D>(sV(s), &tmV, row, I.bh, kv_full(s));
+          ++gk;
+        }
       }
       if (*abort_flag) {
-        drain_wait(qdo_full, 0, p.wait_limit_ns);
         for (int s = 0; s < ST; ++s) {
-          const int cnt = it > s ? (it - s + ST - 1) / ST : 0;
+          const int cnt = gk > s ? (gk - s + ST - 1) / ST : 0;
           if (cnt > 0) drain_wait(kv_full(s), (cnt - 1) & 1, p.wait_limit_ns);
         }
       }
@@ -491,97 +620,138 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, false);  // S, dP: M = queries, N = 64 keys
       constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);    // dQ: N = d, B (K) is MN-major
-      auto issue_grad = [&](int gp) -> bool {
-        const int bp = gp & 1, sp = (gp >> 1) % ST;
+      int li = 0, gk = 0, gh = 0;
+      auto issue_grad = [&](int gp, int sp, bool first) -> bool {
+        const int bp = gp & 1;
+        if (first && li >= 2 && !wait_bounded(acc_free, (li - 2) & 1, g, 4)) return false;
         if (!wait_bounded(ds_full(bp), (gp >> 1) & 1, g, 5)) return false;
         tc_fence_after();
         const uint32_t tset = tmem + 128u * bp;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tdQ, tset + 64u + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sK(sp), 4 * bp + kk),
-                 kIdG, (gp > 0 || kk > 0));
-        tc_commit(set_free(bp));
+                 kIdG, (!first || kk > 0));
         if (bp == 1) tc_commit(kv_empty(sp));
         return true;
       };
-      bool ok = wait_bounded(qdo_full, 0, g, 2);
-      for (int gh = 0; ok && gh < nh; ++gh) {
-        const int it = gh >> 1, h = gh & 1, s = it % ST;
-        if (h == 0 && !wait_bounded(kv_full(s), (it / ST) & 1, g, 3)) break;
-        // set h is reused: the dQ MMAs of half gh-2 must have finished reading it
-        if (gh >= 2 && !wait_bounded(set_free(h), ((gh - 2) >> 1) & 1, g, 4)) break;
-        tc_fence_after();
-        const uint32_t tset = tmem + 128u * h;
-        const uint32_t off = (uint32_t)(64 * h * Tl::SW);  // key rows 64h.. of the stage tile
+      bool ok = true;
+      for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
+        const DqItem I = dq_item(p, w);
+        // Q / dO of this item are in TMEM
+        if (!wait_bounded(qdo_tmem, li & 1, g, 2)) break;
+        ++li;
+        int prev_s = 0;
+        for (int it = 0; ok && it < I.n; ++it, ++gk) {
+          const int s = gk % ST;
+          if (!wait_bounded(kv_full(s), (gk / ST) & 1, g, 3)) { ok = false; break; }
+          for (int h = 0; h < 2; ++h, ++gh) {
+            tc_fence_after();
+            const uint32_t tset = tmem + 128u * h;
+            const uint32_t off = (uint32_t)(64 * h * Tl::SW);  // key rows 64h.. of the stage tile
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tset, desc_k<D>(sQ, kk), desc_k<D>(sK(s) + off, kk), kIdS, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ts(tset, tQ + 8u * kk, desc_k<D>(sK(s) + off, kk), kIdS, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tset + 64u, desc_k<D>(sdO, kk), desc_k<D>(sV(s) + off, kk), kIdS, kk > 0);
-        tc_commit(s_full(h));
-        if (gh >= 1 && !issue_grad(gh - 1)) { ok = false; break; }
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ts(tset + 64u, tdO + 8u * kk, desc_k<D>(sV(s) + off, kk), kIdS, kk > 0);
+            tc_commit(s_full(h));
+            if ((it > 0 || h > 0) && !issue_grad(gh - 1, h == 0 ? prev_s : s, it == 0 && h == 1)) {
+              ok = false;
+              break;
+            }
+          }
+          prev_s = s;
+        }
+        // the item's last half (never its first: that one was issued inside the loop)
+        if (ok && !issue_grad(gh - 1, prev_s, false)) ok = false;
+        if (ok) tc_commit(acc_done);
       }
-      if (ok) issue_grad(nh - 1);
-      tc_commit(acc_done);
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
     }
     __syncwarp();
   } else {
     const int qd = warp & 3, cs = warp >> 2;
-    const int r = q0 + qd * 32 + lane;  // query position owned by this thread
+    const int rl = qd * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const float sl2 = p.scale_log2;
-    // rows past T: -LSE = -inf makes every weight zero
-    const float nlse2 = (r < T) ? -p.lse[(size_t)bh * T + r] * kLog2e : -INFINITY;
-    const float ndlt = (r < T) ? -p.delta[(size_t)bh * T + r] : 0.f;
-    const int ds = p.doc ? p.doc[(size_t)b * T + (r < T ? r : T - 1)] : 0;
-    const uint64_t sl2x2 = f2(sl2, sl2), nlse2x2 = f2(nlse2, nlse2), ndltx2 = f2(ndlt, ndlt);
+    const uint64_t sl2x2 = f2(sl2, sl2);
     bool ok = true;
-    for (int gh = 0; gh < nh; ++gh) {
-      const int it = gh >> 1, h = gh & 1;
-      if (!wait_bounded_warp(s_full(h), (gh >> 1) & 1, g, 6)) { ok = false; break; }
-      tc_fence_after();
-      const int c0 = (kv_lo + it) * kRows + 64 * h + 32 * cs;  // first key of my columns
-      const uint32_t tS = tmem + lane_off + 128u * h + 32u * cs;
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tS, sr);
-      tmem_ld32(tS + 64u, dr);
-      tc_wait_ld();
-      reg_fence(sr);
-      reg_fence(dr);
-      if (!((c0 + 31 <= r) && (c0 >= ds))) {
-        const int hi = r - c0, lo = ds - c0;  // visible keys: e in [lo, hi]
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (e > hi || e < lo) sr[e] = 0xFF800000u;  // -inf: weight 0
+    int li = 0, gh = 0;
+    for (int k_ = 0; k_ * dw < p.n_items; ++k_, ++li) {
+      const int w = snake_item(k_, w0, dw, p.n_items);
+      if (w < 0) break;  // past the last item: no later round has one either
+      const DqItem I = dq_item(p, w);
+      const int r = I.q0 + rl;  // query position owned by this thread
+      // -------- Q (warps 0-3) / dO (warps 4-7) rows: shared memory -> TMEM.  The previous
+      // item's MMAs are all complete (its acc_done was waited for in its epilogue).
+      if (ok && wait_bounded_warp(qdo_full, li & 1, g, 9)) {
+        tile_row_to_tmem<D>(gsm + (cs ? L::DO_OFF : L::Q_OFF), rl, (cs ? tdO : tQ) + lane_off);
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(qdo_tmem);
+      } else {
+        ok = false;
       }
-      uint32_t dk[16];
+      // rows past T: -LSE = -inf makes every weight zero
+      const float nlse2 = (r < T) ? -p.lse[(size_t)I.bh * T + r] * kLog2e : -INFINITY;
+      const float ndlt = (r < T) ? -p.delta[(size_t)I.bh * T + r] : 0.f;
+      const int ds = p.doc ? p.doc[(size_t)I.b * T + (r < T ? r : T - 1)] : 0;
+      const uint64_t nlse2x2 = f2(nlse2, nlse2), ndltx2 = f2(ndlt, ndlt);
+      for (int it = 0; ok && it < I.n; ++it) {
+        for (int h = 0; h < 2; ++h, ++gh) {
+          if (!wait_bounded_warp(s_full(h), (gh >> 1) & 1, g, 6)) { ok = false; break; }
+          tc_fence_after();
+          const int c0 = (I.kv_lo + it) * kRows + 64 * h + 32 * cs;  // first key of my columns
+          const uint32_t tS = tmem + lane_off + 128u * h + 32u * cs;
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tS, sr);
+          tmem_ld32(tS + 64u, dr);
+          tc_wait_ld();
+          reg_fence(sr);
+          reg_fence(dr);
+          if (!((c0 + 31 <= r) && (c0 >= ds))) {
+            const int hi = r - c0, lo = ds - c0;  // visible keys: e in [lo, hi]
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        // P = exp2(S * scale * log2e - LSE * log2e);  dS = P * (dP - delta)
-        const float2 x = f2split(ffma2(f2u(sr[2 * e], sr[2 * e + 1]), sl2x2, nlse2x2));
-        const uint64_t p2 = f2(ex2(x.x), ex2(x.y));
-        const float2 d = f2split(fmul2(p2, fadd2(f2u(dr[2 * e], dr[2 * e + 1]), ndltx2)));
-        dk[e] = pack_bf16(d.x, d.y);
+            for (int e = 0; e < 32; ++e)
+              if (e > hi || e < lo) sr[e] = 0xFF800000u;  // -inf: weight 0
+          }
+          uint32_t dk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            // P = exp2(S * scale * log2e - LSE * log2e);  dS = P * (dP - delta)
+            const float2 x = f2split(ffma2(f2u(sr[2 * e], sr[2 * e + 1]), sl2x2, nlse2x2));
+            const uint64_t p2 = f2(ex2(x.x), ex2(x.y));
+            const float2 d = f2split(fmul2(p2, fadd2(f2u(dr[2 * e], dr[2 * e + 1]), ndltx2)));
+            dk[e] = pack_bf16(d.x, d.y);
+          }
+          tmem_st16(tS + 64u, dk);
+          tc_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(ds_full(h));
+        }
       }
-      tmem_st16(tS + 64u, dk);
-      tc_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full(h));
-    }
-    if (ok && wait_bounded_warp(acc_done, 0, g, 8)) {
-      tc_fence_after();
-      __nv_bfloat16* dq_row = p.g0 + ((size_t)bh * T + r) * D;
+      // ---------------------------------------------------------- epilogue
+      if (ok && wait_bounded_warp(acc_done, li & 1, g, 8)) {
+        tc_fence_after();
+        __nv_bfloat16* dq_row = p.g0 + ((size_t)I.bh * T + r) * D;
 #pragma unroll
-      for (int j = cs; j < D / 16; j += 2) {
-        uint32_t v[16];
-        tmem_ld16(tdQ + lane_off + 16u * j, v);
-        tc_wait_ld();
-        reg_fence16(v);
-        if (r < T) store16_bf16(dq_row + 16 * j, v, p.scale);
+        for (int j = cs; j < D / 16; j += 2) {
+          uint32_t v[16];
+          tmem_ld16(tdQ + lane_off + 16u * j, v);
+          tc_wait_ld();
+          reg_fence16(v);
+          if (r < T) store16_bf16(dq_row + 16 * j, v, p.scale);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_free);
+      } else {
+        ok = false;
       }
     }
   }

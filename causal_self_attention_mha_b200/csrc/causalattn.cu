@@ -211,10 +211,13 @@ int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const
   p.T = T;
   p.BH = BH;
   p.n_t = (T + ca::kRows - 1) / ca::kRows;
+  p.n_items = p.n_t * BH;
   p.scale = scale;
   p.scale_log2 = scale * ca::kLog2e;
   p.wait_limit_ns = kWaitLimitNs;
-  const unsigned grid = (unsigned)p.n_t * (unsigned)BH;
+  // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int sms = sm_count();
+  const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
   if (dkdv)
     ca::attn_bwd_dkdv_kernel<D>
         <<<grid, ca::DkdvLayout<D>::THREADS, ca::DkdvLayout<D>::SMEM, st>>>(mq, mk, mv, mdo, p);

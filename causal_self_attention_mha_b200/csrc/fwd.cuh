@@ -175,7 +175,9 @@ __global__ void __launch_bounds__(384, 1)
       int nq[2] = {0, 0};  // Q loads issued into buffer A / B
       int gk = 0;          // K loads issued
       bool ok = true;
-      for (int w = w0; ok && w < p.n_items; w += dw) {
+      for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
         const FwdItem I = fwd_item(p, w);
         for (int x = 0; x < 2; ++x) {
           if (x == 1 && !I.hasB) continue;
@@ -204,7 +206,9 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tmV);
       int gv = 0;
       bool ok = true;
-      for (int w = w0; ok && w < p.n_items; w += dw) {
+      for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
         const FwdItem I = fwd_item(p, w);
         for (int j = I.j_lo; j <= I.j_hi; ++j) {
           const int s = gv % STV, u = gv / STV;
@@ -252,7 +256,9 @@ __global__ void __launch_bounds__(384, 1)
         pend_t[x] = -1;
         return true;
       };
-      for (int w = w0; ok && w < p.n_items; w += dw) {
+      for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
         const FwdItem I = fwd_item(p, w);
         for (int x = 0; x < 2; ++x) {
           if (x == 1 && !I.hasB) continue;
@@ -304,7 +310,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t sl2x2 = f2(sl2, sl2);
     bool ok = true;
     int t = 0;   // tiles processed by this slot (s_full / p_full / o_done phases)
-    for (int w = w0; w < p.n_items; w += dw) {
+    for (int k_ = 0; k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
       const FwdItem I = fwd_item(p, w);
       if (x == 1 && !I.hasB) continue;
       const int row = I.qt[x] * kRows + rl;

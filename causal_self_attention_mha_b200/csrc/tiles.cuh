@@ -88,6 +88,15 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// Persistent work distribution: items are numbered heaviest first; CTA c of G
+// takes, in round k, item k*G + c for even k and k*G + (G-1-c) for odd k, so a
+// CTA that got one of the heavier items of a round gets one of the lighter
+// items of the next.  Returns -1 past the end.
+__device__ __forceinline__ int snake_item(int k, int c, int G, int n_items) {
+  const int w = k * G + ((k & 1) ? (G - 1 - c) : c);
+  return w < n_items ? w : -1;
+}
+
 // Shared-memory carve-up helper: 1024-byte aligned base inside dynamic smem.
 __device__ __forceinline__ uint32_t aligned_smem_base(const void* raw, uint8_t** generic) {
   const uint32_t a = smem_u32(raw);
