@@ -208,6 +208,22 @@ def run_reference(args, w, rank: int):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest `value` over all ranks (every rank gets it); plain value without a group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_value(step_flops: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every replica does step_flops per step; time is the slowest rank's."""
+    return world * step_flops / (ms_per_step * 1e-3) / 1e12
+
+
 def workload_config(w, parallelism):
     return {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} d={w.d}, "
                         f"{'document-causal' if w.doc_packed else 'causal'} mask",
@@ -297,11 +313,7 @@ def main():
     barrier()
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
-    elapsed_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
     per_kernel_ms = [0.0] * len(kernels)
     for ev in events:
         for j in range(len(kernels)):
@@ -327,17 +339,13 @@ def main():
         step_host.run(qh, kh, vh, doh, outs, w.scale, stream)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e_start.elapsed_time(e_end) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.e2e_steps, dev)
     barrier()
 
     if rank == 0:
         pk = peaks()
         ms_per_step = elapsed_ms / args.steps
-        value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+        value = replica_value(step_flops, world, ms_per_step)
         fwd_flops, bwd_flops = 4.0 * d * pairs, 10.0 * d * pairs
         fwd_ms = per_kernel_ms[0]
         bwd_ms = sum(per_kernel_ms[1:])
@@ -373,7 +381,7 @@ def main():
             "bwd_tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,
             "kernel_ms": dict(zip(kernels, per_kernel_ms)),
             "roofline": roof,
-            "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": replica_value(step_flops, world, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": step_host.h2d_bytes(),
                     "d2h_bytes_per_step": step_host.d2h_bytes(), "ms_per_step": e2e_ms},
             "gpu_launches": len(kernels) * args.steps,

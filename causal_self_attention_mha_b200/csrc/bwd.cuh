@@ -75,6 +75,25 @@ __device__ __forceinline__ void store16_bf16(__nv_bfloat16* dst, const uint32_t 
   d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
+// Half a row of a D-column fp32 TMEM accumulator (columns [half*D/2, (half+1)*D/2)
+// of this thread's lane), times `mul`, to bf16 in global memory: all TMEM loads
+// of the half row in flight together, one wait, then contiguous stores.
+template <int D>
+__device__ __forceinline__ void epilogue_rows(uint32_t tacc, __nv_bfloat16* row, int half,
+                                              bool store, float mul) {
+  constexpr int NC = (D / 2 + 15) / 16;  // 16-column chunks per half row
+  uint32_t r[NC][16];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) tmem_ld16(tacc + (uint32_t)(half * (D / 2) + 16 * c), r[c]);
+  tc_wait_ld();
+#pragma unroll
+  for (int c = 0; c < NC; ++c) reg_fence16(r[c]);
+  if (store) {
+#pragma unroll
+    for (int c = 0; c < NC; ++c) store16_bf16(row + half * (D / 2) + 16 * c, r[c], mul);
+  }
+}
+
 // Both tiled backward kernels are persistent: one CTA per SM walks work items
 // w = blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest first) and streams the
 // other operand in 64-row halves of its 128-row tiles (N = 64 for the S / dP
@@ -403,17 +422,9 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         __nv_bfloat16* dk_row = p.g0 + ((size_t)I.bh * T + c) * D;
         __nv_bfloat16* dv_row = p.g1 + ((size_t)I.bh * T + c) * D;
-        // 16-column jobs over (dV, dK), split between the two warps that share these lanes
-#pragma unroll
-        for (int j = cs; j < 2 * (D / 16); j += 2) {
-          const bool is_k = j >= D / 16;
-          const int col = 16 * (is_k ? j - D / 16 : j);
-          uint32_t r[16];
-          tmem_ld16((is_k ? tdK : tdV) + lane_off + col, r);
-          tc_wait_ld();
-          reg_fence16(r);
-          if (c < T) store16_bf16((is_k ? dk_row : dv_row) + col, r, is_k ? p.scale : 1.0f);
-        }
+        // the two warps sharing these lanes split the columns: [cs*D/2, (cs+1)*D/2) of dV and dK
+        epilogue_rows<D>(tdV + lane_off, dv_row, cs, c < T, 1.0f);
+        epilogue_rows<D>(tdK + lane_off, dk_row, cs, c < T, p.scale);
         // dV / dK have been read: the next item's first gradient MMA may overwrite them
         tc_fence_before();
         __syncwarp();
@@ -439,14 +450,17 @@ __global__ void __launch_bounds__(320, 1)
 // half from shared memory.
 template <int D>
 struct DqLayout {
-  static constexpr int ST = (D == 128) ? 2 : 3;   // K/V ring depth (128-row tiles)
+  // K is read by S (first) and by dQ (last), V only by dP: separate rings, K deeper
+  static constexpr int STK = (D == 128) ? 3 : 4;  // K ring depth (128-row tiles)
+  static constexpr int STV = (D == 128) ? 2 : 3;  // V ring depth
   static constexpr int Q_OFF = 0;                  // Q, dO staging for the TMEM copy
   static constexpr int DO_OFF = Q_OFF + Tile<D>::BYTES;
   static constexpr int K_OFF = DO_OFF + Tile<D>::BYTES;           // + s * BYTES
-  static constexpr int V_OFF = K_OFF + ST * Tile<D>::BYTES;       // + s * BYTES
-  static constexpr int BAR_OFF = V_OFF + ST * Tile<D>::BYTES;
-  // barriers: qdo_full qdo_tmem | kv_full[ST] kv_empty[ST] | s_full[2] ds_full[2] | acc_done acc_free drain
-  static constexpr int NBAR = 2 + 2 * ST + 4 + 3;
+  static constexpr int V_OFF = K_OFF + STK * Tile<D>::BYTES;      // + s * BYTES
+  static constexpr int BAR_OFF = V_OFF + STV * Tile<D>::BYTES;
+  // barriers: qdo_full qdo_tmem | k_full[STK] k_empty[STK] | v_full[STV] v_empty[STV] |
+  //           s_full[2] ds_full[2] | acc_done acc_free drain
+  static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 4 + 3;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
@@ -520,7 +534,7 @@ __global__ void __launch_bounds__(320, 1)
                        const __grid_constant__ CUtensorMap tmdO, const BwdParams p) {
   using Tl = Tile<D>;
   using L = DqLayout<D>;
-  constexpr int ST = L::ST;
+  constexpr int STK = L::STK, STV = L::STV;
   constexpr int kProducerWarp = L::COMPUTE_WARPS, kMmaWarp = L::COMPUTE_WARPS + 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* gsm;
@@ -530,13 +544,16 @@ __global__ void __launch_bounds__(320, 1)
   auto sV = [&](int s) { return sbase + L::V_OFF + s * Tl::BYTES; };
   const uint32_t bar0 = sbase + L::BAR_OFF;
   const uint32_t qdo_full = bar0, qdo_tmem = bar0 + 8u;
-  auto kv_full = [&](int s) { return bar0 + 8u * (2 + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + ST + s); };
-  auto s_full = [&](int b) { return bar0 + 8u * (2 + 2 * ST + b); };
-  auto ds_full = [&](int b) { return bar0 + 8u * (4 + 2 * ST + b); };
-  const uint32_t acc_done = bar0 + 8u * (6 + 2 * ST);
-  const uint32_t acc_free = bar0 + 8u * (7 + 2 * ST);
-  const uint32_t drain = bar0 + 8u * (8 + 2 * ST);
+  auto k_full = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto k_empty = [&](int s) { return bar0 + 8u * (2 + STK + s); };
+  auto v_full = [&](int s) { return bar0 + 8u * (2 + 2 * STK + s); };
+  auto v_empty = [&](int s) { return bar0 + 8u * (2 + 2 * STK + STV + s); };
+  const uint32_t xb = bar0 + 8u * (2 + 2 * STK + 2 * STV);
+  auto s_full = [&](int b) { return xb + 8u * b; };
+  auto ds_full = [&](int b) { return xb + 8u * (2 + b); };
+  const uint32_t acc_done = xb + 8u * 4;
+  const uint32_t acc_free = xb + 8u * 5;
+  const uint32_t drain = xb + 8u * 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -547,9 +564,13 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
     mbar_init(qdo_tmem, L::COMPUTE_WARPS);
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+    for (int s = 0; s < STK; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+    }
+    for (int s = 0; s < STV; ++s) {
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
@@ -589,9 +610,11 @@ __global__ void __launch_bounds__(320, 1)
         ++li;
       }
       if (*abort_flag && li > 0) drain_wait(qdo_full, (li - 1) & 1, p.wait_limit_ns);
-    } else if (lane == 1) {  // the K/V ring
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+    } else if (lane == 1 || lane == 2) {  // lane 1: the K ring, lane 2: the V ring
+      const bool isK = (lane == 1);
+      const int NS = isK ? STK : STV;
+      const CUtensorMap* tm = isK ? &tmK : &tmV;
+      tma_prefetch_desc(tm);
       int gk = 0;
       bool ok = true;
       for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
@@ -599,19 +622,21 @@ __global__ void __launch_bounds__(320, 1)
         if (w < 0) break;  // past the last item: no later round has one either
         const DqItem I = dq_item(p, w);
         for (int it = 0; it < I.n; ++it) {
-          const int s = gk % ST, u = gk / ST;
-          if (u > 0 && !wait_bounded(kv_empty(s), (u - 1) & 1, g, 1)) { ok = false; break; }
-          const int row = (I.kv_lo + it) * kRows;
-          mbar_arrive_expect_tx(kv_full(s), 2 * Tl::BYTES);
-          load_tile<D>(sK(s), &tmK, row, I.bh, kv_full(s));
-          load_tile<D>(sV(s), &tmV, row, I.bh, kv_full(s));
+          const int s = gk % NS, u = gk / NS;
+          const uint32_t full = isK ? k_full(s) : v_full(s);
+          if (u > 0 && !wait_bounded(isK ? k_empty(s) : v_empty(s), (u - 1) & 1, g, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full, Tl::BYTES);
+          load_tile<D>(isK ? sK(s) : sV(s), tm, (I.kv_lo + it) * kRows, I.bh, full);
           ++gk;
         }
       }
       if (*abort_flag) {
-        for (int s = 0; s < ST; ++s) {
-          const int cnt = gk > s ? (gk - s + ST - 1) / ST : 0;
-          if (cnt > 0) drain_wait(kv_full(s), (cnt - 1) & 1, p.wait_limit_ns);
+        for (int s = 0; s < NS; ++s) {
+          const int cnt = gk > s ? (gk - s + NS - 1) / NS : 0;
+          if (cnt > 0) drain_wait(isK ? k_full(s) : v_full(s), (cnt - 1) & 1, p.wait_limit_ns);
         }
       }
     }
@@ -631,7 +656,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tdQ, tset + 64u + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sK(sp), 4 * bp + kk),
                  kIdG, (!first || kk > 0));
-        if (bp == 1) tc_commit(kv_empty(sp));
+        if (bp == 1) tc_commit(k_empty(sp));  // K of this key tile no longer read
         return true;
       };
       bool ok = true;
@@ -644,8 +669,12 @@ __global__ void __launch_bounds__(320, 1)
         ++li;
         int prev_s = 0;
         for (int it = 0; ok && it < I.n; ++it, ++gk) {
-          const int s = gk % ST;
-          if (!wait_bounded(kv_full(s), (gk / ST) & 1, g, 3)) { ok = false; break; }
+          const int s = gk % STK, sv = gk % STV;
+          if (!wait_bounded(k_full(s), (gk / STK) & 1, g, 3) ||
+              !wait_bounded(v_full(sv), (gk / STV) & 1, g, 3)) {
+            ok = false;
+            break;
+          }
           for (int h = 0; h < 2; ++h, ++gh) {
             tc_fence_after();
             const uint32_t tset = tmem + 128u * h;
@@ -655,8 +684,9 @@ __global__ void __launch_bounds__(320, 1)
               mma_ts(tset, tQ + 8u * kk, desc_k<D>(sK(s) + off, kk), kIdS, kk > 0);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              mma_ts(tset + 64u, tdO + 8u * kk, desc_k<D>(sV(s) + off, kk), kIdS, kk > 0);
+              mma_ts(tset + 64u, tdO + 8u * kk, desc_k<D>(sV(sv) + off, kk), kIdS, kk > 0);
             tc_commit(s_full(h));
+            if (h == 1) tc_commit(v_empty(sv));  // V of this key tile no longer read
             if ((it > 0 || h > 0) && !issue_grad(gh - 1, h == 0 ? prev_s : s, it == 0 && h == 1)) {
               ok = false;
               break;
@@ -739,14 +769,7 @@ __global__ void __launch_bounds__(320, 1)
       if (ok && wait_bounded_warp(acc_done, li & 1, g, 8)) {
         tc_fence_after();
         __nv_bfloat16* dq_row = p.g0 + ((size_t)I.bh * T + r) * D;
-#pragma unroll
-        for (int j = cs; j < D / 16; j += 2) {
-          uint32_t v[16];
-          tmem_ld16(tdQ + lane_off + 16u * j, v);
-          tc_wait_ld();
-          reg_fence16(v);
-          if (r < T) store16_bf16(dq_row + 16 * j, v, p.scale);
-        }
+        epilogue_rows<D>(tdQ + lane_off, dq_row, cs, r < T, p.scale);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_free);

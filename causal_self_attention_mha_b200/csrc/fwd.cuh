@@ -52,7 +52,7 @@ struct FwdParams {
 
 template <int D>
 struct FwdLayout {
-  static constexpr int STK = (D == 128) ? 2 : 4;            // K ring depth
+  static constexpr int STK = (D == 128) ? 3 : 4;            // K ring depth
   static constexpr int STV = (D == 128) ? 2 : 3;            // V ring depth
   static constexpr int Q_OFF = 0;                            // Q_A, Q_B
   static constexpr int K_OFF = Q_OFF + 2 * Tile<D>::BYTES;
@@ -330,25 +330,37 @@ __global__ void __launch_bounds__(384, 1)
         if (!wait_bounded_warp(s_full(x), t & 1, g, 8)) { ok = false; break; }
         // s_full(t) also means PV(t-1) has completed: O_x may be read and rescaled
         tc_fence_after();
+        // two load waves: the max over the first 64 columns overlaps the second wave
         uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32u * c, sr[c]);
+        tmem_ld32(tS, sr[0]);
+        tmem_ld32(tS + 32u, sr[1]);
         tc_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
-        if (!((c0 + kRows - 1 <= row) && (c0 >= ds))) {
-          const int hi = row - c0, lo = ds - c0;  // visible keys: e in [lo, hi]
-#pragma unroll
-          for (int e = 0; e < 128; ++e)
-            if (e > hi || e < lo) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf
-        }
+        reg_fence(sr[0]);
+        reg_fence(sr[1]);
+        tmem_ld32(tS + 64u, sr[2]);
+        tmem_ld32(tS + 96u, sr[3]);
+        const bool need_mask = !((c0 + kRows - 1 <= row) && (c0 >= ds));
+        const int hi = row - c0, lo = ds - c0;  // visible keys: e in [lo, hi]
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int e = 0; e < 128; e += 8)
+        for (int half = 0; half < 2; ++half) {
+          if (half == 1) {
+            tc_wait_ld();
+            reg_fence(sr[2]);
+            reg_fence(sr[3]);
+          }
+          if (need_mask) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            mx4[q] = fmax3(mx4[q], __uint_as_float(sr[(e + 2 * q) >> 5][(e + 2 * q) & 31]),
-                           __uint_as_float(sr[(e + 2 * q + 1) >> 5][(e + 2 * q + 1) & 31]));
+            for (int e = 64 * half; e < 64 * half + 64; ++e)
+              if (e > hi || e < lo) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf
+          }
+#pragma unroll
+          for (int e = 64 * half; e < 64 * half + 64; e += 8)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              mx4[q] = fmax3(mx4[q], __uint_as_float(sr[(e + 2 * q) >> 5][(e + 2 * q) & 31]),
+                             __uint_as_float(sr[(e + 2 * q + 1) >> 5][(e + 2 * q + 1) & 31]));
+        }
         const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
         const float m_new = fmaxf(m, mx);
         const bool grow = m_new > m + 8.0f;  // also true the first time a row sees a key
@@ -415,13 +427,20 @@ __global__ void __launch_bounds__(384, 1)
         if (row < T) p.lse[(size_t)I.bh * T + row] = (mu + lg2(l)) * kLn2;
         const float inv = 1.0f / lr;
         __nv_bfloat16* orow = p.o + ((size_t)I.bh * T + row) * D;
+        // the row in up to two waves of (at most) 64 columns: loads in flight together
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + 32u * c, r);
+        for (int w2 = 0; w2 < (D + 63) / 64; ++w2) {
+          constexpr int NC = (D >= 64) ? 2 : 1;
+          uint32_t r[NC][32];
+#pragma unroll
+          for (int c = 0; c < NC; ++c) tmem_ld32(tO + 64u * w2 + 32u * c, r[c]);
           tc_wait_ld();
-          reg_fence(r);
-          if (row < T) store_row_chunk_bf16(orow + 32 * c, r, inv);
+#pragma unroll
+          for (int c = 0; c < NC; ++c) reg_fence(r[c]);
+          if (row < T) {
+#pragma unroll
+            for (int c = 0; c < NC; ++c) store_row_chunk_bf16(orow + 64 * w2 + 32 * c, r[c], inv);
+          }
         }
         // O_x has been read: the next item's first PV may overwrite it
         tc_fence_before();
