@@ -94,21 +94,26 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tacc, __nv_bfloat16* row,
   }
 }
 
+
 // Both tiled backward kernels are persistent: one CTA per SM walks work items
-// w = blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest first) and streams the
-// other operand in 64-row halves of its 128-row tiles (N = 64 for the S / dP
-// products).  Half g uses TMEM "set" g % 2: its S (or S^T) in columns
-// [128*set, +64) and dP (or dP^T) in [128*set + 64, +64), so the MMAs of half
-// g+1 run while the 8 element-wise warps work on half g.  A set is reused two
-// halves later by the next S / dP MMAs, which the single in-order MMA stream
-// issues after the gradient MMAs that read it.  Element-wise warp w owns TMEM
-// lanes 32*(w%4).. and columns 32*(w/4).. of each half; it writes its bf16 P /
-// dS (16 packed columns) over the first half of the fp32 columns it has just
-// read.  At an item boundary the gradient accumulators are handed over with
-// acc_done (MMA -> epilogue) and acc_free (epilogue -> next item's first
-// gradient MMA).
+// (serpentine, heaviest first) and streams the partner operand through a ring
+// of whole 128-row tiles, so every S / dP product is one M=128, N=128 MMA
+// chain.  384 threads = three warpgroups: warpgroups 0-1 are the element-wise
+// warps (warp w owns TMEM lanes 32*(w%4).. and columns 64*(w/4).. of each
+// tile), the third holds the TMA producer and the single MMA-issuing thread;
+// registers are rebalanced with setmaxnreg (168 at launch; 208 for the
+// element-wise warpgroups, 88 for the third).  An element-wise thread keeps its
+// 64 fp32 P values in registers while it waits for dP.  P and dS go back to
+// TMEM as packed bf16 over the first half of the columns the same warp has
+// just read, and feed the gradient MMAs as their A operand.  At an item
+// boundary the gradient accumulators are handed over with acc_done (MMA ->
+// epilogue) and acc_free (epilogue -> next item's first gradient MMA).
 
 // ------------------------------------------------------------------ dK/dV
+// TMEM: S^T (keys x 128 queries) at 0, dP^T at 128, dV at 256, dK at 256 + D.
+// MMA stream per query tile t:  dV(t), S^T(t+1), dK(t), dP^T(t+1).  S^T(t+1)
+// overwrites P^T(t) only after dV(t) in the in-order stream (likewise dP^T(t+1)
+// after dK(t)), and it runs while the element-wise warps finish dS^T(t).
 template <int D>
 struct DkdvLayout {
   static constexpr int ST = (D == 128) ? 2 : 3;   // Q/dO ring depth (128-row tiles)
@@ -119,14 +124,16 @@ struct DkdvLayout {
   static constexpr int VEC_OFF = DO_OFF + ST * Tile<D>::BYTES;     // per stage: -lse2, -delta, dsq
   static constexpr int VEC_STAGE = 3 * kRows * 4;
   static constexpr int BAR_OFF = VEC_OFF + ST * VEC_STAGE;
-  // barriers: kv_full kv_empty | q_full[ST] q_empty[ST] | st_full[2] pds_full[2] | acc_done acc_free drain
+  // barriers: kv_full kv_empty | q_full[ST] q_empty[ST] | st_full dpt_full p_ready ds_ready |
+  //           acc_done acc_free drain
   static constexpr int NBAR = 2 + 2 * ST + 4 + 3;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem slot, abort flag
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
   static constexpr int COMPUTE_WARPS = 8;
-  static constexpr int THREADS = (COMPUTE_WARPS + 2) * 32;
+  static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 256 + D;
 };
 
 struct DkdvItem {
@@ -159,7 +166,7 @@ __device__ __forceinline__ DkdvItem dkdv_item(const BwdParams& p, int w) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
@@ -179,11 +186,9 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t kv_full = bar0, kv_empty = bar0 + 8u;
   auto q_full = [&](int s) { return bar0 + 8u * (2 + s); };
   auto q_empty = [&](int s) { return bar0 + 8u * (2 + ST + s); };
-  auto st_full = [&](int b) { return bar0 + 8u * (2 + 2 * ST + b); };
-  auto pds_full = [&](int b) { return bar0 + 8u * (4 + 2 * ST + b); };
-  const uint32_t acc_done = bar0 + 8u * (6 + 2 * ST);
-  const uint32_t acc_free = bar0 + 8u * (7 + 2 * ST);
-  const uint32_t drain = bar0 + 8u * (8 + 2 * ST);
+  const uint32_t xb = bar0 + 8u * (2 + 2 * ST);
+  const uint32_t st_full = xb, dpt_full = xb + 8u, p_ready = xb + 16u, ds_ready = xb + 24u;
+  const uint32_t acc_done = xb + 32u, acc_free = xb + 40u, drain = xb + 48u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -198,10 +203,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(q_full(s), 32);
       mbar_init(q_empty(s), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(st_full(i), 1);
-      mbar_init(pds_full(i), L::COMPUTE_WARPS);
-    }
+    mbar_init(st_full, 1);
+    mbar_init(dpt_full, 1);
+    mbar_init(p_ready, L::COMPUTE_WARPS);
+    mbar_init(ds_ready, L::COMPUTE_WARPS);
     mbar_init(acc_done, 1);
     mbar_init(acc_free, L::COMPUTE_WARPS);
     mbar_init(drain, 1);
@@ -217,8 +222,9 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, p.wait_limit_ns};
-  const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D;
 
+  if (warp >= L::COMPUTE_WARPS) {
+    regs_shrink<88>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -230,10 +236,10 @@ __global__ void __launch_bounds__(320, 1)
     int li = 0, gq = 0;  // items whose K/V were loaded, query tiles loaded
     bool ok = true;
     for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
-        const int w = snake_item(k_, w0, dw, p.n_items);
-        if (w < 0) break;  // past the last item: no later round has one either
+      const int w = snake_item(k_, w0, dw, p.n_items);
+      if (w < 0) break;  // past the last item: no later round has one either
       const DkdvItem I = dkdv_item(p, w);
-      // K/V of this item: the previous item's last S^T / dP^T MMAs must be done with them
+      // K/V of this item: the previous item's MMAs must be done with the old ones
       if (li >= 1 && !wait_bounded_warp(kv_empty, (li - 1) & 1, g, 1)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(kv_full, 2 * Tl::BYTES);
@@ -282,149 +288,194 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, false);  // S^T, dP^T: M = keys, N = 64 queries
-      constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);    // dV, dK: N = d, B is MN-major
-      int li = 0, gq = 0, gh = 0;  // items, query tiles, query halves consumed
-      // dV += P^T dO and dK += dS^T Q for global half gp (K = 64 queries, 4 MMA-K steps);
-      // `first`: first half of its item (accumulators start from zero)
-      auto issue_grad = [&](int gp, int sp, bool first) -> bool {
-        const int bp = gp & 1;
-        // the first gradient MMA of an item overwrites dV / dK: the previous epilogue must be done
-        if (first && li >= 2 && !wait_bounded(acc_free, (li - 2) & 1, g, 4)) return false;
-        if (!wait_bounded(pds_full(bp), (gp >> 1) & 1, g, 5)) return false;
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false);  // S^T, dP^T: M = keys, N = queries
+      constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);     // dV, dK: N = d, B is MN-major
+      const uint32_t tST = tmem + L::T_ST, tDPT = tmem + L::T_DPT;
+      const uint32_t tdV = tmem + L::T_DV, tdK = tmem + L::T_DK;
+      auto issue_st = [&](int s) {  // S^T = K Q_s^T
         tc_fence_after();
-        const uint32_t tset = tmem + 128u * bp;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tdV, tset + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sdO(sp), 4 * bp + kk), kIdG,
-                 (!first || kk > 0));
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tdK, tset + 64u + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sQ(sp), 4 * bp + kk),
-                 kIdG, (!first || kk > 0));
-        if (bp == 1) tc_commit(q_empty(sp));
-        return true;
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tST, desc_k<D>(sK, kk), desc_k<D>(sQ(s), kk), kIdS, kk > 0);
+        tc_commit(st_full);
       };
+      auto issue_dpt = [&](int s) {  // dP^T = V dO_s^T
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tDPT, desc_k<D>(sV, kk), desc_k<D>(sdO(s), kk), kIdS, kk > 0);
+        tc_commit(dpt_full);
+      };
+      int li = 0, gq = 0;
       bool ok = true;
       for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
         const int w = snake_item(k_, w0, dw, p.n_items);
         if (w < 0) break;  // past the last item: no later round has one either
         const DkdvItem I = dkdv_item(p, w);
         if (!wait_bounded(kv_full, li & 1, g, 2)) break;
-        ++li;
-        int prev_s = 0;
-        for (int it = 0; ok && it < I.n; ++it, ++gq) {
-          const int s = gq % ST;
-          if (!wait_bounded(q_full(s), (gq / ST) & 1, g, 3)) { ok = false; break; }
-          for (int h = 0; h < 2; ++h, ++gh) {
-            tc_fence_after();
-            const uint32_t tset = tmem + 128u * h;
-            const uint32_t off = (uint32_t)(64 * h * Tl::SW);  // query rows 64h.. of the stage tile
+        const int s0 = gq % ST;
+        if (!wait_bounded(q_full(s0), (gq / ST) & 1, g, 3)) break;
+        issue_st(s0);
+        issue_dpt(s0);
+        if (I.n == 1) tc_commit(kv_empty);  // K, V of this item no longer read after these
+        for (int it = 0; it < I.n; ++it, ++gq) {
+          const int t = gq, s = t % ST;
+          // dV += P^T dO: the first one of an item overwrites dV, so the previous
+          // item's epilogue must have read it
+          if (it == 0 && li >= 1 && !wait_bounded(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
+          if (!wait_bounded(p_ready, t & 1, g, 5)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tset, desc_k<D>(sK, kk), desc_k<D>(sQ(s) + off, kk), kIdS, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_ss(tset + 64u, desc_k<D>(sV, kk), desc_k<D>(sdO(s) + off, kk), kIdS, kk > 0);
-            tc_commit(st_full(h));
-            if (it == I.n - 1 && h == 1) tc_commit(kv_empty);  // K, V of this item no longer read
-            if ((it > 0 || h > 0) && !issue_grad(gh - 1, h == 0 ? prev_s : s, it == 0 && h == 1)) {
-              ok = false;
-              break;
-            }
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            mma_ts(tdV, tST + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sdO(s), kk), kIdG,
+                   (it > 0 || kk > 0));
+          const bool more = it + 1 < I.n;
+          const int s1 = (t + 1) % ST;
+          if (more) {  // S^T of the next query tile, behind dV(t) in the stream
+            if (!wait_bounded(q_full(s1), ((t + 1) / ST) & 1, g, 3)) { ok = false; break; }
+            issue_st(s1);
           }
-          prev_s = s;
+          if (!wait_bounded(ds_ready, t & 1, g, 6)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            mma_ts(tdK, tDPT + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sQ(s), kk), kIdG,
+                   (it > 0 || kk > 0));
+          tc_commit(q_empty(s));  // Q_t, dO_t no longer read
+          if (more) {
+            issue_dpt(s1);
+            if (it + 2 == I.n) tc_commit(kv_empty);  // that was the item's last S^T / dP^T
+          }
         }
-        // the item's last half (never its first: that one was issued inside the loop)
-        if (ok && !issue_grad(gh - 1, prev_s, false)) ok = false;
-        if (ok) tc_commit(acc_done);
+        if (!ok) break;
+        tc_commit(acc_done);
+        ++li;
       }
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
     }
     __syncwarp();
+  }
   } else {
+    regs_grow<208>();
     // ------------------------------------------- P^T / dS^T (thread = key row)
     const int qd = warp & 3, cs = warp >> 2;
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    const uint32_t tS = tmem + lane_off + L::T_ST + 64u * cs;   // my 64 columns of S^T
+    const uint32_t tD = tmem + lane_off + L::T_DPT + 64u * cs;  // ... and of dP^T
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2(sl2, sl2);
     bool ok = true;
-    int li = 0, gq = 0, gh = 0;
+    int li = 0, gq = 0;
     for (int k_ = 0; k_ * dw < p.n_items; ++k_, ++li) {
-        const int w = snake_item(k_, w0, dw, p.n_items);
-        if (w < 0) break;  // past the last item: no later round has one either
+      const int w = snake_item(k_, w0, dw, p.n_items);
+      if (w < 0) break;  // past the last item: no later round has one either
       const DkdvItem I = dkdv_item(p, w);
       const int c = I.k0 + qd * 32 + lane;  // key position owned by this thread
       for (int it = 0; ok && it < I.n; ++it, ++gq) {
-        const int s = gq % ST;
-        for (int h = 0; h < 2; ++h, ++gh) {
-          if (!wait_bounded_warp(st_full(h), (gh >> 1) & 1, g, 6)) { ok = false; break; }
-          if (!wait_bounded_warp(q_full(s), (gq / ST) & 1, g, 7)) { ok = false; break; }
-          tc_fence_after();
-          const float* lse2 = vec + s * 3 * kRows;
-          const float* dl = lse2 + kRows;
-          const int* dsq = reinterpret_cast<const int*>(dl + kRows);
-          const int rb = 64 * h + 32 * cs;                 // first query row (in the tile) of my columns
-          const int r0 = (I.i_lo + it) * kRows + rb;       // its position
-          const uint32_t tS = tmem + lane_off + 128u * h + 32u * cs;
-          uint32_t sr[32], dr[32];
-          tmem_ld32(tS, sr);
-          tmem_ld32(tS + 64u, dr);
-          tc_wait_ld();
-          reg_fence(sr);
-          reg_fence(dr);
-          // no mask needed when all my query rows are at or below this key and their
-          // documents start at or before it (dsq is nondecreasing; huge past T)
-          if (!((r0 >= c) && (dsq[rb + 31] <= c))) {
-            const int4* ds4 = reinterpret_cast<const int4*>(dsq + rb);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const int4 dv4 = ds4[q4];
-              const int dsv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int e = 4 * q4 + k;
-                if (c > r0 + e || c < dsv[k]) sr[e] = 0xFF800000u;  // -inf: weight 0
-              }
-            }
-          }
-          const float4* l4 = reinterpret_cast<const float4*>(lse2 + rb);  // -LSE*log2(e)
-          const float4* d4 = reinterpret_cast<const float4*>(dl + rb);    // -delta
-          uint32_t pk[16], dk[16];
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 lv = l4[q4], dv4 = d4[q4];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int e = 4 * q4 + 2 * h2;
-              const uint64_t nl = h2 ? f2(lv.z, lv.w) : f2(lv.x, lv.y);
-              const uint64_t nd = h2 ? f2(dv4.z, dv4.w) : f2(dv4.x, dv4.y);
-              // P^T = exp2(S^T * scale * log2e - LSE * log2e);  dS^T = P^T * (dP^T - delta)
-              const float2 x = f2split(ffma2(f2u(sr[e], sr[e + 1]), sl2x2, nl));
-              const float p0 = ex2(x.x), p1 = ex2(x.y);
-              const float2 dd = f2split(fmul2(f2(p0, p1), fadd2(f2u(dr[e], dr[e + 1]), nd)));
-              pk[e >> 1] = pack_bf16(p0, p1);
-              dk[e >> 1] = pack_bf16(dd.x, dd.y);
-            }
-          }
-          tmem_st16(tS, pk);
-          tmem_st16(tS + 64u, dk);
-          tc_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(pds_full(h));
+        const int t = gq, s = t % ST;
+        if (!wait_bounded_warp(st_full, t & 1, g, 7) ||
+            !wait_bounded_warp(q_full(s), (t / ST) & 1, g, 7)) {
+          ok = false;
+          break;
         }
-        if (!ok) break;
+        tc_fence_after();
+        const float* lse2 = vec + s * 3 * kRows;
+        const float* dl = lse2 + kRows;
+        const int* dsq = reinterpret_cast<const int*>(dl + kRows);
+        const int rb = 64 * cs;                       // first query row (in the tile) of my columns
+        const int r0 = (I.i_lo + it) * kRows + rb;    // its position
+        uint32_t sr[2][32];
+        tmem_ld32(tS, sr[0]);
+        tmem_ld32(tS + 32u, sr[1]);
+        tc_wait_ld();
+        reg_fence(sr[0]);
+        reg_fence(sr[1]);
+        // no mask needed when all my query rows are at or below this key and their
+        // documents start at or before it (dsq is nondecreasing; huge past T)
+        if (!((r0 >= c) && (dsq[rb + 63] <= c))) {
+          const int4* ds4 = reinterpret_cast<const int4*>(dsq + rb);
+#pragma unroll
+          for (int q4 = 0; q4 < 16; ++q4) {
+            const int4 dv4 = ds4[q4];
+            const int dsv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = 4 * q4 + k;
+              if (c > r0 + e || c < dsv[k]) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf: weight 0
+            }
+          }
+        }
+        // P^T = exp2(S^T * scale * log2e - LSE * log2e), kept in fp32 for dS^T
+        const float4* l4 = reinterpret_cast<const float4*>(lse2 + rb);  // -LSE*log2(e)
+        float pf[64];
+        uint32_t pk[32];
+#pragma unroll
+        for (int q4 = 0; q4 < 16; ++q4) {
+          const float4 lv = l4[q4];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 4 * q4 + 2 * h2;
+            const uint64_t nl = h2 ? f2(lv.z, lv.w) : f2(lv.x, lv.y);
+            const float2 x =
+                f2split(ffma2(f2u(sr[e >> 5][e & 31], sr[e >> 5][(e & 31) + 1]), sl2x2, nl));
+            pf[e] = ex2(x.x);
+            pf[e + 1] = ex2(x.y);
+            pk[e >> 1] = pack_bf16(pf[e], pf[e + 1]);
+          }
+        }
+        {
+          uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pk[0]);
+          uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pk[16]);
+          tmem_st16(tS, lo);
+          tmem_st16(tS + 16u, hi);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_ready);
+        // dS^T = P^T * (dP^T - delta)
+        if (!wait_bounded_warp(dpt_full, t & 1, g, 8)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t dr[2][32];
+        tmem_ld32(tD, dr[0]);
+        tmem_ld32(tD + 32u, dr[1]);
+        tc_wait_ld();
+        reg_fence(dr[0]);
+        reg_fence(dr[1]);
+        const float4* d4 = reinterpret_cast<const float4*>(dl + rb);  // -delta
+        uint32_t dk[32];
+#pragma unroll
+        for (int q4 = 0; q4 < 16; ++q4) {
+          const float4 dv4 = d4[q4];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 4 * q4 + 2 * h2;
+            const uint64_t nd = h2 ? f2(dv4.z, dv4.w) : f2(dv4.x, dv4.y);
+            const float2 dd = f2split(fmul2(
+                f2(pf[e], pf[e + 1]), fadd2(f2u(dr[e >> 5][e & 31], dr[e >> 5][(e & 31) + 1]), nd)));
+            dk[e >> 1] = pack_bf16(dd.x, dd.y);
+          }
+        }
+        {
+          uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dk[0]);
+          uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dk[16]);
+          tmem_st16(tD, lo);
+          tmem_st16(tD + 16u, hi);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_ready);
       }
       // ---------------------------------------------------------- epilogue
-      if (ok && wait_bounded_warp(acc_done, li & 1, g, 8)) {
+      if (ok && wait_bounded_warp(acc_done, li & 1, g, 9)) {
         tc_fence_after();
         __nv_bfloat16* dk_row = p.g0 + ((size_t)I.bh * T + c) * D;
         __nv_bfloat16* dv_row = p.g1 + ((size_t)I.bh * T + c) * D;
-        // the two warps sharing these lanes split the columns: [cs*D/2, (cs+1)*D/2) of dV and dK
-        epilogue_rows<D>(tdV + lane_off, dv_row, cs, c < T, 1.0f);
-        epilogue_rows<D>(tdK + lane_off, dk_row, cs, c < T, p.scale);
+        // the two warps sharing these lanes split the columns: [cs*D/2, (cs+1)*D/2)
+        epilogue_rows<D>(tmem + lane_off + L::T_DV, dv_row, cs, c < T, 1.0f);
+        epilogue_rows<D>(tmem + lane_off + L::T_DK, dk_row, cs, c < T, p.scale);
         // dV / dK have been read: the next item's first gradient MMA may overwrite them
         tc_fence_before();
         __syncwarp();
@@ -444,31 +495,31 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // --------------------------------------------------------------------- dQ
-// Q and dO are the stationary operands of the dQ kernel: they are staged in
-// shared memory by TMA and then copied, once per item, into TMEM, so S = Q K^T
-// and dP = dO V^T run as TMEM-operand MMAs that read only the streamed K / V
-// half from shared memory.
+// Q and dO of the item's query tile stay in shared memory; K and V stream
+// through rings of their own (K is read by S and by dQ, V only by dP).
+// TMEM: S double-buffered at 0 / 128, dP at 256 (dS is written back over its
+// first half), dQ at 384.  MMA stream per key tile t:  dQ(t), dP(t+1), S(t+2):
+// S(t+1) is ready before the element-wise warps need it, and the only
+// tensor-core work they wait for is dP.
 template <int D>
 struct DqLayout {
-  // K is read by S (first) and by dQ (last), V only by dP: separate rings, K deeper
   static constexpr int STK = (D == 128) ? 3 : 4;  // K ring depth (128-row tiles)
   static constexpr int STV = (D == 128) ? 2 : 3;  // V ring depth
-  static constexpr int Q_OFF = 0;                  // Q, dO staging for the TMEM copy
+  static constexpr int Q_OFF = 0;
   static constexpr int DO_OFF = Q_OFF + Tile<D>::BYTES;
   static constexpr int K_OFF = DO_OFF + Tile<D>::BYTES;           // + s * BYTES
   static constexpr int V_OFF = K_OFF + STK * Tile<D>::BYTES;      // + s * BYTES
   static constexpr int BAR_OFF = V_OFF + STV * Tile<D>::BYTES;
-  // barriers: qdo_full qdo_tmem | k_full[STK] k_empty[STK] | v_full[STV] v_empty[STV] |
-  //           s_full[2] ds_full[2] | acc_done acc_free drain
+  // barriers: qdo_full qdo_empty | k_full[STK] k_empty[STK] | v_full[STV] v_empty[STV] |
+  //           s_full[2] dp_full ds_full | acc_done acc_free drain
   static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 4 + 3;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
   static constexpr int COMPUTE_WARPS = 8;
-  static constexpr int THREADS = (COMPUTE_WARPS + 2) * 32;
+  static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
-  // TMEM columns: sets at 0 and 128, dQ at 256, Q at 256 + D, dO at 256 + 3D/2
-  static constexpr uint32_t T_DQ = 256, T_Q = 256 + D, T_DO = 256 + D + D / 2;
+  static constexpr uint32_t T_S = 0, T_DP = 256, T_DQ = 384;
 };
 
 struct DqItem {
@@ -483,7 +534,7 @@ __device__ __forceinline__ DqItem dq_item(const BwdParams& p, int w) {
   I.b = I.bh / p.H;
   I.q0 = I.qt * kRows;
   I.kv_lo = 0;
-  if (p.doc) {
+  if (p.doc) {  // no key before the document start of the tile's first row is visible
     const int lo = p.doc[(size_t)I.b * p.T + I.q0] / kRows;
     I.kv_lo = lo < 0 ? 0 : (lo > I.qt ? I.qt : lo);
   }
@@ -491,45 +542,10 @@ __device__ __forceinline__ DqItem dq_item(const BwdParams& p, int w) {
   return I;
 }
 
-// Copy row `rl` of a TMA-swizzled 128-row tile from shared memory into TMEM
-// (this thread's lane) as packed bf16 pairs: D/2 columns starting at `taddr`.
-// The hardware swizzle puts 16-byte granule g of row r at g ^ (r & 7) (128-byte
-// rows) or g ^ ((r >> 1) & 3) (64-byte rows).
 template <int D>
-__device__ __forceinline__ void tile_row_to_tmem(const uint8_t* tile, int rl, uint32_t taddr) {
-  using Tl = Tile<D>;
-#pragma unroll
-  for (int c = 0; c < Tl::CHUNKS; ++c) {
-    const uint8_t* row = tile + c * Tl::CHUNK_BYTES + rl * Tl::SW;
-    if constexpr (Tl::SW == 128) {
-      uint32_t r[32];
-#pragma unroll
-      for (int gi = 0; gi < 8; ++gi) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + ((gi ^ (rl & 7)) * 16));
-        r[4 * gi] = v.x;
-        r[4 * gi + 1] = v.y;
-        r[4 * gi + 2] = v.z;
-        r[4 * gi + 3] = v.w;
-      }
-      tmem_st32(taddr + 32u * c, r);
-    } else {
-      uint32_t r[16];
-#pragma unroll
-      for (int gi = 0; gi < 4; ++gi) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + ((gi ^ ((rl >> 1) & 3)) * 16));
-        r[4 * gi] = v.x;
-        r[4 * gi + 1] = v.y;
-        r[4 * gi + 2] = v.z;
-        r[4 * gi + 3] = v.w;
-      }
-      tmem_st16(taddr + 16u * c, r);
-    }
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(320, 1)
-    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(384, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmdO, const BwdParams p) {
   using Tl = Tile<D>;
@@ -543,17 +559,15 @@ __global__ void __launch_bounds__(320, 1)
   auto sK = [&](int s) { return sbase + L::K_OFF + s * Tl::BYTES; };
   auto sV = [&](int s) { return sbase + L::V_OFF + s * Tl::BYTES; };
   const uint32_t bar0 = sbase + L::BAR_OFF;
-  const uint32_t qdo_full = bar0, qdo_tmem = bar0 + 8u;
+  const uint32_t qdo_full = bar0, qdo_empty = bar0 + 8u;
   auto k_full = [&](int s) { return bar0 + 8u * (2 + s); };
   auto k_empty = [&](int s) { return bar0 + 8u * (2 + STK + s); };
   auto v_full = [&](int s) { return bar0 + 8u * (2 + 2 * STK + s); };
   auto v_empty = [&](int s) { return bar0 + 8u * (2 + 2 * STK + STV + s); };
   const uint32_t xb = bar0 + 8u * (2 + 2 * STK + 2 * STV);
   auto s_full = [&](int b) { return xb + 8u * b; };
-  auto ds_full = [&](int b) { return xb + 8u * (2 + b); };
-  const uint32_t acc_done = xb + 8u * 4;
-  const uint32_t acc_free = xb + 8u * 5;
-  const uint32_t drain = xb + 8u * 6;
+  const uint32_t dp_full = xb + 16u, ds_full = xb + 24u;
+  const uint32_t acc_done = xb + 32u, acc_free = xb + 40u, drain = xb + 48u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -563,7 +577,7 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
-    mbar_init(qdo_tmem, L::COMPUTE_WARPS);
+    mbar_init(qdo_empty, 1);
     for (int s = 0; s < STK; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
@@ -572,10 +586,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(v_full(s), 1);
       mbar_init(v_empty(s), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full(i), 1);
-      mbar_init(ds_full(i), L::COMPUTE_WARPS);
-    }
+    mbar_init(s_full(0), 1);
+    mbar_init(s_full(1), 1);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, L::COMPUTE_WARPS);
     mbar_init(acc_done, 1);
     mbar_init(acc_free, L::COMPUTE_WARPS);
     mbar_init(drain, 1);
@@ -591,10 +605,12 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, p.wait_limit_ns};
-  const uint32_t tdQ = tmem + L::T_DQ, tQ = tmem + L::T_Q, tdO = tmem + L::T_DO;
 
+  if (warp >= L::COMPUTE_WARPS) {
+    regs_shrink<88>();
   if (warp == kProducerWarp) {
-    if (lane == 0) {  // Q / dO staging, one pair per item
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {  // Q / dO, one pair per item
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmdO);
       int li = 0;
@@ -602,8 +618,8 @@ __global__ void __launch_bounds__(320, 1)
         const int w = snake_item(k_, w0, dw, p.n_items);
         if (w < 0) break;  // past the last item: no later round has one either
         const DqItem I = dq_item(p, w);
-        // the previous item's Q / dO must have been copied into TMEM
-        if (li >= 1 && !wait_bounded(qdo_tmem, (li - 1) & 1, g, 1)) break;
+        // the previous item's S / dP MMAs must be done with the old Q / dO
+        if (li >= 1 && !wait_bounded(qdo_empty, (li - 1) & 1, g, 1)) break;
         mbar_arrive_expect_tx(qdo_full, 2 * Tl::BYTES);
         load_tile<D>(sQ, &tmQ, I.q0, I.bh, qdo_full);
         load_tile<D>(sdO, &tmdO, I.q0, I.bh, qdo_full);
@@ -633,7 +649,7 @@ __global__ void __launch_bounds__(320, 1)
           ++gk;
         }
       }
-      if (*abort_flag) {
+      if (*abort_flag) {  // let every copy already issued land before the CTA exits
         for (int s = 0; s < NS; ++s) {
           const int cnt = gk > s ? (gk - s + NS - 1) / NS : 0;
           if (cnt > 0) drain_wait(isK ? k_full(s) : v_full(s), (cnt - 1) & 1, p.wait_limit_ns);
@@ -642,134 +658,152 @@ __global__ void __launch_bounds__(320, 1)
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
+    // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(128, 64, false);  // S, dP: M = queries, N = 64 keys
-      constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);    // dQ: N = d, B (K) is MN-major
-      int li = 0, gk = 0, gh = 0;
-      auto issue_grad = [&](int gp, int sp, bool first) -> bool {
-        const int bp = gp & 1;
-        if (first && li >= 2 && !wait_bounded(acc_free, (li - 2) & 1, g, 4)) return false;
-        if (!wait_bounded(ds_full(bp), (gp >> 1) & 1, g, 5)) return false;
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false);  // S, dP: M = queries, N = keys
+      constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);     // dQ: N = d, B (K) is MN-major
+      const uint32_t tDP = tmem + L::T_DP, tdQ = tmem + L::T_DQ;
+      auto issue_s = [&](int t) -> bool {  // S(t) = Q K_t^T into buffer t & 1
+        const int s = t % STK;
+        if (!wait_bounded(k_full(s), (t / STK) & 1, g, 3)) return false;
         tc_fence_after();
-        const uint32_t tset = tmem + 128u * bp;
+        const uint32_t tS = tmem + L::T_S + 128u * (uint32_t)(t & 1);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tdQ, tset + 64u + 32u * (kk >> 1) + 8u * (kk & 1), desc_mn<D>(sK(sp), 4 * bp + kk),
-                 kIdG, (!first || kk > 0));
-        if (bp == 1) tc_commit(k_empty(sp));  // K of this key tile no longer read
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tS, desc_k<D>(sQ, kk), desc_k<D>(sK(s), kk), kIdS, kk > 0);
+        tc_commit(s_full(t & 1));
         return true;
       };
+      auto issue_dp = [&](int t) -> bool {  // dP(t) = dO V_t^T
+        const int s = t % STV;
+        if (!wait_bounded(v_full(s), (t / STV) & 1, g, 3)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tDP, desc_k<D>(sdO, kk), desc_k<D>(sV(s), kk), kIdS, kk > 0);
+        tc_commit(dp_full);
+        tc_commit(v_empty(s));  // V of this key tile no longer read
+        return true;
+      };
+      int li = 0, gk = 0;
       bool ok = true;
       for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
         const int w = snake_item(k_, w0, dw, p.n_items);
         if (w < 0) break;  // past the last item: no later round has one either
         const DqItem I = dq_item(p, w);
-        // Q / dO of this item are in TMEM
-        if (!wait_bounded(qdo_tmem, li & 1, g, 2)) break;
-        ++li;
-        int prev_s = 0;
-        for (int it = 0; ok && it < I.n; ++it, ++gk) {
-          const int s = gk % STK, sv = gk % STV;
-          if (!wait_bounded(k_full(s), (gk / STK) & 1, g, 3) ||
-              !wait_bounded(v_full(sv), (gk / STV) & 1, g, 3)) {
-            ok = false;
-            break;
-          }
-          for (int h = 0; h < 2; ++h, ++gh) {
-            tc_fence_after();
-            const uint32_t tset = tmem + 128u * h;
-            const uint32_t off = (uint32_t)(64 * h * Tl::SW);  // key rows 64h.. of the stage tile
+        if (!wait_bounded(qdo_full, li & 1, g, 2)) break;
+        const int t0 = gk;
+        ok = issue_s(t0) && issue_dp(t0);
+        if (ok && I.n == 1) tc_commit(qdo_empty);  // Q, dO of this item no longer read
+        if (ok && I.n > 1) ok = issue_s(t0 + 1);
+        for (int it = 0; ok && it < I.n; ++it) {
+          const int t = t0 + it;
+          // the first dQ MMA of an item overwrites dQ: the previous epilogue must have read it
+          if (it == 0 && li >= 1 && !wait_bounded(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
+          if (!wait_bounded(ds_full, t & 1, g, 5)) { ok = false; break; }
+          tc_fence_after();
+          const int s = t % STK;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_ts(tset, tQ + 8u * kk, desc_k<D>(sK(s) + off, kk), kIdS, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_ts(tset + 64u, tdO + 8u * kk, desc_k<D>(sV(sv) + off, kk), kIdS, kk > 0);
-            tc_commit(s_full(h));
-            if (h == 1) tc_commit(v_empty(sv));  // V of this key tile no longer read
-            if ((it > 0 || h > 0) && !issue_grad(gh - 1, h == 0 ? prev_s : s, it == 0 && h == 1)) {
-              ok = false;
-              break;
-            }
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            mma_ts(tdQ, tDP + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sK(s), kk), kIdG,
+                   (it > 0 || kk > 0));
+          tc_commit(k_empty(s));  // K of this key tile no longer read
+          if (it + 1 < I.n) {
+            if (!issue_dp(t + 1)) { ok = false; break; }
+            if (it + 2 == I.n) tc_commit(qdo_empty);  // that was the item's last S / dP
           }
-          prev_s = s;
+          if (it + 2 < I.n && !issue_s(t + 2)) { ok = false; break; }
         }
-        // the item's last half (never its first: that one was issued inside the loop)
-        if (ok && !issue_grad(gh - 1, prev_s, false)) ok = false;
-        if (ok) tc_commit(acc_done);
+        if (!ok) break;
+        gk += I.n;
+        tc_commit(acc_done);
+        ++li;
       }
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
     }
     __syncwarp();
+  }
   } else {
+    regs_grow<208>();
+    // ----------------------------------------------- P / dS (thread = query row)
     const int qd = warp & 3, cs = warp >> 2;
     const int rl = qd * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    const uint32_t tD = tmem + lane_off + L::T_DP + 64u * cs;  // my 64 columns of dP
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2(sl2, sl2);
     bool ok = true;
-    int li = 0, gh = 0;
-    for (int k_ = 0; k_ * dw < p.n_items; ++k_, ++li) {
+    int li = 0, gk = 0;
+    for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_, ++li) {
       const int w = snake_item(k_, w0, dw, p.n_items);
       if (w < 0) break;  // past the last item: no later round has one either
       const DqItem I = dq_item(p, w);
       const int r = I.q0 + rl;  // query position owned by this thread
-      // -------- Q (warps 0-3) / dO (warps 4-7) rows: shared memory -> TMEM.  The previous
-      // item's MMAs are all complete (its acc_done was waited for in its epilogue).
-      if (ok && wait_bounded_warp(qdo_full, li & 1, g, 9)) {
-        tile_row_to_tmem<D>(gsm + (cs ? L::DO_OFF : L::Q_OFF), rl, (cs ? tdO : tQ) + lane_off);
-        tc_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(qdo_tmem);
-      } else {
-        ok = false;
-      }
       // rows past T: -LSE = -inf makes every weight zero
       const float nlse2 = (r < T) ? -p.lse[(size_t)I.bh * T + r] * kLog2e : -INFINITY;
       const float ndlt = (r < T) ? -p.delta[(size_t)I.bh * T + r] : 0.f;
       const int ds = p.doc ? p.doc[(size_t)I.b * T + (r < T ? r : T - 1)] : 0;
       const uint64_t nlse2x2 = f2(nlse2, nlse2), ndltx2 = f2(ndlt, ndlt);
-      for (int it = 0; ok && it < I.n; ++it) {
-        for (int h = 0; h < 2; ++h, ++gh) {
-          if (!wait_bounded_warp(s_full(h), (gh >> 1) & 1, g, 6)) { ok = false; break; }
-          tc_fence_after();
-          const int c0 = (I.kv_lo + it) * kRows + 64 * h + 32 * cs;  // first key of my columns
-          const uint32_t tS = tmem + lane_off + 128u * h + 32u * cs;
-          uint32_t sr[32], dr[32];
-          tmem_ld32(tS, sr);
-          tmem_ld32(tS + 64u, dr);
-          tc_wait_ld();
-          reg_fence(sr);
-          reg_fence(dr);
-          if (!((c0 + 31 <= r) && (c0 >= ds))) {
-            const int hi = r - c0, lo = ds - c0;  // visible keys: e in [lo, hi]
+      for (int it = 0; it < I.n; ++it, ++gk) {
+        const int t = gk;
+        if (!wait_bounded_warp(s_full(t & 1), (t >> 1) & 1, g, 6)) { ok = false; break; }
+        tc_fence_after();
+        const int c0 = (I.kv_lo + it) * kRows + 64 * cs;  // first key of my columns
+        const uint32_t tS = tmem + lane_off + L::T_S + 128u * (uint32_t)(t & 1) + 64u * cs;
+        uint32_t sr[2][32];
+        tmem_ld32(tS, sr[0]);
+        tmem_ld32(tS + 32u, sr[1]);
+        tc_wait_ld();
+        reg_fence(sr[0]);
+        reg_fence(sr[1]);
+        if (!((c0 + 63 <= r) && (c0 >= ds))) {
+          const int hi = r - c0, lo = ds - c0;  // visible keys: e in [lo, hi]
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (e > hi || e < lo) sr[e] = 0xFF800000u;  // -inf: weight 0
-          }
-          uint32_t dk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            // P = exp2(S * scale * log2e - LSE * log2e);  dS = P * (dP - delta)
-            const float2 x = f2split(ffma2(f2u(sr[2 * e], sr[2 * e + 1]), sl2x2, nlse2x2));
-            const uint64_t p2 = f2(ex2(x.x), ex2(x.y));
-            const float2 d = f2split(fmul2(p2, fadd2(f2u(dr[2 * e], dr[2 * e + 1]), ndltx2)));
-            dk[e] = pack_bf16(d.x, d.y);
-          }
-          tmem_st16(tS + 64u, dk);
-          tc_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(ds_full(h));
+          for (int e = 0; e < 64; ++e)
+            if (e > hi || e < lo) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf: weight 0
         }
+        // P = exp2(S * scale * log2e - LSE * log2e), kept in fp32 until dP arrives
+        float pf[64];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          const float2 x =
+              f2split(ffma2(f2u(sr[e >> 5][e & 31], sr[e >> 5][(e & 31) + 1]), sl2x2, nlse2x2));
+          pf[e] = ex2(x.x);
+          pf[e + 1] = ex2(x.y);
+        }
+        if (!wait_bounded_warp(dp_full, t & 1, g, 7)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t dr[2][32];
+        tmem_ld32(tD, dr[0]);
+        tmem_ld32(tD + 32u, dr[1]);
+        tc_wait_ld();
+        reg_fence(dr[0]);
+        reg_fence(dr[1]);
+        // dS = P * (dP - delta), bf16, over the first 32 of my dP columns
+        uint32_t dk[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          const float2 d = f2split(fmul2(
+              f2(pf[e], pf[e + 1]), fadd2(f2u(dr[e >> 5][e & 31], dr[e >> 5][(e & 31) + 1]), ndltx2)));
+          dk[e >> 1] = pack_bf16(d.x, d.y);
+        }
+        {
+          uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dk[0]);
+          uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dk[16]);
+          tmem_st16(tD, lo);
+          tmem_st16(tD + 16u, hi);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full);
       }
       // ---------------------------------------------------------- epilogue
       if (ok && wait_bounded_warp(acc_done, li & 1, g, 8)) {
         tc_fence_after();
         __nv_bfloat16* dq_row = p.g0 + ((size_t)I.bh * T + r) * D;
-        epilogue_rows<D>(tdQ + lane_off, dq_row, cs, r < T, p.scale);
+        epilogue_rows<D>(tmem + lane_off + L::T_DQ, dq_row, cs, r < T, p.scale);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_free);
