@@ -64,36 +64,25 @@ struct BwdParams {
 };
 
 
-// Store 16 fp32 values (one TMEM x16 chunk of a row), times `mul`, as 16 bf16 to global.
-__device__ __forceinline__ void store16_bf16(__nv_bfloat16* dst, const uint32_t (&r)[16], float mul) {
-  uint32_t pk[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e)
-    pk[e] = pack_bf16(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-  d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-}
-
 // Half a row of a D-column fp32 TMEM accumulator (columns [half*D/2, (half+1)*D/2)
-// of this thread's lane), times `mul`, to bf16 in global memory: all TMEM loads
-// of the half row in flight together, one wait, then contiguous stores.
+// of this thread's lane), times `mul`, as packed bf16 pairs: all TMEM loads in
+// flight together, one wait.
 template <int D>
-__device__ __forceinline__ void epilogue_rows(uint32_t tacc, __nv_bfloat16* row, int half,
-                                              bool store, float mul) {
-  constexpr int NC = (D / 2 + 15) / 16;  // 16-column chunks per half row
+__device__ __forceinline__ void tmem_half_row_bf16(uint32_t tacc, int half, float mul,
+                                                   uint32_t (&w)[D / 4]) {
+  constexpr int NC = D / 32;  // 16-column chunks per half row
   uint32_t r[NC][16];
 #pragma unroll
   for (int c = 0; c < NC; ++c) tmem_ld16(tacc + (uint32_t)(half * (D / 2) + 16 * c), r[c]);
   tc_wait_ld();
 #pragma unroll
   for (int c = 0; c < NC; ++c) reg_fence16(r[c]);
-  if (store) {
 #pragma unroll
-    for (int c = 0; c < NC; ++c) store16_bf16(row + half * (D / 2) + 16 * c, r[c], mul);
-  }
+  for (int c = 0; c < NC; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      w[8 * c + e] = pack_bf16(__uint_as_float(r[c][2 * e]) * mul, __uint_as_float(r[c][2 * e + 1]) * mul);
 }
-
 
 // Both tiled backward kernels are persistent: one CTA per SM walks work items
 // (serpentine, heaviest first) and streams the partner operand through a ring
@@ -113,23 +102,34 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tacc, __nv_bfloat16* row,
 // TMEM: S^T (keys x 128 queries) at 0, dP^T at 128, dV at 256, dK at 256 + D.
 // MMA stream per query tile t:  dV(t), S^T(t+1), dK(t), dP^T(t+1).  S^T(t+1)
 // overwrites P^T(t) only after dV(t) in the in-order stream (likewise dP^T(t+1)
-// after dK(t)), and it runs while the element-wise warps finish dS^T(t).
+// after dK(t)), and it runs while the element-wise warps finish dS^T(t).  dV(t)
+// starts on the first half of P^T(t) while the second half is still being
+// computed.  The per-row vectors -LSE*log2(e) and -delta ride with the dO
+// stages.  dV and dK leave through one staged bf16 tile in shared memory and
+// TMA stores issued by warp 10: row-per-thread global stores from every SM at
+// the same item boundary congest the memory system for microseconds.
 template <int D>
 struct DkdvLayout {
-  static constexpr int ST = (D == 128) ? 2 : 3;   // Q/dO ring depth (128-row tiles)
+  static constexpr int QST = (D == 128) ? 2 : 3;  // Q ring depth (128-row tiles)
+  static constexpr int DST = (D == 128) ? 2 : 3;  // dO ring depth
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + Tile<D>::BYTES;
   static constexpr int Q_OFF = V_OFF + Tile<D>::BYTES;             // + s * BYTES
-  static constexpr int DO_OFF = Q_OFF + ST * Tile<D>::BYTES;       // + s * BYTES
-  static constexpr int VEC_OFF = DO_OFF + ST * Tile<D>::BYTES;     // per stage: -lse2, -delta, dsq
-  static constexpr int VEC_STAGE = 3 * kRows * 4;
-  static constexpr int BAR_OFF = VEC_OFF + ST * VEC_STAGE;
-  // barriers: kv_full kv_empty | q_full[ST] q_empty[ST] | st_full dpt_full p_ready ds_ready |
-  //           acc_done acc_free drain
-  static constexpr int NBAR = 2 + 2 * ST + 4 + 3;
+  static constexpr int DO_OFF = Q_OFF + QST * Tile<D>::BYTES;      // + s * BYTES
+  static constexpr int VEC_OFF = DO_OFF + DST * Tile<D>::BYTES;    // per dO stage: -lse2, -delta
+  static constexpr int VEC_STAGE = 2 * kRows * 4;
+  static constexpr int STG_OFF = VEC_OFF + DST * VEC_STAGE;       // output staging tile
+  static constexpr int BAR_OFF = STG_OFF + Tile<D>::BYTES;
+  // barriers: kv_full kv_empty | q_full[QST] q_empty[QST] | do_full[DST] do_empty[DST]
+  //           vec_full[DST] | st_full dpt_full p_ready[2] ds_ready | acc_done acc_free drain |
+  //           stg_full stg_free
+  static constexpr int NBAR = 2 + 2 * QST + 3 * DST + 5 + 3 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;   // tmem slot, abort flag
   static constexpr int BYTES = MISC_OFF + 16;
-  static constexpr int SMEM = BYTES + 1024;
+  static_assert(BYTES <= kMaxDynSmem, "dK/dV shared-memory layout");
+  // room to round the base up to 1 KB where the opt-in limit leaves it (the
+  // kernel checks the rounded layout against what it was given)
+  static constexpr int SMEM = (BYTES + 1024 <= kMaxDynSmem) ? BYTES + 1024 : kMaxDynSmem;
   static constexpr int COMPUTE_WARPS = 8;
   static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -165,30 +165,63 @@ __device__ __forceinline__ DkdvItem dkdv_item(const BwdParams& p, int w) {
   return I;
 }
 
+// Number of the 64 query rows r0 .. r0+63 that lie in key c's document or an
+// earlier one (and before T): those rows form a prefix because document starts
+// never decrease.  Lane l holds the document start of rows r0 + l and
+// r0 + 32 + l (INT_MAX past T); the search runs on shuffles, so every lane of
+// the warp must call it.
+__device__ __forceinline__ int rows_in_doc_prefix(int a, int b, int c) {
+  int n = 0;
+#pragma unroll
+  for (int step = 32; step >= 1; step >>= 1) {
+    const int probe = n + step - 1;
+    const int va = __shfl_sync(0xffffffffu, a, probe & 31);
+    const int vb = __shfl_sync(0xffffffffu, b, probe & 31);
+    if ((probe < 32 ? va : vb) <= c) n += step;
+  }
+  const int va = __shfl_sync(0xffffffffu, a, n & 31);
+  const int vb = __shfl_sync(0xffffffffu, b, n & 31);
+  if (n < 64 && (n < 32 ? va : vb) <= c) ++n;
+  return n;
+}
+
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
-                         const __grid_constant__ CUtensorMap tmdO, const BwdParams p) {
+                         const __grid_constant__ CUtensorMap tmdO,
+                         const __grid_constant__ CUtensorMap tmdK,
+                         const __grid_constant__ CUtensorMap tmdV, const BwdParams p) {
   using Tl = Tile<D>;
   using L = DkdvLayout<D>;
-  constexpr int ST = L::ST;
+  constexpr int QST = L::QST, DST = L::DST;
   constexpr int kProducerWarp = L::COMPUTE_WARPS, kMmaWarp = L::COMPUTE_WARPS + 1;
+  constexpr int kStoreWarp = L::COMPUTE_WARPS + 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* gsm;
   const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
+  if (sbase - smem_u32(smem_raw) + L::BYTES > dynamic_smem_bytes()) {
+    if (threadIdx.x == 0) report_smem_shortfall();
+    return;  // uniform across the CTA, before any barrier
+  }
   const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF;
   auto sQ = [&](int s) { return sbase + L::Q_OFF + s * Tl::BYTES; };
   auto sdO = [&](int s) { return sbase + L::DO_OFF + s * Tl::BYTES; };
-  float* vec = reinterpret_cast<float*>(gsm + L::VEC_OFF);   // [ST][3][128]
+  float* vec = reinterpret_cast<float*>(gsm + L::VEC_OFF);   // [DST][2][128]
   const uint32_t bar0 = sbase + L::BAR_OFF;
   const uint32_t kv_full = bar0, kv_empty = bar0 + 8u;
   auto q_full = [&](int s) { return bar0 + 8u * (2 + s); };
-  auto q_empty = [&](int s) { return bar0 + 8u * (2 + ST + s); };
-  const uint32_t xb = bar0 + 8u * (2 + 2 * ST);
-  const uint32_t st_full = xb, dpt_full = xb + 8u, p_ready = xb + 16u, ds_ready = xb + 24u;
-  const uint32_t acc_done = xb + 32u, acc_free = xb + 40u, drain = xb + 48u;
+  auto q_empty = [&](int s) { return bar0 + 8u * (2 + QST + s); };
+  auto do_full = [&](int s) { return bar0 + 8u * (2 + 2 * QST + s); };
+  auto do_empty = [&](int s) { return bar0 + 8u * (2 + 2 * QST + DST + s); };
+  auto vec_full = [&](int s) { return bar0 + 8u * (2 + 2 * QST + 2 * DST + s); };
+  const uint32_t xb = bar0 + 8u * (2 + 2 * QST + 3 * DST);
+  const uint32_t st_full = xb, dpt_full = xb + 8u, ds_ready = xb + 16u;
+  auto p_ready = [&](int h) { return xb + 24u + 8u * h; };  // P^T query columns [32h, 32h+32) of each warp
+  const uint32_t acc_done = xb + 40u, acc_free = xb + 48u, drain = xb + 56u;
+  const uint32_t stg_full = xb + 64u, stg_free = xb + 72u;  // output staging tile handshake
+  const uint32_t sStg = sbase + L::STG_OFF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -197,15 +230,23 @@ __global__ void __launch_bounds__(384, 1)
   const int w0 = blockIdx.x, dw = gridDim.x;
 
   if (threadIdx.x == 0) {
+    mbar_init(stg_full, L::COMPUTE_WARPS);
+    mbar_init(stg_free, 1);
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(q_full(s), 32);
+    for (int s = 0; s < QST; ++s) {
+      mbar_init(q_full(s), 1);
       mbar_init(q_empty(s), 1);
+    }
+    for (int s = 0; s < DST; ++s) {
+      mbar_init(do_full(s), 1);
+      mbar_init(do_empty(s), 1);
+      mbar_init(vec_full(s), 32);
     }
     mbar_init(st_full, 1);
     mbar_init(dpt_full, 1);
-    mbar_init(p_ready, L::COMPUTE_WARPS);
+    mbar_init(p_ready(0), L::COMPUTE_WARPS);
+    mbar_init(p_ready(1), L::COMPUTE_WARPS);
     mbar_init(ds_ready, L::COMPUTE_WARPS);
     mbar_init(acc_done, 1);
     mbar_init(acc_free, L::COMPUTE_WARPS);
@@ -248,40 +289,46 @@ __global__ void __launch_bounds__(384, 1)
       }
       ++li;
       for (int it = 0; it < I.n; ++it) {
-        const int s = gq % ST, u = gq / ST;
-        if (u > 0 && !wait_bounded_warp(q_empty(s), (u - 1) & 1, g, 1)) { ok = false; break; }
+        const int t = gq;
         const int r0 = (I.i_lo + it) * kRows;
-        float* lse2 = vec + s * 3 * kRows;
+        const int sq = t % QST, uq = t / QST;
+        if (uq > 0 && !wait_bounded_warp(q_empty(sq), (uq - 1) & 1, g, 1)) { ok = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full(sq), Tl::BYTES);
+          load_tile<D>(sQ(sq), &tmQ, r0, I.bh, q_full(sq));
+        }
+        const int sd = t % DST, ud = t / DST;
+        if (ud > 0 && !wait_bounded_warp(do_empty(sd), (ud - 1) & 1, g, 1)) { ok = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(do_full(sd), Tl::BYTES);
+          load_tile<D>(sdO(sd), &tmdO, r0, I.bh, do_full(sd));
+        }
+        float* lse2 = vec + sd * 2 * kRows;
         float* dl = lse2 + kRows;
-        int* dsq = reinterpret_cast<int*>(dl + kRows);
 #pragma unroll
         for (int k = 0; k < kRows / 32; ++k) {
           const int rl = lane + 32 * k, r = r0 + rl;
           if (r < T) {  // stored negated: -LSE*log2(e) and -delta
             lse2[rl] = -p.lse[(size_t)I.bh * T + r] * kLog2e;
             dl[rl] = -p.delta[(size_t)I.bh * T + r];
-            dsq[rl] = p.doc ? p.doc[(size_t)I.b * T + r] : 0;
-          } else {  // rows past the end: no key is visible
+          } else {  // rows past the end: every weight is zero
             lse2[rl] = -INFINITY;
             dl[rl] = 0.f;
-            dsq[rl] = 0x7fffffff;
           }
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(q_full(s), 2 * Tl::BYTES);
-          load_tile<D>(sQ(s), &tmQ, r0, I.bh, q_full(s));
-          load_tile<D>(sdO(s), &tmdO, r0, I.bh, q_full(s));
-        } else {
-          mbar_arrive(q_full(s));
-        }
+        mbar_arrive(vec_full(sd));
         ++gq;
       }
     }
     if (lane == 0 && *abort_flag) {  // let every copy already issued land before the CTA exits
       if (li > 0) drain_wait(kv_full, (li - 1) & 1, p.wait_limit_ns);
-      for (int s = 0; s < ST; ++s) {
-        const int cnt = gq > s ? (gq - s + ST - 1) / ST : 0;
+      for (int s = 0; s < QST; ++s) {
+        const int cnt = gq > s ? (gq - s + QST - 1) / QST : 0;
         if (cnt > 0) drain_wait(q_full(s), (cnt - 1) & 1, p.wait_limit_ns);
+      }
+      for (int s = 0; s < DST; ++s) {
+        const int cnt = gq > s ? (gq - s + DST - 1) / DST : 0;
+        if (cnt > 0) drain_wait(do_full(s), (cnt - 1) & 1, p.wait_limit_ns);
       }
     }
     __syncwarp();
@@ -292,19 +339,25 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);     // dV, dK: N = d, B is MN-major
       const uint32_t tST = tmem + L::T_ST, tDPT = tmem + L::T_DPT;
       const uint32_t tdV = tmem + L::T_DV, tdK = tmem + L::T_DK;
-      auto issue_st = [&](int s) {  // S^T = K Q_s^T
+      auto issue_st = [&](int t) -> bool {  // S^T = K Q_t^T
+        const int s = t % QST;
+        if (!wait_bounded(q_full(s), (t / QST) & 1, g, 3)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tST, desc_k<D>(sK, kk), desc_k<D>(sQ(s), kk), kIdS, kk > 0);
         tc_commit(st_full);
+        return true;
       };
-      auto issue_dpt = [&](int s) {  // dP^T = V dO_s^T
+      auto issue_dpt = [&](int t) -> bool {  // dP^T = V dO_t^T
+        const int s = t % DST;
+        if (!wait_bounded(do_full(s), (t / DST) & 1, g, 3)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tDPT, desc_k<D>(sV, kk), desc_k<D>(sdO(s), kk), kIdS, kk > 0);
         tc_commit(dpt_full);
+        return true;
       };
       int li = 0, gq = 0;
       bool ok = true;
@@ -313,37 +366,38 @@ __global__ void __launch_bounds__(384, 1)
         if (w < 0) break;  // past the last item: no later round has one either
         const DkdvItem I = dkdv_item(p, w);
         if (!wait_bounded(kv_full, li & 1, g, 2)) break;
-        const int s0 = gq % ST;
-        if (!wait_bounded(q_full(s0), (gq / ST) & 1, g, 3)) break;
-        issue_st(s0);
-        issue_dpt(s0);
+        if (!issue_st(gq) || !issue_dpt(gq)) break;
         if (I.n == 1) tc_commit(kv_empty);  // K, V of this item no longer read after these
         for (int it = 0; it < I.n; ++it, ++gq) {
-          const int t = gq, s = t % ST;
+          const int t = gq, sq = t % QST, sd = t % DST;
           // dV += P^T dO: the first one of an item overwrites dV, so the previous
           // item's epilogue must have read it
           if (it == 0 && li >= 1 && !wait_bounded(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
-          if (!wait_bounded(p_ready, t & 1, g, 5)) { ok = false; break; }
-          tc_fence_after();
+          // half h holds query rows 64c + 32h + [0, 32) of the tile, c = 0, 1: K-steps 4c + 2h + {0, 1}
+          for (int h = 0; h < 2; ++h) {
+            if (!wait_bounded(p_ready(h), t & 1, g, 5)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk)
-            mma_ts(tdV, tST + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sdO(s), kk), kIdG,
-                   (it > 0 || kk > 0));
-          const bool more = it + 1 < I.n;
-          const int s1 = (t + 1) % ST;
-          if (more) {  // S^T of the next query tile, behind dV(t) in the stream
-            if (!wait_bounded(q_full(s1), ((t + 1) / ST) & 1, g, 3)) { ok = false; break; }
-            issue_st(s1);
+            for (int j = 0; j < 4; ++j) {
+              const int kk = 4 * (j >> 1) + 2 * h + (j & 1);
+              mma_ts(tdV, tST + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sdO(sd), kk), kIdG,
+                     (it > 0 || h > 0 || j > 0));
+            }
           }
+          if (!ok) break;
+          const bool more = it + 1 < I.n;
+          // S^T of the next query tile, behind dV(t) in the stream
+          if (more && !issue_st(t + 1)) { ok = false; break; }
           if (!wait_bounded(ds_ready, t & 1, g, 6)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kRows / 16; ++kk)
-            mma_ts(tdK, tDPT + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sQ(s), kk), kIdG,
+            mma_ts(tdK, tDPT + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sQ(sq), kk), kIdG,
                    (it > 0 || kk > 0));
-          tc_commit(q_empty(s));  // Q_t, dO_t no longer read
+          tc_commit(q_empty(sq));   // Q_t no longer read
+          tc_commit(do_empty(sd));  // dO_t and its row vectors no longer read
           if (more) {
-            issue_dpt(s1);
+            if (!issue_dpt(t + 1)) { ok = false; break; }
             if (it + 2 == I.n) tc_commit(kv_empty);  // that was the item's last S^T / dP^T
           }
         }
@@ -353,6 +407,28 @@ __global__ void __launch_bounds__(384, 1)
       }
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == kStoreWarp) {
+    // ------------------------------------------- output stores (dV, then dK)
+    if (lane == 0) {
+      tma_prefetch_desc(&tmdK);
+      tma_prefetch_desc(&tmdV);
+      int u = 0;  // staging uses so far
+      bool ok = true;
+      for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
+        const int k0 = (w / p.BH) * kRows, bh = w % p.BH;
+        for (int j = 0; j < 2; ++j, ++u) {
+          if (!wait_bounded(stg_full, u & 1, g, 10)) { ok = false; break; }
+          store_tile<D>(j ? &tmdK : &tmdV, sStg, k0, bh);
+          bulk_commit();
+          bulk_wait_read_all();  // the staging tile may be overwritten from here on
+          mbar_arrive(stg_free);
+        }
+      }
+      bulk_wait_all();
     }
     __syncwarp();
   }
@@ -372,68 +448,71 @@ __global__ void __launch_bounds__(384, 1)
       if (w < 0) break;  // past the last item: no later round has one either
       const DkdvItem I = dkdv_item(p, w);
       const int c = I.k0 + qd * 32 + lane;  // key position owned by this thread
+      const int32_t* drow = p.doc ? p.doc + (size_t)I.b * T : nullptr;
       for (int it = 0; ok && it < I.n; ++it, ++gq) {
-        const int t = gq, s = t % ST;
+        const int t = gq, sd = t % DST;
+        const int rb = 64 * cs;                       // first query row (in the tile) of my columns
+        const int r0 = (I.i_lo + it) * kRows + rb;    // its position
+        // document start of my last query row (read before the wait hides its latency)
+        const int dlast = (drow && r0 + 63 < T) ? __ldg(drow + r0 + 63) : 0;
         if (!wait_bounded_warp(st_full, t & 1, g, 7) ||
-            !wait_bounded_warp(q_full(s), (t / ST) & 1, g, 7)) {
+            !wait_bounded_warp(vec_full(sd), (t / DST) & 1, g, 7)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const float* lse2 = vec + s * 3 * kRows;
+        const float* lse2 = vec + sd * 2 * kRows;
         const float* dl = lse2 + kRows;
-        const int* dsq = reinterpret_cast<const int*>(dl + kRows);
-        const int rb = 64 * cs;                       // first query row (in the tile) of my columns
-        const int r0 = (I.i_lo + it) * kRows + rb;    // its position
         uint32_t sr[2][32];
         tmem_ld32(tS, sr[0]);
         tmem_ld32(tS + 32u, sr[1]);
         tc_wait_ld();
         reg_fence(sr[0]);
         reg_fence(sr[1]);
-        // no mask needed when all my query rows are at or below this key and their
-        // documents start at or before it (dsq is nondecreasing; huge past T)
-        if (!((r0 >= c) && (dsq[rb + 63] <= c))) {
-          const int4* ds4 = reinterpret_cast<const int4*>(dsq + rb);
-#pragma unroll
-          for (int q4 = 0; q4 < 16; ++q4) {
-            const int4 dv4 = ds4[q4];
-            const int dsv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int e = 4 * q4 + k;
-              if (c > r0 + e || c < dsv[k]) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf: weight 0
-            }
+        // no mask needed when all my query rows are at or below this key, before T,
+        // and in its document (document starts never decrease along the rows)
+        const bool full = (r0 >= c) && (r0 + 63 < T) && (dlast <= c);
+        if (__any_sync(0xffffffffu, !full)) {
+          int n_vis;  // rows r0 .. r0 + n_vis - 1 are in c's document or an earlier one, and < T
+          if (drow) {
+            const int ra = r0 + lane, rbb = r0 + 32 + lane;
+            const int da = ra < T ? __ldg(drow + ra) : 0x7fffffff;
+            const int db = rbb < T ? __ldg(drow + rbb) : 0x7fffffff;
+            n_vis = rows_in_doc_prefix(da, db, c);
+          } else {
+            n_vis = T - r0 < 0 ? 0 : (T - r0 > 64 ? 64 : T - r0);
           }
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (e >= n_vis || r0 + e < c) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf: weight 0
         }
-        // P^T = exp2(S^T * scale * log2e - LSE * log2e), kept in fp32 for dS^T
+        // P^T = exp2(S^T * scale * log2e - LSE * log2e), kept in fp32 for dS^T; each half of
+        // my columns goes to the dV MMA as soon as it is in TMEM
         const float4* l4 = reinterpret_cast<const float4*>(lse2 + rb);  // -LSE*log2(e)
         float pf[64];
-        uint32_t pk[32];
 #pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4) {
-          const float4 lv = l4[q4];
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int e = 4 * q4 + 2 * h2;
-            const uint64_t nl = h2 ? f2(lv.z, lv.w) : f2(lv.x, lv.y);
-            const float2 x =
-                f2split(ffma2(f2u(sr[e >> 5][e & 31], sr[e >> 5][(e & 31) + 1]), sl2x2, nl));
-            pf[e] = ex2(x.x);
-            pf[e + 1] = ex2(x.y);
-            pk[e >> 1] = pack_bf16(pf[e], pf[e + 1]);
+          for (int q4 = 8 * h; q4 < 8 * h + 8; ++q4) {
+            const float4 lv = l4[q4];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = 4 * q4 + 2 * h2;
+              const uint64_t nl = h2 ? f2(lv.z, lv.w) : f2(lv.x, lv.y);
+              const float2 x =
+                  f2split(ffma2(f2u(sr[e >> 5][e & 31], sr[e >> 5][(e & 31) + 1]), sl2x2, nl));
+              pf[e] = ex2(x.x);
+              pf[e + 1] = ex2(x.y);
+              pk[(e & 31) >> 1] = pack_bf16(pf[e], pf[e + 1]);
+            }
           }
+          tmem_st16(tS + 16u * h, pk);
+          tc_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_ready(h));
         }
-        {
-          uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pk[0]);
-          uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pk[16]);
-          tmem_st16(tS, lo);
-          tmem_st16(tS + 16u, hi);
-        }
-        tc_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_ready);
         // dS^T = P^T * (dP^T - delta)
         if (!wait_bounded_warp(dpt_full, t & 1, g, 8)) { ok = false; break; }
         tc_fence_after();
@@ -444,24 +523,22 @@ __global__ void __launch_bounds__(384, 1)
         reg_fence(dr[0]);
         reg_fence(dr[1]);
         const float4* d4 = reinterpret_cast<const float4*>(dl + rb);  // -delta
-        uint32_t dk[32];
 #pragma unroll
-        for (int q4 = 0; q4 < 16; ++q4) {
-          const float4 dv4 = d4[q4];
+        for (int h = 0; h < 2; ++h) {
+          uint32_t dk[16];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int e = 4 * q4 + 2 * h2;
-            const uint64_t nd = h2 ? f2(dv4.z, dv4.w) : f2(dv4.x, dv4.y);
-            const float2 dd = f2split(fmul2(
-                f2(pf[e], pf[e + 1]), fadd2(f2u(dr[e >> 5][e & 31], dr[e >> 5][(e & 31) + 1]), nd)));
-            dk[e >> 1] = pack_bf16(dd.x, dd.y);
+          for (int q4 = 8 * h; q4 < 8 * h + 8; ++q4) {
+            const float4 dv4 = d4[q4];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = 4 * q4 + 2 * h2;
+              const uint64_t nd = h2 ? f2(dv4.z, dv4.w) : f2(dv4.x, dv4.y);
+              const float2 dd = f2split(fmul2(
+                  f2(pf[e], pf[e + 1]), fadd2(f2u(dr[e >> 5][e & 31], dr[e >> 5][(e & 31) + 1]), nd)));
+              dk[(e & 31) >> 1] = pack_bf16(dd.x, dd.y);
+            }
           }
-        }
-        {
-          uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dk[0]);
-          uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dk[16]);
-          tmem_st16(tD, lo);
-          tmem_st16(tD + 16u, hi);
+          tmem_st16(tD + 16u * h, dk);
         }
         tc_wait_st();
         tc_fence_before();
@@ -469,17 +546,35 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) mbar_arrive(ds_ready);
       }
       // ---------------------------------------------------------- epilogue
+      // the two warps sharing these lanes split the columns: [cs*D/2, (cs+1)*D/2)
       if (ok && wait_bounded_warp(acc_done, li & 1, g, 9)) {
         tc_fence_after();
-        __nv_bfloat16* dk_row = p.g0 + ((size_t)I.bh * T + c) * D;
-        __nv_bfloat16* dv_row = p.g1 + ((size_t)I.bh * T + c) * D;
-        // the two warps sharing these lanes split the columns: [cs*D/2, (cs+1)*D/2)
-        epilogue_rows<D>(tmem + lane_off + L::T_DV, dv_row, cs, c < T, 1.0f);
-        epilogue_rows<D>(tmem + lane_off + L::T_DK, dk_row, cs, c < T, p.scale);
+        uint32_t wv[D / 4], wk[D / 4];
+        tmem_half_row_bf16<D>(tmem + lane_off + L::T_DV, cs, 1.0f, wv);
+        tmem_half_row_bf16<D>(tmem + lane_off + L::T_DK, cs, p.scale, wk);
         // dV / dK have been read: the next item's first gradient MMA may overwrite them
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_free);
+        const int r = qd * 32 + lane;  // row of the staged tile
+        // staging use 2*li holds dV, 2*li + 1 dK; use u may start once the store of
+        // use u - 1 has read the tile
+        if (li > 0 && !wait_bounded_warp(stg_free, (2 * li - 1) & 1, g, 11)) {
+          ok = false;
+        } else {
+          stage_row<D>(gsm + L::STG_OFF, r, cs * (D / 2), wv);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(stg_full);
+          if (!wait_bounded_warp(stg_free, (2 * li) & 1, g, 11)) {
+            ok = false;
+          } else {
+            stage_row<D>(gsm + L::STG_OFF, r, cs * (D / 2), wk);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(stg_full);
+          }
+        }
       } else {
         ok = false;
       }
@@ -500,7 +595,10 @@ __global__ void __launch_bounds__(384, 1)
 // TMEM: S double-buffered at 0 / 128, dP at 256 (dS is written back over its
 // first half), dQ at 384.  MMA stream per key tile t:  dQ(t), dP(t+1), S(t+2):
 // S(t+1) is ready before the element-wise warps need it, and the only
-// tensor-core work they wait for is dP.
+// tensor-core work they wait for is dP.  dQ leaves through a TMA store from a
+// staged bf16 tile that borrows one slot of the K ring: after an item's key
+// tiles the producer hands the next slot to the epilogue instead of loading
+// it, and the store warp (warp 10) returns it once the store has read it.
 template <int D>
 struct DqLayout {
   static constexpr int STK = (D == 128) ? 3 : 4;  // K ring depth (128-row tiles)
@@ -511,8 +609,8 @@ struct DqLayout {
   static constexpr int V_OFF = K_OFF + STK * Tile<D>::BYTES;      // + s * BYTES
   static constexpr int BAR_OFF = V_OFF + STV * Tile<D>::BYTES;
   // barriers: qdo_full qdo_empty | k_full[STK] k_empty[STK] | v_full[STV] v_empty[STV] |
-  //           s_full[2] dp_full ds_full | acc_done acc_free drain
-  static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 4 + 3;
+  //           s_full[2] dp_full ds_full | acc_done acc_free drain | stg_full
+  static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 4 + 3 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
@@ -547,11 +645,13 @@ __global__ void __launch_bounds__(384, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
-                       const __grid_constant__ CUtensorMap tmdO, const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmdO,
+                       const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
   using Tl = Tile<D>;
   using L = DqLayout<D>;
   constexpr int STK = L::STK, STV = L::STV;
   constexpr int kProducerWarp = L::COMPUTE_WARPS, kMmaWarp = L::COMPUTE_WARPS + 1;
+  constexpr int kStoreWarp = L::COMPUTE_WARPS + 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* gsm;
   const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
@@ -568,6 +668,7 @@ __global__ void __launch_bounds__(384, 1)
   auto s_full = [&](int b) { return xb + 8u * b; };
   const uint32_t dp_full = xb + 16u, ds_full = xb + 24u;
   const uint32_t acc_done = xb + 32u, acc_free = xb + 40u, drain = xb + 48u;
+  const uint32_t stg_full = xb + 56u;  // the staged dQ tile is complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -576,6 +677,7 @@ __global__ void __launch_bounds__(384, 1)
   const int w0 = blockIdx.x, dw = gridDim.x;
 
   if (threadIdx.x == 0) {
+    mbar_init(stg_full, L::COMPUTE_WARPS);
     mbar_init(qdo_full, 1);
     mbar_init(qdo_empty, 1);
     for (int s = 0; s < STK; ++s) {
@@ -637,15 +739,21 @@ __global__ void __launch_bounds__(384, 1)
         const int w = snake_item(k_, w0, dw, p.n_items);
         if (w < 0) break;  // past the last item: no later round has one either
         const DqItem I = dq_item(p, w);
-        for (int it = 0; it < I.n; ++it) {
+        // the K ring carries one more element per item: the slot that stages dQ
+        const int n_el = isK ? I.n + 1 : I.n;
+        for (int it = 0; it < n_el; ++it) {
           const int s = gk % NS, u = gk / NS;
           const uint32_t full = isK ? k_full(s) : v_full(s);
           if (u > 0 && !wait_bounded(isK ? k_empty(s) : v_empty(s), (u - 1) & 1, g, 1)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full, Tl::BYTES);
-          load_tile<D>(isK ? sK(s) : sV(s), tm, (I.kv_lo + it) * kRows, I.bh, full);
+          if (it < I.n) {
+            mbar_arrive_expect_tx(full, Tl::BYTES);
+            load_tile<D>(isK ? sK(s) : sV(s), tm, (I.kv_lo + it) * kRows, I.bh, full);
+          } else {
+            mbar_arrive(full);  // hand the slot to the epilogue
+          }
           ++gk;
         }
       }
@@ -663,9 +771,11 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false);  // S, dP: M = queries, N = keys
       constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);     // dQ: N = d, B (K) is MN-major
       const uint32_t tDP = tmem + L::T_DP, tdQ = tmem + L::T_DQ;
+      int li = 0, gk = 0;
+      // key tile t of item li is element t + li of the K ring (one staging slot per earlier item)
       auto issue_s = [&](int t) -> bool {  // S(t) = Q K_t^T into buffer t & 1
-        const int s = t % STK;
-        if (!wait_bounded(k_full(s), (t / STK) & 1, g, 3)) return false;
+        const int s = (t + li) % STK;
+        if (!wait_bounded(k_full(s), ((t + li) / STK) & 1, g, 3)) return false;
         tc_fence_after();
         const uint32_t tS = tmem + L::T_S + 128u * (uint32_t)(t & 1);
 #pragma unroll
@@ -685,7 +795,6 @@ __global__ void __launch_bounds__(384, 1)
         tc_commit(v_empty(s));  // V of this key tile no longer read
         return true;
       };
-      int li = 0, gk = 0;
       bool ok = true;
       for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
         const int w = snake_item(k_, w0, dw, p.n_items);
@@ -702,7 +811,7 @@ __global__ void __launch_bounds__(384, 1)
           if (it == 0 && li >= 1 && !wait_bounded(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
           if (!wait_bounded(ds_full, t & 1, g, 5)) { ok = false; break; }
           tc_fence_after();
-          const int s = t % STK;
+          const int s = (t + li) % STK;
 #pragma unroll
           for (int kk = 0; kk < kRows / 16; ++kk)
             mma_ts(tdQ, tDP + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sK(s), kk), kIdG,
@@ -721,6 +830,26 @@ __global__ void __launch_bounds__(384, 1)
       }
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == kStoreWarp) {
+    // ------------------------------------------------------------ dQ stores
+    if (lane == 0) {
+      tma_prefetch_desc(&tmdQ);
+      int li = 0, gk = 0;  // items, key tiles so far
+      for (int k_ = 0; k_ * dw < p.n_items; ++k_, ++li) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
+        const DqItem I = dq_item(p, w);
+        gk += I.n;
+        const int s = (gk + li) % STK;  // the item's staging slot
+        if (!wait_bounded(stg_full, li & 1, g, 10)) break;
+        store_tile<D>(&tmdQ, sK(s), I.q0, I.bh);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(k_empty(s));  // the slot goes back to the K ring
+      }
+      bulk_wait_all();
     }
     __syncwarp();
   }
@@ -800,13 +929,24 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) mbar_arrive(ds_full);
       }
       // ---------------------------------------------------------- epilogue
+      // the two warps sharing these lanes split the columns: [cs*D/2, (cs+1)*D/2)
       if (ok && wait_bounded_warp(acc_done, li & 1, g, 8)) {
         tc_fence_after();
-        __nv_bfloat16* dq_row = p.g0 + ((size_t)I.bh * T + r) * D;
-        epilogue_rows<D>(tmem + lane_off + L::T_DQ, dq_row, cs, r < T, p.scale);
+        uint32_t wq[D / 4];
+        tmem_half_row_bf16<D>(tmem + lane_off + L::T_DQ, cs, p.scale, wq);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_free);
+        // the K-ring slot after this item's key tiles stages the tile
+        const int ks = gk + li;
+        if (!wait_bounded_warp(k_full(ks % STK), (ks / STK) & 1, g, 11)) {
+          ok = false;
+        } else {
+          stage_row<D>(gsm + L::K_OFF + (ks % STK) * Tl::BYTES, rl, cs * (D / 2), wq);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(stg_full);
+        }
       } else {
         ok = false;
       }

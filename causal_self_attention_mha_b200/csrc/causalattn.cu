@@ -218,12 +218,16 @@ int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const
   // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
   const int sms = sm_count();
   const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
+  // outputs leave through TMA stores of whole tiles (rows past T are dropped)
+  CUtensorMap mg0, mg1;
+  if (!make_map<D>(&mg0, g0, BH, T) || (dkdv && !make_map<D>(&mg1, g1, BH, T)))
+    return GPT_ATTN_ERR_LAUNCH;
   if (dkdv)
-    ca::attn_bwd_dkdv_kernel<D>
-        <<<grid, ca::DkdvLayout<D>::THREADS, ca::DkdvLayout<D>::SMEM, st>>>(mq, mk, mv, mdo, p);
+    ca::attn_bwd_dkdv_kernel<D><<<grid, ca::DkdvLayout<D>::THREADS, ca::DkdvLayout<D>::SMEM, st>>>(
+        mq, mk, mv, mdo, mg0, mg1, p);
   else
-    ca::attn_bwd_dq_kernel<D>
-        <<<grid, ca::DqLayout<D>::THREADS, ca::DqLayout<D>::SMEM, st>>>(mq, mk, mv, mdo, p);
+    ca::attn_bwd_dq_kernel<D><<<grid, ca::DqLayout<D>::THREADS, ca::DqLayout<D>::SMEM, st>>>(
+        mq, mk, mv, mdo, mg0, p);
   return launch_status();
 }
 

@@ -56,6 +56,40 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m, in
     tma_load_3d(dst + c * Tile<D>::CHUNK_BYTES, m, c * Tile<D>::BOX_COLS, row0, bh, bar);
 }
 
+// L2 prefetch of the same tile (rows past T are skipped by the hardware).
+template <int D>
+__device__ __forceinline__ void prefetch_tile(const CUtensorMap* m, int row0, int bh) {
+#pragma unroll
+  for (int c = 0; c < Tile<D>::CHUNKS; ++c)
+    tma_prefetch_l2_3d(m, c * Tile<D>::BOX_COLS, row0, bh);
+}
+
+// Writes packed bf16 pairs w (columns col0 .. col0 + 2*NW - 1 of tile row r)
+// into a staged tile with the layout load_tile produces (16-byte units XORed
+// with the row inside each swizzle atom), ready for store_tile.  A warp writing
+// 32 consecutive rows at the same columns hits every bank once per 8 rows.
+template <int D, int NW>
+__device__ __forceinline__ void stage_row(uint8_t* stage, int r, int col0, const uint32_t (&w)[NW]) {
+  using Tl = Tile<D>;
+  static_assert(NW % 4 == 0, "whole 16-byte units");
+#pragma unroll
+  for (int u = 0; u < NW / 4; ++u) {
+    const int col = col0 + 8 * u;
+    const int ch = col / Tl::BOX_COLS, cu = (col % Tl::BOX_COLS) / 8;
+    const int phys = (Tl::SW == 128) ? (cu ^ (r & 7)) : (cu ^ ((r >> 1) & 3));
+    *reinterpret_cast<uint4*>(stage + ch * Tl::CHUNK_BYTES + r * Tl::SW + phys * 16) =
+        make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+  }
+}
+
+// TMA store of a staged tile to rows row0 .. row0 + 127 of head bh (rows past T are dropped).
+template <int D>
+__device__ __forceinline__ void store_tile(const CUtensorMap* m, uint32_t src, int row0, int bh) {
+#pragma unroll
+  for (int c = 0; c < Tile<D>::CHUNKS; ++c)
+    tma_store_3d(m, src + c * Tile<D>::CHUNK_BYTES, c * Tile<D>::BOX_COLS, row0, bh);
+}
+
 // Keeps the compiler from using TMEM-load destination registers before
 // tcgen05.wait::ld has been executed.
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {

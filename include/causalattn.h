@@ -147,8 +147,10 @@ int gpt_attn_check_doc_offsets(const int32_t* doc_offsets, int B, int T, void* s
 
 /*
  * Reads (and, if clear != 0, resets) the device status word of the current
- * device: 0 when no kernel has given up on a wait, otherwise bit 31 plus one
- * bit per wait site.  Synchronises the device.  Returns GPT_ATTN_OK, or an
+ * device: 0 when no kernel has reported a problem.  Bit 31 plus one bit per
+ * wait site: a kernel gave up on a bounded wait.  Bit 30: a kernel found its
+ * shared-memory layout larger than the dynamic shared memory it was given
+ * (after rounding the base up to 1 KB) and returned without computing.  Synchronises the device.  Returns GPT_ATTN_OK, or an
  * error status if the device cannot be read.
  */
 int gpt_attn_device_status(unsigned int* out, int clear);
