@@ -609,8 +609,8 @@ struct DqLayout {
   static constexpr int V_OFF = K_OFF + STK * Tile<D>::BYTES;      // + s * BYTES
   static constexpr int BAR_OFF = V_OFF + STV * Tile<D>::BYTES;
   // barriers: qdo_full qdo_empty | k_full[STK] k_empty[STK] | v_full[STV] v_empty[STV] |
-  //           s_full[2] dp_full ds_full | acc_done acc_free drain | stg_full
-  static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 4 + 3 + 1;
+  //           s_full[2] dp_full ds_full | acc_done acc_free drain | stg_full stg_free
+  static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 4 + 3 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
@@ -669,6 +669,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t dp_full = xb + 16u, ds_full = xb + 24u;
   const uint32_t acc_done = xb + 32u, acc_free = xb + 40u, drain = xb + 48u;
   const uint32_t stg_full = xb + 56u;  // the staged dQ tile is complete
+  const uint32_t stg_free = xb + 64u;  // ... and its store has read it
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -678,6 +679,7 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(stg_full, L::COMPUTE_WARPS);
+    mbar_init(stg_free, 1);
     mbar_init(qdo_full, 1);
     mbar_init(qdo_empty, 1);
     for (int s = 0; s < STK; ++s) {
@@ -847,6 +849,7 @@ __global__ void __launch_bounds__(384, 1)
         store_tile<D>(&tmdQ, sK(s), I.q0, I.bh);
         bulk_commit();
         bulk_wait_read_all();
+        mbar_arrive(stg_free);
         mbar_arrive(k_empty(s));  // the slot goes back to the K ring
       }
       bulk_wait_all();
@@ -937,9 +940,11 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_free);
-        // the K-ring slot after this item's key tiles stages the tile
+        // the K-ring slot after this item's key tiles stages the tile, once the
+        // producer has handed it over and the previous item's store has been read
         const int ks = gk + li;
-        if (!wait_bounded_warp(k_full(ks % STK), (ks / STK) & 1, g, 11)) {
+        if (!wait_bounded_warp(k_full(ks % STK), (ks / STK) & 1, g, 11) ||
+            (li > 0 && !wait_bounded_warp(stg_free, (li - 1) & 1, g, 12))) {
           ok = false;
         } else {
           stage_row<D>(gsm + L::K_OFF + (ks % STK) * Tl::BYTES, rl, cs * (D / 2), wq);

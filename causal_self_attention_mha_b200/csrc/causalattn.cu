@@ -157,8 +157,9 @@ template <int D>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
              float scale, const int32_t* doc, cudaStream_t st) {
   const int BH = B * H;
-  CUtensorMap mq, mk, mv;
-  if (!make_map<D>(&mq, q, BH, T) || !make_map<D>(&mk, k, BH, T) || !make_map<D>(&mv, v, BH, T))
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map<D>(&mq, q, BH, T) || !make_map<D>(&mk, k, BH, T) || !make_map<D>(&mv, v, BH, T) ||
+      !make_map<D>(&mo, o, BH, T))
     return GPT_ATTN_ERR_LAUNCH;
   ca::FwdParams p;
   p.doc = doc;
@@ -175,8 +176,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
   const int sms = sm_count();
   const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
-  ca::attn_fwd_kernel<D><<<grid, ca::FwdLayout<D>::THREADS, ca::FwdLayout<D>::SMEM, st>>>(mq, mk,
-                                                                                         mv, p);
+  ca::attn_fwd_kernel<D><<<grid, ca::FwdLayout<D>::THREADS, ca::FwdLayout<D>::SMEM, st>>>(
+      mq, mk, mv, mo, p);
   return launch_status();
 }
 

@@ -19,7 +19,8 @@
 //              query row (= TMEM lane), so row max and sums are in-thread
 //   warp 8     TMA producer: lane 0 loads Q_A, Q_B and the K ring, lane 1 the V ring
 //   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 10-11 idle
+//   warp 10    TMA stores of O
+//   warp 11    idle
 // Registers: launched at 168 per thread; the third warpgroup drops to 88 and
 // the two softmax warpgroups rise to 208 (2*128*208 + 128*88 = 384*168), room
 // for a whole 128-column row of S in registers.
@@ -35,6 +36,12 @@
 // by more than 2^8.  Normalisation uses the sum of the bf16-rounded weights
 // the MMA actually multiplied (the weights of each output row sum to one);
 // the LSE uses the sum of the fp32 weights.
+//
+// O leaves through TMA stores of a staged bf16 tile: after an item's key tiles
+// the producer hands the next K-ring slot to the epilogue instead of loading
+// it; O_A and then O_B are staged there in turn, and the store warp returns the
+// slot once the last store has read it.  Row-per-thread global stores from
+// every SM at the same item boundary congest the memory system.
 #pragma once
 
 #include "tiles.cuh"
@@ -59,8 +66,8 @@ struct FwdLayout {
   static constexpr int V_OFF = K_OFF + STK * Tile<D>::BYTES;
   static constexpr int BAR_OFF = V_OFF + STV * Tile<D>::BYTES;
   // barriers: q_full[2] q_empty[2] k_full[STK] k_empty[STK] v_full[STV] v_empty[STV]
-  //           s_full[2] p_full[2] o_done[2] o_free[2] drain
-  static constexpr int NBAR = 4 + 2 * STK + 2 * STV + 8 + 1;
+  //           s_full[2] p_full[2] o_done[2] o_free[2] drain stg_full stg_free
+  static constexpr int NBAR = 4 + 2 * STK + 2 * STV + 8 + 3;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;       // tmem base slot, abort flag
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;                  // + alignment slack
@@ -105,11 +112,13 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const FwdParams p) {
   using Tl = Tile<D>;
   using L = FwdLayout<D>;
   constexpr int STK = L::STK, STV = L::STV;
   constexpr int kProducerWarp = L::SOFTMAX_WARPS, kMmaWarp = L::SOFTMAX_WARPS + 1;
+  constexpr int kStoreWarp = L::SOFTMAX_WARPS + 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* gsm;
   const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
@@ -127,6 +136,8 @@ __global__ void __launch_bounds__(384, 1)
   auto o_done = [&](int x) { return xb + 8u * (4 + x); };
   auto o_free = [&](int x) { return xb + 8u * (6 + x); };
   const uint32_t drain = xb + 8u * 8;
+  // staging use u (O_A, then O_B, of each item in turn) is complete / has been read
+  const uint32_t stg_full = xb + 8u * 9, stg_free = xb + 8u * 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -152,6 +163,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(v_empty(s), 1);
     }
     mbar_init(drain, 1);
+    mbar_init(stg_full, 4);
+    mbar_init(stg_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -186,11 +199,16 @@ __global__ void __launch_bounds__(384, 1)
           load_tile<D>(sQ + x * Tl::BYTES, &tmQ, I.qt[x] * kRows, I.bh, q_full(x));
           ++nq[x];
         }
-        for (int j = I.j_lo; ok && j <= I.j_hi; ++j) {
+        // the item's key tiles, then one more ring element: the slot that stages O
+        for (int j = I.j_lo; ok && j <= I.j_hi + 1; ++j) {
           const int s = gk % STK, u = gk / STK;
           if (u > 0 && !wait_bounded(k_empty(s), (u - 1) & 1, g, 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(k_full(s), Tl::BYTES);
-          load_tile<D>(sK + s * Tl::BYTES, &tmK, j * kRows, I.bh, k_full(s));
+          if (j <= I.j_hi) {
+            mbar_arrive_expect_tx(k_full(s), Tl::BYTES);
+            load_tile<D>(sK + s * Tl::BYTES, &tmK, j * kRows, I.bh, k_full(s));
+          } else {
+            mbar_arrive(k_full(s));  // hand the slot to the epilogue
+          }
           ++gk;
         }
       }
@@ -292,9 +310,35 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (ok && pend_t[0] >= 0 && !issue_pv(0)) ok = false;
         if (ok && pend_t[1] >= 0 && !issue_pv(1)) ok = false;
+        ++gk;  // the ring element that stages O
       }
       tc_commit(drain);
       drain_wait(drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == kStoreWarp) {
+    // ------------------------------------------------------------- O stores
+    if (lane == 0) {
+      tma_prefetch_desc(&tmO);
+      int gk = 0, u = 0;  // K-ring elements, staging uses so far
+      bool ok = true;
+      for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
+        const int w = snake_item(k_, w0, dw, p.n_items);
+        if (w < 0) break;  // past the last item: no later round has one either
+        const FwdItem I = fwd_item(p, w);
+        gk += I.j_hi - I.j_lo + 1;
+        const uint32_t stage = sK + (gk % STK) * Tl::BYTES;
+        for (int x = 0; x < (I.hasB ? 2 : 1); ++x, ++u) {
+          if (!wait_bounded(stg_full, u & 1, g, 11)) { ok = false; break; }
+          store_tile<D>(&tmO, stage, I.qt[x] * kRows, I.bh);
+          bulk_commit();
+          bulk_wait_read_all();  // the stage may be overwritten from here on
+          mbar_arrive(stg_free);
+          if (x == (I.hasB ? 1 : 0)) mbar_arrive(k_empty(gk % STK));  // back to the K ring
+        }
+        ++gk;
+      }
+      bulk_wait_all();
     }
     __syncwarp();
   }
@@ -310,10 +354,15 @@ __global__ void __launch_bounds__(384, 1)
     const uint64_t sl2x2 = f2(sl2, sl2);
     bool ok = true;
     int t = 0;   // tiles processed by this slot (s_full / p_full / o_done phases)
+    int gk = 0, u0 = 0;  // K-ring elements and staging uses before this item
     for (int k_ = 0; k_ * dw < p.n_items; ++k_) {
-        const int w = snake_item(k_, w0, dw, p.n_items);
-        if (w < 0) break;  // past the last item: no later round has one either
+      const int w = snake_item(k_, w0, dw, p.n_items);
+      if (w < 0) break;  // past the last item: no later round has one either
       const FwdItem I = fwd_item(p, w);
+      const int ks = gk + (I.j_hi - I.j_lo + 1);  // this item's staging element
+      const int u = u0 + x;                        // this tile's staging use
+      gk = ks + 1;
+      u0 += I.hasB ? 2 : 1;
       if (x == 1 && !I.hasB) continue;
       const int row = I.qt[x] * kRows + rl;
       const int ds = p.doc ? p.doc[(size_t)I.b * T + (row < T ? row : T - 1)] : 0;
@@ -426,8 +475,8 @@ __global__ void __launch_bounds__(384, 1)
         const float mu = (m == -INFINITY) ? 0.f : m;
         if (row < T) p.lse[(size_t)I.bh * T + row] = (mu + lg2(l)) * kLn2;
         const float inv = 1.0f / lr;
-        __nv_bfloat16* orow = p.o + ((size_t)I.bh * T + row) * D;
-        // the row in up to two waves of (at most) 64 columns: loads in flight together
+        // the row, normalised, as packed bf16: up to two waves of 64 columns, loads in flight together
+        uint32_t wo[D / 2];
 #pragma unroll
         for (int w2 = 0; w2 < (D + 63) / 64; ++w2) {
           constexpr int NC = (D >= 64) ? 2 : 1;
@@ -437,15 +486,28 @@ __global__ void __launch_bounds__(384, 1)
           tc_wait_ld();
 #pragma unroll
           for (int c = 0; c < NC; ++c) reg_fence(r[c]);
-          if (row < T) {
 #pragma unroll
-            for (int c = 0; c < NC; ++c) store_row_chunk_bf16(orow + 64 * w2 + 32 * c, r[c], inv);
-          }
+          for (int c = 0; c < NC; ++c)
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              wo[32 * w2 + 16 * c + e] = pack_bf16(__uint_as_float(r[c][2 * e]) * inv,
+                                                   __uint_as_float(r[c][2 * e + 1]) * inv);
         }
         // O_x has been read: the next item's first PV may overwrite it
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(o_free(x));
+        // stage the row once the slot is ours (handed over by the producer) and the store of
+        // the previous staging use has read it; rows past T are dropped by the store
+        if (!wait_bounded_warp(k_full(ks % STK), (ks / STK) & 1, g, 12) ||
+            (u > 0 && !wait_bounded_warp(stg_free, (u - 1) & 1, g, 13))) {
+          ok = false;
+        } else {
+          stage_row<D>(gsm + L::K_OFF + (ks % STK) * Tl::BYTES, rl, 0, wo);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(stg_full);
+        }
       } else {
         ok = false;
       }
