@@ -42,8 +42,8 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.md")
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wide_d128")
     ap.add_argument("--e2e-steps", type=int, default=10)
