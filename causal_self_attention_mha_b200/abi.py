@@ -317,3 +317,66 @@ class HostStep:
                          self.dv, self.delta, scale, self.doc, s)
             for name in ("o", "lse", "dq", "dk", "dv"):
                 out_h[name].copy_(getattr(self, name), non_blocking=True)
+
+
+class HostStream:
+    """Forward + backward over a sequence of steps whose inputs and outputs all
+    live in pinned HOST memory, with neighbouring steps overlapped: while step k
+    computes, step k+1's inputs are copied in and step k-1's outputs copied out
+    (host-to-device and device-to-host copies use opposite directions of the bus,
+    so they run at the same time).  Two sets of device buffers alternate between
+    steps; three CUDA streams carry the copies in, the kernels and the copies
+    out, ordered by events.  Every step still moves all of its inputs to the
+    device and all of its outputs (O, LSE, dQ, dK, dV) back."""
+
+    def __init__(self, B: int, H: int, T: int, d: int, device="cuda"):
+        dev = torch.device(device)
+        self.sets = [HostStep(B, H, T, d, dev) for _ in range(2)]
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        self.device = dev
+
+    def set_doc_offsets(self, doc_host):
+        for st in self.sets:
+            st.set_doc_offsets(doc_host)
+
+    def h2d_bytes(self) -> int:
+        return self.sets[0].h2d_bytes()
+
+    def d2h_bytes(self) -> int:
+        return self.sets[0].d2h_bytes()
+
+    def run(self, steps, scale: float, after=None):
+        """steps: sequence of (q_h, k_h, v_h, do_h, out_h); out_h is a dict of pinned host
+        tensors 'o', 'lse', 'dq', 'dk', 'dv'.  `after`: an optional CUDA event the first copy
+        waits for.  Enqueues everything and returns the event recorded after the last copy
+        out (asynchronous: synchronise on it before reading the outputs)."""
+        ev_comp, ev_out = [], []
+        for k, (q_h, k_h, v_h, do_h, out_h) in enumerate(steps):
+            st = self.sets[k % 2]
+            if k == 0 and after is not None:
+                self.s_in.wait_event(after)
+            if k >= 2:  # set k % 2 holds step k-2's inputs until its kernels have read them
+                self.s_in.wait_event(ev_comp[k - 2])
+            with torch.cuda.stream(self.s_in):
+                for dst, src in ((st.q, q_h), (st.k, k_h), (st.v, v_h), (st.do, do_h)):
+                    dst.copy_(src, non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(self.s_in)
+            self.s_comp.wait_event(ev_in)
+            if k >= 2:  # ... and step k-2's outputs until they have been copied out
+                self.s_comp.wait_event(ev_out[k - 2])
+            gpt_attn_fwd(st.q, st.k, st.v, st.o, st.lse, scale, st.doc, self.s_comp)
+            gpt_attn_bwd(st.q, st.k, st.v, st.o, st.do, st.lse, st.dq, st.dk, st.dv, st.delta,
+                         scale, st.doc, self.s_comp)
+            ec = torch.cuda.Event()
+            ec.record(self.s_comp)
+            ev_comp.append(ec)
+            self.s_out.wait_event(ec)
+            with torch.cuda.stream(self.s_out):
+                for name in ("o", "lse", "dq", "dk", "dv"):
+                    out_h[name].copy_(getattr(st, name), non_blocking=True)
+                eo = torch.cuda.Event()
+                eo.record(self.s_out)
+            ev_out.append(eo)
+        return ev_out[-1] if ev_out else None
+

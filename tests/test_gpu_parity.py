@@ -154,6 +154,32 @@ def test_deterministic(cuda_device):
         assert torch.equal(x, y)
 
 
+def test_host_stream_matches_device_path(cuda_device):
+    """HostStream (pinned host buffers, neighbouring steps overlapped on three streams,
+    two device buffer sets) gives, for every step of a sequence of different inputs,
+    bit-for-bit the outputs of the device path, and the first step matches the oracle."""
+    B, H, T, d = 2, 3, 333, 64
+    scale = inputs.fp32_scale(d)
+    doc = inputs.doc_start_from_lengths([[100, 233], [50, 283]], T)
+    steps, expect = [], []
+    for seed in (41, 42, 43, 44, 45):
+        q, k, v, do = inputs.make_qkvdo(B, H, T, d, seed)
+        expect.append(run_gpu(q, k, v, do, doc, scale))
+        outs = {n: torch.empty(B, H, T, d, dtype=torch.bfloat16).pin_memory()
+                for n in ("o", "dq", "dk", "dv")}
+        outs["lse"] = torch.empty(B, H, T, dtype=torch.float32).pin_memory()
+        steps.append(tuple(t.pin_memory() for t in (q, k, v, do)) + (outs,))
+    hs = abi.HostStream(B, H, T, d)
+    hs.set_doc_offsets(doc)
+    hs.run(steps, scale).synchronize()
+    for st, ex in zip(steps, expect):
+        out = st[4]
+        for name, ref in zip(("o", "lse", "dq", "dk", "dv"), ex):
+            assert torch.equal(out[name], ref), name
+    q, k, v, do = steps[0][:4]
+    compare(expect[0], q, k, v, do, doc, scale, label="hoststream")
+
+
 def test_uniform_values_on_gpu(cuda_device):
     """All value rows equal: every output row equals that row (up to its bf16 rounding)."""
     B, H, T, d = 1, 2, 300, 64
