@@ -592,10 +592,12 @@ __global__ void __launch_bounds__(384, 1)
 // --------------------------------------------------------------------- dQ
 // Q and dO of the item's query tile stay in shared memory; K and V stream
 // through rings of their own (K is read by S and by dQ, V only by dP).
-// TMEM: S double-buffered at 0 / 128, dP at 256 (dS is written back over its
-// first half), dQ at 384.  MMA stream per key tile t:  dQ(t), dP(t+1), S(t+2):
-// S(t+1) is ready before the element-wise warps need it, and the only
-// tensor-core work they wait for is dP.  dQ leaves through a TMA store from a
+// TMEM: S double-buffered at 0 / 128, dP at 256, dQ at 384.  dS(t) is written
+// back (packed bf16) over S(t)'s own buffer, already read out, so dP(t+1) may
+// overwrite dP(t) as soon as the element-wise warps have loaded it.  MMA stream
+// per key tile t:  dP(t+1), dQ(t), S(t+2): dP(t+1) runs while dS(t) is being
+// formed, and S(t+2) follows dQ(t), which has consumed dS(t), in the in-order
+// stream.  dQ leaves through a TMA store from a
 // staged bf16 tile that borrows one slot of the K ring: after an item's key
 // tiles the producer hands the next slot to the epilogue instead of loading
 // it, and the store warp (warp 10) returns it once the store has read it.
@@ -609,8 +611,8 @@ struct DqLayout {
   static constexpr int V_OFF = K_OFF + STK * Tile<D>::BYTES;      // + s * BYTES
   static constexpr int BAR_OFF = V_OFF + STV * Tile<D>::BYTES;
   // barriers: qdo_full qdo_empty | k_full[STK] k_empty[STK] | v_full[STV] v_empty[STV] |
-  //           s_full[2] dp_full ds_full | acc_done acc_free drain | stg_full stg_free
-  static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 4 + 3 + 2;
+  //           s_full[2] dp_full dp_read ds_full | acc_done acc_free drain | stg_full stg_free
+  static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 5 + 3 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
@@ -670,6 +672,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t acc_done = xb + 32u, acc_free = xb + 40u, drain = xb + 48u;
   const uint32_t stg_full = xb + 56u;  // the staged dQ tile is complete
   const uint32_t stg_free = xb + 64u;  // ... and its store has read it
+  const uint32_t dp_read = xb + 72u;   // dP(t) is in the element-wise warps' registers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -693,6 +696,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(s_full(0), 1);
     mbar_init(s_full(1), 1);
     mbar_init(dp_full, 1);
+    mbar_init(dp_read, L::COMPUTE_WARPS);
     mbar_init(ds_full, L::COMPUTE_WARPS);
     mbar_init(acc_done, 1);
     mbar_init(acc_free, L::COMPUTE_WARPS);
@@ -804,25 +808,30 @@ __global__ void __launch_bounds__(384, 1)
         const DqItem I = dq_item(p, w);
         if (!wait_bounded(qdo_full, li & 1, g, 2)) break;
         const int t0 = gk;
+        // dP(t0) overwrites dP(t0 - 1): the element-wise warps must have loaded it
+        if (t0 > 0 && !wait_bounded(dp_read, (t0 - 1) & 1, g, 9)) break;
         ok = issue_s(t0) && issue_dp(t0);
         if (ok && I.n == 1) tc_commit(qdo_empty);  // Q, dO of this item no longer read
         if (ok && I.n > 1) ok = issue_s(t0 + 1);
         for (int it = 0; ok && it < I.n; ++it) {
           const int t = t0 + it;
+          // dP of the next key tile as soon as dP(t) has been read out of TMEM
+          if (it + 1 < I.n) {
+            if (!wait_bounded(dp_read, t & 1, g, 9) || !issue_dp(t + 1)) { ok = false; break; }
+            if (it + 2 == I.n) tc_commit(qdo_empty);  // that was the item's last S / dP
+          }
           // the first dQ MMA of an item overwrites dQ: the previous epilogue must have read it
           if (it == 0 && li >= 1 && !wait_bounded(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
           if (!wait_bounded(ds_full, t & 1, g, 5)) { ok = false; break; }
           tc_fence_after();
           const int s = (t + li) % STK;
+          const uint32_t tdS = tmem + L::T_S + 128u * (uint32_t)(t & 1);  // dS(t) over S(t)
 #pragma unroll
           for (int kk = 0; kk < kRows / 16; ++kk)
-            mma_ts(tdQ, tDP + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sK(s), kk), kIdG,
+            mma_ts(tdQ, tdS + 64u * (kk >> 2) + 8u * (kk & 3), desc_mn<D>(sK(s), kk), kIdG,
                    (it > 0 || kk > 0));
           tc_commit(k_empty(s));  // K of this key tile no longer read
-          if (it + 1 < I.n) {
-            if (!issue_dp(t + 1)) { ok = false; break; }
-            if (it + 2 == I.n) tc_commit(qdo_empty);  // that was the item's last S / dP
-          }
+          // S(t+2) reuses S(t)'s buffer, after dQ(t) in the stream
           if (it + 2 < I.n && !issue_s(t + 2)) { ok = false; break; }
         }
         if (!ok) break;
@@ -912,7 +921,11 @@ __global__ void __launch_bounds__(384, 1)
         tc_wait_ld();
         reg_fence(dr[0]);
         reg_fence(dr[1]);
-        // dS = P * (dP - delta), bf16, over the first 32 of my dP columns
+        // dP(t) is in registers: dP(t+1) may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dp_read);
+        // dS = P * (dP - delta), bf16, over the first 32 of my columns of S(t)'s buffer
         uint32_t dk[32];
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
@@ -923,8 +936,8 @@ __global__ void __launch_bounds__(384, 1)
         {
           uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dk[0]);
           uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(&dk[16]);
-          tmem_st16(tD, lo);
-          tmem_st16(tD + 16u, hi);
+          tmem_st16(tS, lo);
+          tmem_st16(tS + 16u, hi);
         }
         tc_wait_st();
         tc_fence_before();
