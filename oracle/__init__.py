@@ -11,7 +11,8 @@ with gcc on first use and marshals numpy float64 arrays through ctypes.
 
 What is computed (see the C file header for the passages it follows):
   forward:   S = scale * Q K^T, S_ij = -inf for j > i (and, with a document
-             mask, for j < doc_start[i]), P = softmax_rows(S), O = P V,
+             mask, for j < doc_start[i]; with a sliding window of w keys, for
+             j <= i - w), P = softmax_rows(S), O = P V,
              LSE_i = log sum_j exp(S_ij)  (natural log, scaled scores)
   backward:  dV = P^T dO, dP = dO V^T, dS_i = (diag(p_i) - p_i p_i^T) dP_i
              with the Jacobian formed explicitly, dQ = scale dS K,
@@ -56,6 +57,14 @@ def _load():
         lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_double, ip, dp, dp, dp]
         lib.oracle_attn_bwd.restype = ctypes.c_int
+        lib.oracle_attn_fwd_window.argtypes = [dp, dp, dp, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_double, ip,
+                                               ctypes.c_int, dp, dp, dp]
+        lib.oracle_attn_fwd_window.restype = ctypes.c_int
+        lib.oracle_attn_bwd_window.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_double, ip,
+                                               ctypes.c_int, dp, dp, dp]
+        lib.oracle_attn_bwd_window.restype = ctypes.c_int
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -95,8 +104,15 @@ def max_threads() -> int:
     return int(_load().oracle_max_threads())
 
 
-def attention_forward(q, k, v, scale: float, doc_start=None, return_probs: bool = False):
-    """O [B,H,T,d], LSE [B,H,T] (float64); with return_probs also P [B,H,T,T]."""
+def _window(window) -> int:
+    """None or <= 0: no window; otherwise the number of keys a query sees, itself included."""
+    return 0 if window is None or int(window) <= 0 else int(window)
+
+
+def attention_forward(q, k, v, scale: float, doc_start=None, return_probs: bool = False,
+                      window=None):
+    """O [B,H,T,d], LSE [B,H,T] (float64); with return_probs also P [B,H,T,T].
+    window: i sees j iff i - window < j <= i (None: plain causal)."""
     lib = _load()
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, T, d = q.shape
@@ -106,16 +122,18 @@ def attention_forward(q, k, v, scale: float, doc_start=None, return_probs: bool 
     o = np.empty_like(q)
     lse = np.empty((B, H, T), dtype=np.float64)
     probs = np.empty((B, H, T, T), dtype=np.float64) if return_probs else None
-    rc = lib.oracle_attn_fwd(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
-                             _ptr(v, ctypes.c_double), B, H, T, d, float(scale),
-                             _ptr(doc, ctypes.c_int32), _ptr(o, ctypes.c_double),
-                             _ptr(lse, ctypes.c_double), _ptr(probs, ctypes.c_double))
+    rc = lib.oracle_attn_fwd_window(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
+                                    _ptr(v, ctypes.c_double), B, H, T, d, float(scale),
+                                    _ptr(doc, ctypes.c_int32), _window(window),
+                                    _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
+                                    _ptr(probs, ctypes.c_double))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd failed with code {rc}")
     return (o, lse, probs) if return_probs else (o, lse)
 
 
-def attention_backward(q, k, v, dout, scale: float, doc_start=None) -> Tuple[np.ndarray, ...]:
+def attention_backward(q, k, v, dout, scale: float, doc_start=None,
+                       window=None) -> Tuple[np.ndarray, ...]:
     """dQ, dK, dV [B,H,T,d] float64, by the explicit softmax Jacobian."""
     lib = _load()
     q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
@@ -125,11 +143,11 @@ def attention_backward(q, k, v, dout, scale: float, doc_start=None) -> Tuple[np.
             raise ValueError("q, k, v, dout must share one [B,H,T,d] shape")
     doc = _doc(doc_start, B, T)
     dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
-    rc = lib.oracle_attn_bwd(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
-                             _ptr(v, ctypes.c_double), _ptr(dout, ctypes.c_double),
-                             B, H, T, d, float(scale), _ptr(doc, ctypes.c_int32),
-                             _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
-                             _ptr(dv, ctypes.c_double))
+    rc = lib.oracle_attn_bwd_window(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
+                                    _ptr(v, ctypes.c_double), _ptr(dout, ctypes.c_double),
+                                    B, H, T, d, float(scale), _ptr(doc, ctypes.c_int32),
+                                    _window(window), _ptr(dq, ctypes.c_double),
+                                    _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd failed with code {rc}")
     return dq, dk, dv

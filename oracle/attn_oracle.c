@@ -25,6 +25,12 @@
  *   doc_start[b*T + i] is the first position of the document holding i, and
  *   i attends to j iff doc_start[i] <= j <= i.
  *
+ *   Optional sliding window -- the same page, section 9 (gpt.py walkthrough),
+ *   lists sliding-window attention among the model's attention features
+ *   without stating its definition.  Reading: a window of w keys, the query's
+ *   own position included: i attends to j iff i - w < j <= i (and the
+ *   document rule, when both apply).  window <= 0 means no window.
+ *
  *   Log-sum-exp -- the natural log of the softmax denominator of the SCALED
  *   scores: lse_i = max_j s_ij + log(sum_j exp(s_ij - max_j s_ij)).
  *
@@ -77,9 +83,10 @@ int oracle_max_threads(void) {
 }
 
 /* Is key position j visible from query position i?  (diagonal included) */
-static int visible(const int32_t *doc_row, int i, int j) {
+static int visible(const int32_t *doc_row, int window, int i, int j) {
     if (j > i) return 0;
     if (doc_row != NULL && j < doc_row[i]) return 0;
+    if (window > 0 && j <= i - window) return 0;
     return 1;
 }
 
@@ -95,11 +102,11 @@ static int check_args(const void *a, const void *b, const void *c, int B, int H,
  * s is scratch of length >= i+1.
  */
 static double softmax_row(const double *qh, const double *kh, int d, double scale,
-                          const int32_t *doc_row, int i, double *s, double *p) {
+                          const int32_t *doc_row, int window, int i, double *s, double *p) {
     const double *qi = qh + (size_t)i * d;
     double m = -INFINITY;
     for (int j = 0; j <= i; ++j) {
-        if (!visible(doc_row, i, j)) { s[j] = -INFINITY; continue; }
+        if (!visible(doc_row, window, i, j)) { s[j] = -INFINITY; continue; }
         const double *kj = kh + (size_t)j * d;
         double acc = 0.0;
         for (int c = 0; c < d; ++c) acc += qi[c] * kj[c];
@@ -120,9 +127,10 @@ static double softmax_row(const double *qh, const double *kh, int d, double scal
  * Forward.  o: [B,H,T,d]; lse: [B,H,T] (may be NULL); probs: [B,H,T,T] or
  * NULL (the full attention matrix, invisible entries 0 -- for small tests).
  */
-int oracle_attn_fwd(const double *q, const double *k, const double *v,
-                    int B, int H, int T, int d, double scale,
-                    const int32_t *doc_start, double *o, double *lse, double *probs) {
+int oracle_attn_fwd_window(const double *q, const double *k, const double *v,
+                           int B, int H, int T, int d, double scale,
+                           const int32_t *doc_start, int window,
+                           double *o, double *lse, double *probs) {
     if (check_args(q, k, v, B, H, T, d) || o == NULL) return ORACLE_ERR_ARGS;
     const long BH = (long)B * H;
     int err = ORACLE_OK;
@@ -142,7 +150,7 @@ int oracle_attn_fwd(const double *q, const double *k, const double *v,
                 double *oh = o + off;
                 const int32_t *doc_row = doc_start ? doc_start + (size_t)b * T : NULL;
                 for (int i = 0; i < T; ++i) {
-                    double l = softmax_row(qh, kh, d, scale, doc_row, i, s, p);
+                    double l = softmax_row(qh, kh, d, scale, doc_row, window, i, s, p);
                     if (lse) lse[(size_t)bh * T + i] = l;
                     double *oi = oh + (size_t)i * d;
                     for (int c = 0; c < d; ++c) oi[c] = 0.0;
@@ -168,9 +176,10 @@ int oracle_attn_fwd(const double *q, const double *k, const double *v,
  * Backward by the explicit softmax Jacobian.  dq, dk, dv: [B,H,T,d], fully
  * overwritten.
  */
-int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dout,
-                    int B, int H, int T, int d, double scale, const int32_t *doc_start,
-                    double *dq, double *dk, double *dv) {
+int oracle_attn_bwd_window(const double *q, const double *k, const double *v,
+                           const double *dout, int B, int H, int T, int d, double scale,
+                           const int32_t *doc_start, int window,
+                           double *dq, double *dk, double *dv) {
     if (check_args(q, k, v, B, H, T, d) || dout == NULL || dq == NULL || dk == NULL || dv == NULL)
         return ORACLE_ERR_ARGS;
     const long BH = (long)B * H;
@@ -197,7 +206,7 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
                 memset(dkh, 0, sizeof(double) * (size_t)T * d);
                 memset(dvh, 0, sizeof(double) * (size_t)T * d);
                 for (int i = 0; i < T; ++i) {
-                    softmax_row(qh, kh, d, scale, doc_row, i, s, p);
+                    softmax_row(qh, kh, d, scale, doc_row, window, i, s, p);
                     const double *doi = doh + (size_t)i * d;
                     const double *qi = qh + (size_t)i * d;
                     /* dV_j += p_ij dO_i ;  dP_ij = <dO_i, v_j> */
@@ -241,4 +250,17 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
         free(jrow);
     }
     return err;
+}
+
+/* Plain causal (or document-causal) attention: no window. */
+int oracle_attn_fwd(const double *q, const double *k, const double *v,
+                    int B, int H, int T, int d, double scale,
+                    const int32_t *doc_start, double *o, double *lse, double *probs) {
+    return oracle_attn_fwd_window(q, k, v, B, H, T, d, scale, doc_start, 0, o, lse, probs);
+}
+
+int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dout,
+                    int B, int H, int T, int d, double scale, const int32_t *doc_start,
+                    double *dq, double *dk, double *dv) {
+    return oracle_attn_bwd_window(q, k, v, dout, B, H, T, d, scale, doc_start, 0, dq, dk, dv);
 }

@@ -21,6 +21,8 @@ MUTATIONS = {
     "scores_without_scale": ("s[j] = scale * acc;", "s[j] = acc;"),
     "mask_drops_diagonal": ("if (j > i) return 0;", "if (j >= i) return 0;"),
     "doc_mask_off_by_one": ("j < doc_row[i]) return 0;", "j <= doc_row[i]) return 0;"),
+    "window_off_by_one": ("j <= i - window) return 0;", "j < i - window) return 0;"),
+    "window_ignored": ("if (window > 0 && j <= i - window) return 0;", ""),
     "lse_in_log2": ("return m + log(z);", "return m + log2(z);"),
     "jacobian_sign": ("(j == kk ? p[j] : 0.0) - p[j] * p[kk]", "(j == kk ? p[j] : 0.0) + p[j] * p[kk]"),
     "jacobian_drops_diag": ("(j == kk ? p[j] : 0.0) - p[j] * p[kk]", "- p[j] * p[kk]"),
@@ -43,6 +45,9 @@ PIN_TESTS = [
     (pins.test_central_finite_differences, {"T": 5, "d": 2, "with_doc": True}),
     (pins.test_against_torch_sdpa_fp64, {"B": 1, "H": 2, "T": 64, "d": 32, "with_doc": False}),
     (pins.test_against_torch_sdpa_fp64, {"B": 2, "H": 1, "T": 60, "d": 16, "with_doc": True}),
+    (pins.test_window_of_one_key_closed_form, {}),
+    (pins.test_window_probability_rows, {"w": 3}),
+    (pins.test_window_against_torch_sdpa_fp64, {"T": 64, "d": 32, "w": 16, "with_doc": False}),
 ]
 
 
@@ -63,7 +68,8 @@ def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
     so = _compile_mutant(tmp_path, old, new)
     real = oracle._load()
     lib = ctypes.CDLL(so)
-    for fn in ("oracle_attn_fwd", "oracle_attn_bwd"):
+    for fn in ("oracle_attn_fwd", "oracle_attn_bwd", "oracle_attn_fwd_window",
+               "oracle_attn_bwd_window"):
         getattr(lib, fn).argtypes = getattr(real, fn).argtypes
         getattr(lib, fn).restype = ctypes.c_int
     monkeypatch.setattr(oracle, "_lib", lib)

@@ -271,3 +271,140 @@ def test_against_torch_sdpa_fp64(B, H, T, d, with_doc):
     ro, rl, rq, rk, rv = torch_reference(q, k, v, do, scale, doc)
     for a, b in ((o, ro), (lse, rl), (dq, rq), (dk, rk), (dv, rv)):
         assert np.max(np.abs(a - b)) <= 1e-10
+
+
+# ------------------------------------------------------------- sliding window
+# Reading of "How to build an LLM by hand" (agmtopy.github.io), section 9:
+# a window of w keys, the query included: i sees j iff i - w < j <= i.
+
+def test_window_covering_everything_is_plain_causal():
+    """w >= T changes nothing: bit-identical to the unwindowed oracle (with and without documents)."""
+    B, H, T, d = 2, 2, 37, 8
+    q, k, v, do = (rnd((B, H, T, d), 500 + s) for s in range(4))
+    doc = inputs.random_doc_start(B, T, 4, 5, 15).numpy()
+    for dc in (None, doc):
+        base_f = oracle.attention_forward(q, k, v, 0.4, dc)
+        base_b = oracle.attention_backward(q, k, v, do, 0.4, dc)
+        for w in (T, T + 1, 10 ** 6):
+            for a, b in zip(oracle.attention_forward(q, k, v, 0.4, dc, window=w), base_f):
+                assert np.array_equal(a, b)
+            for a, b in zip(oracle.attention_backward(q, k, v, do, 0.4, dc, window=w), base_b):
+                assert np.array_equal(a, b)
+
+
+def test_window_of_one_key_closed_form():
+    """w = 1: each query sees only itself: O = V, LSE_i = scale <q_i, k_i>, dQ = dK = 0, dV = dO."""
+    B, H, T, d = 1, 3, 20, 6
+    q, k, v, do = (rnd((B, H, T, d), 510 + s) for s in range(4))
+    o, lse = oracle.attention_forward(q, k, v, 0.7, window=1)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, 0.7, window=1)
+    np.testing.assert_array_equal(o, v)
+    np.testing.assert_allclose(lse, 0.7 * np.einsum("bhtc,bhtc->bht", q, k), atol=1e-13)
+    assert np.max(np.abs(dq)) == 0.0 and np.max(np.abs(dk)) == 0.0
+    np.testing.assert_array_equal(dv, do)
+
+
+def test_window_two_keys_closed_form():
+    """w = 2, row i >= 1 sees keys i-1 and i: a two-term softmax written out by hand."""
+    B, H, T, d = 1, 1, 9, 4
+    q, k, v, _ = (rnd((B, H, T, d), 520 + s) for s in range(4))
+    sc = 0.5
+    o, lse = oracle.attention_forward(q, k, v, sc, window=2)
+    for i in range(1, T):
+        a = sc * float(q[0, 0, i] @ k[0, 0, i - 1])
+        b = sc * float(q[0, 0, i] @ k[0, 0, i])
+        pa = 1.0 / (1.0 + math.exp(b - a))
+        np.testing.assert_allclose(o[0, 0, i], pa * v[0, 0, i - 1] + (1 - pa) * v[0, 0, i], atol=1e-13)
+        np.testing.assert_allclose(lse[0, 0, i], max(a, b) + math.log(math.exp(a - max(a, b)) + math.exp(b - max(a, b))), atol=1e-13)
+    np.testing.assert_allclose(o[0, 0, 0], v[0, 0, 0], atol=0)
+
+
+@pytest.mark.parametrize("w", [1, 3, 8])
+def test_window_probability_rows(w):
+    """Rows of P sum to 1; weights outside [i-w+1, i] (and outside the document) are exactly 0."""
+    B, H, T, d = 2, 2, 30, 4
+    q, k, v = (rnd((B, H, T, d), 530 + s) for s in range(3))
+    doc = inputs.random_doc_start(B, T, 6, 4, 12).numpy()
+    _, _, p = oracle.attention_forward(q, k, v, 0.5, doc, return_probs=True, window=w)
+    np.testing.assert_allclose(p.sum(-1), 1.0, atol=1e-12)
+    for b in range(B):
+        for i in range(T):
+            lo = max(int(doc[b, i]), i - w + 1)
+            outside = np.ones(T, dtype=bool)
+            outside[lo:i + 1] = False
+            assert np.all(p[b, :, i, outside] == 0.0)
+
+
+def test_window_ignores_keys_that_left_it():
+    """Row i's outputs do not change when keys and values older than i - w + 1 change."""
+    B, H, T, d, w = 1, 2, 40, 8, 6
+    q, k, v, do = (rnd((B, H, T, d), 540 + s) for s in range(4))
+    o, lse = oracle.attention_forward(q, k, v, 0.3, window=w)
+    i = 25
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, : i - w + 1] += 3.0
+    v2[:, :, : i - w + 1] -= 5.0
+    o2, lse2 = oracle.attention_forward(q, k2, v2, 0.3, window=w)
+    assert np.array_equal(o[:, :, i], o2[:, :, i]) and np.array_equal(lse[:, :, i], lse2[:, :, i])
+
+
+@pytest.mark.parametrize("T,d,w", [(5, 2, 2), (8, 4, 3)])
+@pytest.mark.parametrize("with_doc", [False, True])
+def test_window_finite_differences(T, d, w, with_doc):
+    """Windowed backward against central differences of L = sum(dO * O), h = 1e-6, fp64."""
+    B, H = 1, 2
+    q, k, v, do = (rnd((B, H, T, d), 560 + 7 * T + d + s) for s in range(4))
+    scale = 1 / math.sqrt(d)
+    doc = inputs.random_doc_start(B, T, T, 1, 5).numpy() if with_doc else None
+    grads = oracle.attention_backward(q, k, v, do, scale, doc, window=w)
+    h = 1e-6
+    for which, g in enumerate(grads):
+        num = np.zeros_like(g)
+        for idx in np.ndindex(*g.shape):
+            plus = [a.copy() for a in (q, k, v)]
+            minus = [a.copy() for a in (q, k, v)]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            lp = np.sum(do * oracle.attention_forward(*plus, scale, doc, window=w)[0])
+            lm = np.sum(do * oracle.attention_forward(*minus, scale, doc, window=w)[0])
+            num[idx] = (lp - lm) / (2 * h)
+        if np.linalg.norm(num) < 1e-12:
+            assert np.max(np.abs(g)) < 1e-9
+        else:
+            assert np.linalg.norm(num - g) / np.linalg.norm(num) <= 1e-6, which
+
+
+def torch_band_reference(q, k, v, do, scale, w, doc=None):
+    """torch CPU float64 SDPA + autograd with an explicit boolean band (and document) mask."""
+    tq, tk, tv = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+    B, T = q.shape[0], q.shape[2]
+    i = torch.arange(T).view(1, T, 1)
+    j = torch.arange(T).view(1, 1, T)
+    start = torch.clamp(i - w + 1, min=0).expand(B, T, 1)
+    if doc is not None:
+        start = torch.maximum(start, torch.tensor(doc, dtype=torch.int64).view(B, T, 1))
+    mask = (j <= i) & (j >= start)  # [B,T,T]
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask.unsqueeze(1),
+                                                         scale=scale)
+    s = torch.einsum("bhic,bhjc->bhij", tq.detach(), tk.detach()) * scale
+    lse = torch.logsumexp(s.masked_fill(~mask.unsqueeze(1), float("-inf")), dim=-1)
+    o.backward(torch.tensor(do, dtype=torch.float64))
+    return (o.detach().numpy(), lse.numpy(), tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy())
+
+
+@pytest.mark.parametrize("T,d,w,with_doc", [
+    (64, 32, 16, False),
+    (130, 64, 50, False),
+    (200, 128, 129, True),
+    (150, 64, 1, True),
+])
+def test_window_against_torch_sdpa_fp64(T, d, w, with_doc):
+    B, H = 2, 2
+    q, k, v, do = (t.to(torch.float64).numpy() for t in inputs.make_qkvdo(B, H, T, d, 88))
+    scale = inputs.fp32_scale(d)
+    doc = inputs.random_doc_start(B, T, 8, 40, 91).numpy() if with_doc else None
+    o, lse = oracle.attention_forward(q, k, v, scale, doc, window=w)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, scale, doc, window=w)
+    ro, rl, rq, rk, rv = torch_band_reference(q, k, v, do, scale, w, doc)
+    for a, b in ((o, ro), (lse, rl), (dq, rq), (dk, rk), (dv, rv)):
+        assert np.max(np.abs(a - b)) <= 1e-10
