@@ -41,6 +41,9 @@ _f = ctypes.c_float
 SIGNATURES = {
     "gpt_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
+    "gpt_attn_fwd_window": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _i, _vp], _i),
+    "gpt_attn_bwd_window": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f,
+                             _vp, _i, _vp], _i),
     "gpt_attn_bwd_preprocess": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "gpt_attn_bwd_dkdv": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_bwd_dq": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
@@ -162,6 +165,33 @@ def gpt_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, scale: float, doc_
         _doc_ptr(doc_offsets, B, T), _stream(stream)))
 
 
+def gpt_attn_fwd_window(q, k, v, o, lse, scale: float, window: int, doc_offsets=None,
+                        stream=None) -> None:
+    """gpt_attn_fwd with a sliding window: i attends to j iff i - window < j <= i."""
+    B, H, T, d = _bhtd("q", q)
+    _bhtd("k", k, q)
+    _bhtd("v", v, q)
+    _bhtd("o", o, q)
+    _side("lse", lse, (B, H, T), torch.float32)
+    _check("gpt_attn_fwd_window", load().gpt_attn_fwd_window(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, d,
+        float(scale), _doc_ptr(doc_offsets, B, T), int(window), _stream(stream)))
+
+
+def gpt_attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, scale: float, window: int,
+                        doc_offsets=None, stream=None) -> None:
+    """gpt_attn_bwd with a sliding window (the one the forward used)."""
+    B, H, T, d = _bhtd("q", q)
+    for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _bhtd(name, t, q)
+    _side("lse", lse, (B, H, T), torch.float32)
+    _side("delta_ws", delta_ws, (B, H, T), torch.float32)
+    _check("gpt_attn_bwd_window", load().gpt_attn_bwd_window(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), delta_ws.data_ptr(), B, H, T, d, float(scale),
+        _doc_ptr(doc_offsets, B, T), int(window), _stream(stream)))
+
+
 def gpt_attn_bwd_static_ws(q, k, v, o, dout, lse, dq, dk, dv, scale: float, doc_offsets=None,
                            stream=None) -> None:
     """gpt_attn_bwd without a caller workspace: for callers that cannot allocate device memory
@@ -235,26 +265,36 @@ def gpt_attn_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
 
 # ------------------------------------------------------------ conveniences
 
-def attention_forward(q, k, v, scale: Optional[float] = None, doc_offsets=None, stream=None):
-    """Allocates O [B,H,T,d] bf16 and LSE [B,H,T] fp32 and runs gpt_attn_fwd."""
+def attention_forward(q, k, v, scale: Optional[float] = None, doc_offsets=None, stream=None,
+                      window: Optional[int] = None):
+    """Allocates O [B,H,T,d] bf16 and LSE [B,H,T] fp32 and runs gpt_attn_fwd (or, with a
+    window, gpt_attn_fwd_window)."""
     B, H, T, d = _bhtd("q", q)
     if scale is None:
         scale = d ** -0.5
     o = torch.empty_like(q)
     lse = torch.empty(B, H, T, device=q.device, dtype=torch.float32)
-    gpt_attn_fwd(q, k, v, o, lse, scale, doc_offsets, stream)
+    if window is None:
+        gpt_attn_fwd(q, k, v, o, lse, scale, doc_offsets, stream)
+    else:
+        gpt_attn_fwd_window(q, k, v, o, lse, scale, window, doc_offsets, stream)
     return o, lse
 
 
 def attention_backward(q, k, v, o, lse, dout, scale: Optional[float] = None, doc_offsets=None,
-                       stream=None):
-    """Allocates dQ, dK, dV and the delta workspace and runs gpt_attn_bwd."""
+                       stream=None, window: Optional[int] = None):
+    """Allocates dQ, dK, dV and the delta workspace and runs gpt_attn_bwd (or, with a
+    window, gpt_attn_bwd_window)."""
     B, H, T, d = _bhtd("q", q)
     if scale is None:
         scale = d ** -0.5
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     delta = torch.empty(B, H, T, device=q.device, dtype=torch.float32)
-    gpt_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta, scale, doc_offsets, stream)
+    if window is None:
+        gpt_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta, scale, doc_offsets, stream)
+    else:
+        gpt_attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, delta, scale, window, doc_offsets,
+                            stream)
     return dq, dk, dv
 
 

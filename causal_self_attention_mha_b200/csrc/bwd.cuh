@@ -58,6 +58,7 @@ struct BwdParams {
   __nv_bfloat16* g1;      // dV (dkdv kernel) or unused
   int H, T, BH, n_t;      // n_t = number of 128-row tiles along T
   int n_items;            // n_t * BH work items (one 128-row tile of one head each)
+  int window;             // keys a query sees, itself included (T: no window)
   float scale;            // softmax scale (1/sqrt(d))
   float scale_log2;       // scale * log2(e)
   uint64_t wait_limit_ns;
@@ -160,6 +161,12 @@ __device__ __forceinline__ DkdvItem dkdv_item(const BwdParams& p, int w) {
     }
     i_hi = (lo - 1) / kRows;
     i_hi = i_hi < I.jt ? I.jt : (i_hi > p.n_t - 1 ? p.n_t - 1 : i_hi);
+  }
+  {  // the last query that still has the tile's last key in its window
+    const int c_last = (I.k0 + kRows - 1 < p.T) ? I.k0 + kRows - 1 : p.T - 1;
+    const int r_max = c_last + p.window - 1;
+    const int i_w = r_max / kRows;
+    i_hi = i_w < i_hi ? i_w : i_hi;
   }
   I.n = i_hi - I.i_lo + 1;
   return I;
@@ -471,7 +478,7 @@ __global__ void __launch_bounds__(384, 1)
         reg_fence(sr[1]);
         // no mask needed when all my query rows are at or below this key, before T,
         // and in its document (document starts never decrease along the rows)
-        const bool full = (r0 >= c) && (r0 + 63 < T) && (dlast <= c);
+        const bool full = (r0 >= c) && (r0 + 63 < T) && (dlast <= c) && (r0 + 63 <= c + p.window - 1);
         if (__any_sync(0xffffffffu, !full)) {
           int n_vis;  // rows r0 .. r0 + n_vis - 1 are in c's document or an earlier one, and < T
           if (drow) {
@@ -482,9 +489,10 @@ __global__ void __launch_bounds__(384, 1)
           } else {
             n_vis = T - r0 < 0 ? 0 : (T - r0 > 64 ? 64 : T - r0);
           }
+          const int r_win = c + p.window - 1 - r0;  // my key leaves the window after row r0 + r_win
 #pragma unroll
           for (int e = 0; e < 64; ++e)
-            if (e >= n_vis || r0 + e < c) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf: weight 0
+            if (e >= n_vis || r0 + e < c || e > r_win) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf
         }
         // P^T = exp2(S^T * scale * log2e - LSE * log2e), kept in fp32 for dS^T; each half of
         // my columns goes to the dV MMA as soon as it is in TMEM
@@ -633,11 +641,14 @@ __device__ __forceinline__ DqItem dq_item(const BwdParams& p, int w) {
   I.bh = w % p.BH;
   I.b = I.bh / p.H;
   I.q0 = I.qt * kRows;
-  I.kv_lo = 0;
-  if (p.doc) {  // no key before the document start of the tile's first row is visible
-    const int lo = p.doc[(size_t)I.b * p.T + I.q0] / kRows;
-    I.kv_lo = lo < 0 ? 0 : (lo > I.qt ? I.qt : lo);
+  // no key before the tile's first row's document start or window start is visible
+  int first = I.q0 - p.window + 1;
+  if (p.doc) {
+    const int ds = p.doc[(size_t)I.b * p.T + I.q0];
+    first = first > ds ? first : ds;
   }
+  const int lo = first < 0 ? 0 : first / kRows;
+  I.kv_lo = lo > I.qt ? I.qt : lo;
   I.n = I.qt - I.kv_lo + 1;
   return I;
 }
@@ -884,7 +895,9 @@ __global__ void __launch_bounds__(384, 1)
       // rows past T: -LSE = -inf makes every weight zero
       const float nlse2 = (r < T) ? -p.lse[(size_t)I.bh * T + r] * kLog2e : -INFINITY;
       const float ndlt = (r < T) ? -p.delta[(size_t)I.bh * T + r] : 0.f;
-      const int ds = p.doc ? p.doc[(size_t)I.b * T + (r < T ? r : T - 1)] : 0;
+      // first visible key of this row: its document start or the window's start
+      int ds = p.doc ? p.doc[(size_t)I.b * T + (r < T ? r : T - 1)] : 0;
+      ds = ds > r - p.window + 1 ? ds : r - p.window + 1;
       const uint64_t nlse2x2 = f2(nlse2, nlse2), ndltx2 = f2(ndlt, ndlt);
       for (int it = 0; it < I.n; ++it, ++gk) {
         const int t = gk;

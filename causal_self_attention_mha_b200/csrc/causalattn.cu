@@ -153,9 +153,13 @@ int launch_status() {
 }
 
 // ------------------------------------------------------------- launchers
+// A window of w keys (the query's own included); w <= 0 or w >= T is no window,
+// which the kernels express as w = T (the band then covers every causal key).
+int effective_window(int window, int T) { return (window <= 0 || window > T) ? T : window; }
+
 template <int D>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
-             float scale, const int32_t* doc, cudaStream_t st) {
+             float scale, const int32_t* doc, int window, cudaStream_t st) {
   const int BH = B * H;
   CUtensorMap mq, mk, mv, mo;
   if (!make_map<D>(&mq, q, BH, T) || !make_map<D>(&mk, k, BH, T) || !make_map<D>(&mv, v, BH, T) ||
@@ -172,6 +176,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.n_pairs = (p.n_qt + 1) / 2;
   p.n_items = p.n_pairs * BH;
   p.scale_log2 = scale * ca::kLog2e;
+  p.window = effective_window(window, T);
   p.wait_limit_ns = kWaitLimitNs;
   // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
   const int sms = sm_count();
@@ -196,7 +201,7 @@ int delta_impl(const void* o, const void* dout, float* delta, int B, int H, int 
 template <int D>
 int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const void* dout,
                    const float* lse, const float* delta, void* g0, void* g1, int B, int H, int T,
-                   float scale, const int32_t* doc, cudaStream_t st) {
+                   float scale, const int32_t* doc, int window, cudaStream_t st) {
   const int BH = B * H;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map<D>(&mq, q, BH, T) || !make_map<D>(&mk, k, BH, T) || !make_map<D>(&mv, v, BH, T) ||
@@ -215,6 +220,7 @@ int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const
   p.n_items = p.n_t * BH;
   p.scale = scale;
   p.scale_log2 = scale * ca::kLog2e;
+  p.window = effective_window(window, T);
   p.wait_limit_ns = kWaitLimitNs;
   // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
   const int sms = sm_count();
@@ -289,8 +295,9 @@ const char* gpt_attn_strerror(int s) {
   }
 }
 
-int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                 int T, int d, float scale, const int32_t* doc_offsets, void* stream) {
+static int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int T, int d, float scale, const int32_t* doc_offsets, int window,
+                     void* stream) {
   if (!q || !k || !v || !o || !lse) return GPT_ATTN_ERR_NULL_PTR;
   int s = common_checks(B, H, T, d);
   if (s) return s;
@@ -301,10 +308,21 @@ int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if ((s = ensure_device())) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 32: return fwd_impl<32>(q, k, v, o, lse, B, H, T, scale, doc_offsets, st);
-    case 64: return fwd_impl<64>(q, k, v, o, lse, B, H, T, scale, doc_offsets, st);
-    default: return fwd_impl<128>(q, k, v, o, lse, B, H, T, scale, doc_offsets, st);
+    case 32: return fwd_impl<32>(q, k, v, o, lse, B, H, T, scale, doc_offsets, window, st);
+    case 64: return fwd_impl<64>(q, k, v, o, lse, B, H, T, scale, doc_offsets, window, st);
+    default: return fwd_impl<128>(q, k, v, o, lse, B, H, T, scale, doc_offsets, window, st);
   }
+}
+
+int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int T, int d, float scale, const int32_t* doc_offsets, void* stream) {
+  return fwd_entry(q, k, v, o, lse, B, H, T, d, scale, doc_offsets, 0, stream);
+}
+
+int gpt_attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int T, int d, float scale, const int32_t* doc_offsets, int window,
+                        void* stream) {
+  return fwd_entry(q, k, v, o, lse, B, H, T, d, scale, doc_offsets, window, stream);
 }
 
 int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B, int H, int T,
@@ -324,7 +342,7 @@ int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B
 
 static int bwd_step(bool dkdv, const void* q, const void* k, const void* v, const void* dout,
                     const float* lse, const float* delta, void* g0, void* g1, int B, int H, int T,
-                    int d, float scale, const int32_t* doc, void* stream) {
+                    int d, float scale, const int32_t* doc, int window, void* stream) {
   if (!q || !k || !v || !dout || !lse || !delta || !g0 || (dkdv && !g1))
     return GPT_ATTN_ERR_NULL_PTR;
   int s = common_checks(B, H, T, d);
@@ -337,28 +355,32 @@ static int bwd_step(bool dkdv, const void* q, const void* k, const void* v, cons
   if ((s = ensure_device())) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d) {
-    case 32: return bwd_tiled_impl<32>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, st);
-    case 64: return bwd_tiled_impl<64>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, st);
-    default: return bwd_tiled_impl<128>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, st);
+    case 32:
+      return bwd_tiled_impl<32>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, window, st);
+    case 64:
+      return bwd_tiled_impl<64>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, window, st);
+    default:
+      return bwd_tiled_impl<128>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, window, st);
   }
 }
 
 int gpt_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
                       const float* lse, const float* delta, void* dk, void* dv, int B, int H,
                       int T, int d, float scale, const int32_t* doc_offsets, void* stream) {
-  return bwd_step(true, q, k, v, dout, lse, delta, dk, dv, B, H, T, d, scale, doc_offsets, stream);
+  return bwd_step(true, q, k, v, dout, lse, delta, dk, dv, B, H, T, d, scale, doc_offsets, 0, stream);
 }
 
 int gpt_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
                     const float* lse, const float* delta, void* dq, int B, int H, int T, int d,
                     float scale, const int32_t* doc_offsets, void* stream) {
-  return bwd_step(false, q, k, v, dout, lse, delta, dq, nullptr, B, H, T, d, scale, doc_offsets,
+  return bwd_step(false, q, k, v, dout, lse, delta, dq, nullptr, B, H, T, d, scale, doc_offsets, 0,
                   stream);
 }
 
-int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                 const float* lse, void* dq, void* dk, void* dv, float* delta_ws, int B, int H,
-                 int T, int d, float scale, const int32_t* doc_offsets, void* stream) {
+static int bwd_entry(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv, float* delta_ws, int B, int H,
+                     int T, int d, float scale, const int32_t* doc_offsets, int window,
+                     void* stream) {
   // validate everything before the first launch, so an error never leaves a partial backward
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !delta_ws)
     return GPT_ATTN_ERR_NULL_PTR;
@@ -371,10 +393,26 @@ int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
     return GPT_ATTN_ERR_MISALIGNED;
   if ((s = ensure_device())) return s;
   if ((s = gpt_attn_bwd_preprocess(o, dout, delta_ws, B, H, T, d, stream))) return s;
-  if ((s = gpt_attn_bwd_dkdv(q, k, v, dout, lse, delta_ws, dk, dv, B, H, T, d, scale, doc_offsets,
-                             stream)))
+  if ((s = bwd_step(true, q, k, v, dout, lse, delta_ws, dk, dv, B, H, T, d, scale, doc_offsets,
+                    window, stream)))
     return s;
-  return gpt_attn_bwd_dq(q, k, v, dout, lse, delta_ws, dq, B, H, T, d, scale, doc_offsets, stream);
+  return bwd_step(false, q, k, v, dout, lse, delta_ws, dq, nullptr, B, H, T, d, scale, doc_offsets,
+                  window, stream);
+}
+
+int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, float* delta_ws, int B, int H,
+                 int T, int d, float scale, const int32_t* doc_offsets, void* stream) {
+  return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, B, H, T, d, scale, doc_offsets, 0,
+                   stream);
+}
+
+int gpt_attn_bwd_window(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        float* delta_ws, int B, int H, int T, int d, float scale,
+                        const int32_t* doc_offsets, int window, void* stream) {
+  return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, B, H, T, d, scale, doc_offsets,
+                   window, stream);
 }
 
 int gpt_attn_check_doc_offsets(const int32_t* doc_offsets, int B, int T, void* stream) {

@@ -53,6 +53,7 @@ struct FwdParams {
   __nv_bfloat16* o;       // [B, H, T, D]
   float* lse;             // [B, H, T]
   int H, T, BH, n_qt, n_pairs, n_items;
+  int window;             // keys a query sees, itself included (T: no window)
   float scale_log2;       // scale * log2(e)
   uint64_t wait_limit_ns;
 };
@@ -96,9 +97,16 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
   I.hasB = I.qt[1] < p.n_qt;
   for (int x = 0; x < 2; ++x) {
     int lo = 0;
-    if (p.doc && (x == 0 || I.hasB)) {
-      lo = p.doc[(size_t)I.b * p.T + I.qt[x] * kRows] / kRows;
-      lo = lo < 0 ? 0 : (lo > I.qt[x] ? I.qt[x] : lo);
+    if (x == 0 || I.hasB) {
+      // the first key any row of the tile sees: its first row's window / document start
+      const int q0 = I.qt[x] * kRows;
+      int first = q0 - p.window + 1;
+      if (p.doc) {
+        const int ds = p.doc[(size_t)I.b * p.T + q0];
+        first = first > ds ? first : ds;
+      }
+      lo = first < 0 ? 0 : first / kRows;
+      lo = lo > I.qt[x] ? I.qt[x] : lo;
     }
     I.lo[x] = lo;
     I.hi[x] = I.qt[x];
@@ -365,7 +373,9 @@ __global__ void __launch_bounds__(384, 1)
       u0 += I.hasB ? 2 : 1;
       if (x == 1 && !I.hasB) continue;
       const int row = I.qt[x] * kRows + rl;
-      const int ds = p.doc ? p.doc[(size_t)I.b * T + (row < T ? row : T - 1)] : 0;
+      // first visible key of this row: its document start or the window's start
+      int ds = p.doc ? p.doc[(size_t)I.b * T + (row < T ? row : T - 1)] : 0;
+      ds = ds > row - p.window + 1 ? ds : row - p.window + 1;
       float m = -INFINITY;
       // acc_l: sum of the fp32 weights (for the LSE); acc_lr: sum of the bf16-rounded weights
       // the PV MMA actually multiplies (for normalising O).  Packed pairs, independent chains.

@@ -99,6 +99,26 @@ int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
                  const float* lse, void* dq, void* dk, void* dv, float* delta_ws, int B, int H,
                  int T, int d, float scale, const int32_t* doc_offsets, void* stream);
 
+/*
+ * Sliding-window variants.  "How to build an LLM by hand" (agmtopy.github.io),
+ * section 9 (the gpt.py walkthrough), lists sliding-window attention among the
+ * model's attention features without defining it.  Reading: a window of
+ * `window` keys, the query's own position included: position i attends to j
+ * iff i - window < j <= i, and, with doc_offsets, also doc_offsets[b,i] <= j.
+ * window <= 0 or window >= T is plain (document-)causal attention, identical
+ * to gpt_attn_fwd / gpt_attn_bwd.  Everything else (layouts, ownership,
+ * asynchrony, errors, limits) is as for those calls; the backward must be
+ * given the same window as the forward that produced o and lse.
+ */
+int gpt_attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int T, int d, float scale, const int32_t* doc_offsets, int window,
+                        void* stream);
+
+int gpt_attn_bwd_window(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        float* delta_ws, int B, int H, int T, int d, float scale,
+                        const int32_t* doc_offsets, int window, void* stream);
+
 /* Backward step 1: delta[b,h,i] = sum_c dout[b,h,i,c] * o[b,h,i,c] (fp32). */
 int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B, int H, int T,
                             int d, void* stream);

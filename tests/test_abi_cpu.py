@@ -92,6 +92,28 @@ def test_bwd_argument_errors(lib):
     assert lib.gpt_attn_device_status(None, 0) == abi.GPT_ATTN_ERR_NULL_PTR
 
 
+def test_window_entry_points_validate_like_the_plain_ones(lib):
+    def fw(q=P[0], B=1, d=64, window=16, scale=0.125):
+        return lib.gpt_attn_fwd_window(q, P[1], P[2], P[3], P[4], B, 2, 64, d, scale, None,
+                                       window, None)
+
+    def bw(dq=P[6], T=64, d=64, window=16):
+        return lib.gpt_attn_bwd_window(P[0], P[1], P[2], P[3], P[5], P[4], dq, P[7], P[8], P[9],
+                                       1, 2, T, d, 0.125, None, window, None)
+    assert fw(q=None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert fw(B=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    assert fw(d=48) == abi.GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM
+    assert fw(scale=-1.0) == abi.GPT_ATTN_ERR_BAD_SCALE
+    assert fw(q=P[0] + 2) == abi.GPT_ATTN_ERR_MISALIGNED
+    assert bw(dq=None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert bw(T=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    assert bw(d=96) == abi.GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM
+    if not torch.cuda.is_available():  # any window value is valid: only the device is missing
+        for w in (-5, 0, 1, 63, 64, 10 ** 6):
+            assert fw(window=w) == abi.GPT_ATTN_ERR_NO_DEVICE
+            assert bw(window=w) == abi.GPT_ATTN_ERR_NO_DEVICE
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_valid_arguments_without_a_gpu_report_no_device(lib):
     assert fwd(lib) == abi.GPT_ATTN_ERR_NO_DEVICE

@@ -25,24 +25,25 @@ pytestmark = pytest.mark.gpu
 O_TOL, LSE_TOL, GRAD_TOL = 1e-2, 1e-3, 2e-2
 
 
-def run_gpu(q, k, v, do, doc, scale):
+def run_gpu(q, k, v, do, doc, scale, window=None):
     dev = torch.device("cuda:0")
     q, k, v, do = (t.to(dev).contiguous() for t in (q, k, v, do))
     docd = doc.to(dev).contiguous() if doc is not None else None
-    o, lse = abi.attention_forward(q, k, v, scale, docd)
-    dq, dk, dv = abi.attention_backward(q, k, v, o, lse, do, scale, docd)
+    o, lse = abi.attention_forward(q, k, v, scale, docd, window=window)
+    dq, dk, dv = abi.attention_backward(q, k, v, o, lse, do, scale, docd, window=window)
     torch.cuda.synchronize()
     return [t.cpu() for t in (o, lse, dq, dk, dv)]
 
 
-def oracle_heads(q, k, v, do, doc, scale, heads, with_grad=True):
+def oracle_heads(q, k, v, do, doc, scale, heads, with_grad=True, window=None):
     """Oracle outputs for the listed (b, h) pairs: dict (b,h) -> (o, lse, dq, dk, dv)."""
     out = {}
     for b, h in heads:
         sl = lambda t: t[b:b + 1, h:h + 1]
         ds = doc[b:b + 1] if doc is not None else None
-        o, lse = oracle.attention_forward(sl(q), sl(k), sl(v), scale, ds)
-        g = oracle.attention_backward(sl(q), sl(k), sl(v), sl(do), scale, ds) if with_grad else None
+        o, lse = oracle.attention_forward(sl(q), sl(k), sl(v), scale, ds, window=window)
+        g = (oracle.attention_backward(sl(q), sl(k), sl(v), sl(do), scale, ds, window=window)
+             if with_grad else None)
         out[(b, h)] = (o, lse, g)
     return out
 
@@ -54,19 +55,19 @@ def rel_l2(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), floor))
 
 
-def compare(gpu, q, k, v, do, doc, scale, grad_heads=None, label=""):
+def compare(gpu, q, k, v, do, doc, scale, grad_heads=None, label="", window=None):
     """Forward on every head (one oracle call); backward on grad_heads (None = all)."""
     o_g, lse_g, dq_g, dk_g, dv_g = (t.to(torch.float64).numpy() for t in gpu)
     B, H = q.shape[:2]
-    o_r, lse_r = oracle.attention_forward(q, k, v, scale, doc)
+    o_r, lse_r = oracle.attention_forward(q, k, v, scale, doc, window=window)
     err_o = float(np.max(np.abs(o_g - o_r)))
     err_l = float(np.max(np.abs(lse_g - lse_r)))
     if grad_heads is None:
-        dq_r, dk_r, dv_r = oracle.attention_backward(q, k, v, do, scale, doc)
+        dq_r, dk_r, dv_r = oracle.attention_backward(q, k, v, do, scale, doc, window=window)
         sel = (slice(None), slice(None))
         errs = [rel_l2(g[sel], r) for g, r in ((dq_g, dq_r), (dk_g, dk_r), (dv_g, dv_r))]
     else:
-        ref = oracle_heads(q, k, v, do, doc, scale, grad_heads)
+        ref = oracle_heads(q, k, v, do, doc, scale, grad_heads, window=window)
         errs = []
         for i, g in enumerate((dq_g, dk_g, dv_g)):
             gs = np.concatenate([g[b, h].ravel() for b, h in grad_heads])
@@ -152,6 +153,45 @@ def test_deterministic(cuda_device):
     b = run_gpu(q, k, v, do, doc, w.scale)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+# ---------------------------------------------------------- sliding window
+
+@pytest.mark.parametrize("T,d,w", [
+    (300, 64, 1), (300, 64, 64), (300, 128, 127), (333, 32, 128), (333, 64, 129),
+    (513, 128, 200), (257, 64, 256), (700, 128, 384),
+])
+@pytest.mark.parametrize("with_doc", [False, True])
+def test_sliding_window(T, d, w, with_doc, cuda_device):
+    """Band of w keys (i - w < j <= i), alone and with document masks, every tile edge case."""
+    B, H = 2, 2
+    q, k, v, do = inputs.make_qkvdo(B, H, T, d, 61 + w)
+    doc = inputs.random_doc_start(B, T, 11, 30, 200) if with_doc else None
+    scale = inputs.fp32_scale(d)
+    compare(run_gpu(q, k, v, do, doc, scale, window=w), q, k, v, do, doc, scale,
+            label=f"window{w}_T{T}_d{d}_doc{int(with_doc)}", window=w)
+    no_device_timeouts()
+
+
+def test_window_at_least_t_is_plain_causal(cuda_device):
+    """window >= T (and window <= 0) must give bit-for-bit the plain causal results."""
+    B, H, T, d = 1, 3, 260, 128
+    q, k, v, do = inputs.make_qkvdo(B, H, T, d, 71)
+    scale = inputs.fp32_scale(d)
+    base = run_gpu(q, k, v, do, None, scale)
+    for w in (T, T + 5, 0, -3):
+        for a, b in zip(run_gpu(q, k, v, do, None, scale, window=w), base):
+            assert torch.equal(a, b), w
+
+
+def test_window_full_size_workload(cuda_device):
+    """wide_d128 with a 512-key window in the benchmark's launch configuration: forward on
+    every head, gradients on sampled heads."""
+    w = inputs.WORKLOADS["wide_d128"]
+    q, k, v, do, doc = inputs.make_workload(w)
+    compare(run_gpu(q, k, v, do, doc, w.scale, window=512), q, k, v, do, doc, w.scale,
+            grad_heads=sampled_heads(w.B, w.H, 4), label="wide_d128_window512", window=512)
+    no_device_timeouts()
 
 
 def test_host_stream_matches_device_path(cuda_device):
