@@ -151,3 +151,27 @@ def attention_backward(q, k, v, dout, scale: float, doc_start=None,
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd failed with code {rc}")
     return dq, dk, dv
+
+
+def decode_forward(q, k_cache, v_cache, scale: float):
+    """KV-cache decode, written out in numpy float64: new token t of Tq sits at position
+    L - Tq + t and attends to cache positions 0 .. L - Tq + t.  q: [B,Tq,H,d];
+    k_cache, v_cache: [B,L,H,d].  Returns O [B,Tq,H,d] and LSE [B,H,Tq] (natural log)."""
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    B, Tq, H, d = q.shape
+    L = kc.shape[1]
+    if kc.shape != (B, L, H, d) or vc.shape != kc.shape or Tq > L:
+        raise ValueError("q [B,Tq,H,d], k_cache / v_cache [B,L,H,d], Tq <= L")
+    o = np.empty((B, Tq, H, d))
+    lse = np.empty((B, H, Tq))
+    for b in range(B):
+        for h in range(H):
+            for t in range(Tq):
+                n = L - Tq + t + 1                       # visible cache positions
+                s = scale * (kc[b, :n, h, :] @ q[b, t, h, :])
+                m = s.max()
+                w = np.exp(s - m)
+                z = w.sum()
+                o[b, t, h] = (w / z) @ vc[b, :n, h, :]
+                lse[b, h, t] = m + np.log(z)
+    return o, lse

@@ -408,3 +408,49 @@ def test_window_against_torch_sdpa_fp64(T, d, w, with_doc):
     ro, rl, rq, rk, rv = torch_band_reference(q, k, v, do, scale, w, doc)
     for a, b in ((o, ro), (lse, rl), (dq, rq), (dk, rk), (dv, rv)):
         assert np.max(np.abs(a - b)) <= 1e-10
+
+
+# ---------------------------------------------------------------- KV-cache decode
+# The pages' inference engine attends from the new tokens to a KV cache ("How to
+# build an LLM by hand", section 2); new token t of Tq sits at position L - Tq + t.
+
+def _decode_case(B, H, Tq, L, d, seed):
+    q = rnd((B, Tq, H, d), seed)
+    kc, vc = rnd((B, L, H, d), seed + 1), rnd((B, L, H, d), seed + 2)
+    return q, kc, vc
+
+
+@pytest.mark.parametrize("B,H,Tq,L,d", [(1, 2, 1, 1, 4), (2, 3, 1, 37, 8), (1, 2, 5, 20, 4),
+                                        (2, 1, 7, 7, 6)])
+def test_decode_is_the_last_rows_of_causal_attention(B, H, Tq, L, d):
+    """The numpy decode oracle equals the C causal oracle's last Tq rows, with the new tokens'
+    queries placed at the end of an otherwise arbitrary query sequence."""
+    q, kc, vc = _decode_case(B, H, Tq, L, d, 600 + L)
+    o, lse = oracle.decode_forward(q, kc, vc, 0.45)
+    qfull = rnd((B, H, L, d), 700 + L)
+    qfull[:, :, L - Tq:, :] = q.transpose(0, 2, 1, 3)
+    of, lf = oracle.attention_forward(qfull, kc.transpose(0, 2, 1, 3), vc.transpose(0, 2, 1, 3), 0.45)
+    np.testing.assert_allclose(o.transpose(0, 2, 1, 3), of[:, :, L - Tq:], atol=1e-13)
+    np.testing.assert_allclose(lse, lf[:, :, L - Tq:], atol=1e-13)
+
+
+def test_decode_single_cached_token():
+    """L = 1: the one new token sees only itself: O = v_0, LSE = scale <q, k_0>."""
+    q, kc, vc = _decode_case(2, 2, 1, 1, 5, 650)
+    o, lse = oracle.decode_forward(q, kc, vc, 0.8)
+    np.testing.assert_array_equal(o, vc)
+    np.testing.assert_allclose(lse, 0.8 * np.einsum("bthc,bthc->bht", q, kc), atol=1e-13)
+
+
+def test_decode_against_torch_sdpa_fp64():
+    B, H, Tq, L, d = 2, 3, 4, 90, 16
+    q, kc, vc = _decode_case(B, H, Tq, L, d, 660)
+    o, lse = oracle.decode_forward(q, kc, vc, 0.25)
+    tq, tk, tv = (torch.tensor(a, dtype=torch.float64).transpose(1, 2) for a in (q, kc, vc))
+    pos = torch.arange(L - Tq, L).view(Tq, 1)
+    mask = torch.arange(L).view(1, L) <= pos
+    ro = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.25)
+    s = torch.einsum("bhtc,bhjc->bhtj", tq, tk) * 0.25
+    rl = torch.logsumexp(s.masked_fill(~mask, float("-inf")), dim=-1)
+    assert np.max(np.abs(o - ro.transpose(1, 2).numpy())) <= 1e-12
+    assert np.max(np.abs(lse - rl.numpy())) <= 1e-12
