@@ -44,6 +44,9 @@ SIGNATURES = {
     "gpt_attn_fwd_window": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _i, _vp], _i),
     "gpt_attn_bwd_window": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f,
                              _vp, _i, _vp], _i),
+    "gpt_attn_decode_workspace_size": ([_i, _i, _i, _i, _i], ctypes.c_size_t),
+    "gpt_attn_decode": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _i, _f, _vp],
+                        _i),
     "gpt_attn_bwd_preprocess": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "gpt_attn_bwd_dkdv": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_bwd_dq": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
@@ -239,6 +242,28 @@ def gpt_attn_bwd_dq(q, k, v, dout, lse, delta, dq, scale: float, doc_offsets=Non
         dq.data_ptr(), B, H, T, d, float(scale), _doc_ptr(doc_offsets, B, T), _stream(stream)))
 
 
+def gpt_attn_decode_workspace_size(B: int, H: int, Tq: int, L: int, d: int) -> int:
+    return int(load().gpt_attn_decode_workspace_size(B, H, Tq, L, d))
+
+
+def gpt_attn_decode(q, k_cache, v_cache, o, lse, workspace, scale: float, stream=None) -> None:
+    """q, o: bf16 [B,Tq,H,d]; k_cache, v_cache: bf16 [B,L,H,d]; lse fp32 [B,H,Tq];
+    workspace: a CUDA tensor of at least gpt_attn_decode_workspace_size bytes."""
+    B, Tq, H, d = _bhtd("q", q)
+    Bk, L, Hk, dk = _bhtd("k_cache", k_cache)
+    if (Bk, Hk, dk) != (B, H, d):
+        raise ValueError("k_cache must be [B, L, H, d] with q's B, H, d")
+    _bhtd("v_cache", v_cache, k_cache)
+    _bhtd("o", o, q)
+    _side("lse", lse, (B, H, Tq), torch.float32)
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check("gpt_attn_decode", load().gpt_attn_decode(
+        q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), o.data_ptr(), lse.data_ptr(),
+        workspace.data_ptr(), nbytes, B, H, Tq, L, d, float(scale), _stream(stream)))
+
+
 def gpt_attn_check_doc_offsets(doc_offsets, stream=None) -> bool:
     """True when the [B,T] int32 device array is a valid document-start array."""
     if not isinstance(doc_offsets, torch.Tensor) or doc_offsets.dim() != 2:
@@ -296,6 +321,20 @@ def attention_backward(q, k, v, o, lse, dout, scale: Optional[float] = None, doc
         gpt_attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, delta, scale, window, doc_offsets,
                             stream)
     return dq, dk, dv
+
+
+def attention_decode(q, k_cache, v_cache, scale: Optional[float] = None, stream=None):
+    """Allocates O [B,Tq,H,d] bf16, LSE [B,H,Tq] fp32 and the workspace; runs gpt_attn_decode."""
+    B, Tq, H, d = _bhtd("q", q)
+    L = k_cache.shape[1]
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, Tq, device=q.device, dtype=torch.float32)
+    ws = torch.empty(max(gpt_attn_decode_workspace_size(B, H, Tq, L, d), 16), device=q.device,
+                     dtype=torch.uint8)
+    gpt_attn_decode(q, k_cache, v_cache, o, lse, ws, scale, stream)
+    return o, lse
 
 
 class CausalSelfAttentionFunction(torch.autograd.Function):

@@ -14,6 +14,7 @@
 
 #include "../../include/causalattn.h"
 #include "bwd.cuh"
+#include "decode.cuh"
 #include "fwd.cuh"
 
 namespace {
@@ -50,6 +51,9 @@ cudaError_t set_smem_attrs() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(ca::attn_bwd_dkdv_kernel<D>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DkdvLayout<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D>::SMEM);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(ca::attn_bwd_dq_kernel<D>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DqLayout<D>::SMEM);
@@ -131,6 +135,25 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int T) {
   cuuint32_t box[3] = {(cuuint32_t)Tl::BOX_COLS, (cuuint32_t)ca::kRows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   Tl::SW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// A [B, L, H, d] bf16 KV cache (the layout of the pages' kv-cache call) viewed as 4-D
+// (d, H, L, B) with boxes of (swizzle width, 1 head, 128 rows, 1 batch); rows past L read
+// as zero.  The staged box has the same shared-memory image as make_map's tiles.
+template <int D>
+bool make_cache_map(CUtensorMap* m, const void* base, int B, int L, int H) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  using Tl = ca::Tile<D>;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)L * H * D * 2};
+  cuuint32_t box[4] = {(cuuint32_t)Tl::BOX_COLS, 1, (cuuint32_t)ca::kDecChunk, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    Tl::SW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -236,6 +259,41 @@ int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const
     ca::attn_bwd_dq_kernel<D><<<grid, ca::DqLayout<D>::THREADS, ca::DqLayout<D>::SMEM, st>>>(
         mq, mk, mv, mdo, mg0, p);
   return launch_status();
+}
+
+template <int D>
+int decode_impl(const void* q, const void* kc, const void* vc, void* o, float* lse, float* ws,
+                int B, int H, int Tq, int L, float scale, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  if (!make_cache_map<D>(&mk, kc, B, L, H) || !make_cache_map<D>(&mv, vc, B, L, H))
+    return GPT_ATTN_ERR_LAUNCH;
+  ca::DecParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.B = B;
+  p.H = H;
+  p.Tq = Tq;
+  p.L = L;
+  p.n_chunks = (L + ca::kDecChunk - 1) / ca::kDecChunk;
+  const size_t rows = (size_t)B * H * Tq * p.n_chunks;
+  p.part_ml = ws;
+  p.part_o = ws + rows * 2;
+  p.scale_log2 = scale * ca::kLog2e;
+  p.wait_limit_ns = kWaitLimitNs;
+  dim3 grid((unsigned)p.n_chunks, (unsigned)H, (unsigned)B);
+  ca::attn_decode_chunk_kernel<D><<<grid, ca::kDecThreads, ca::DecLayout<D>::SMEM, st>>>(mk, mv, p);
+  int s = launch_status();
+  if (s) return s;
+  ca::attn_decode_combine_kernel<D><<<(unsigned)(B * H * Tq), D, 0, st>>>(
+      p.part_ml, p.part_o, static_cast<__nv_bfloat16*>(o), lse, H, Tq, p.n_chunks);
+  return launch_status();
+}
+
+// Workspace of gpt_attn_decode in bytes (0 for arguments it would reject).
+size_t decode_ws_bytes(int B, int H, int Tq, int L, int d) {
+  if (B < 1 || H < 1 || Tq < 1 || Tq > ca::kDecMaxTq || L < Tq) return 0;
+  if (d != 32 && d != 64 && d != 128) return 0;
+  const size_t chunks = ((size_t)L + ca::kDecChunk - 1) / ca::kDecChunk;
+  return (size_t)B * H * Tq * chunks * (2 + (size_t)d) * sizeof(float);
 }
 
 // -------------------------------------------------------- utility kernels
@@ -413,6 +471,35 @@ int gpt_attn_bwd_window(const void* q, const void* k, const void* v, const void*
                         const int32_t* doc_offsets, int window, void* stream) {
   return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, B, H, T, d, scale, doc_offsets,
                    window, stream);
+}
+
+size_t gpt_attn_decode_workspace_size(int B, int H, int Tq, int L, int d) {
+  return decode_ws_bytes(B, H, Tq, L, d);
+}
+
+int gpt_attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                    void* workspace, size_t workspace_bytes, int B, int H, int Tq, int L, int d,
+                    float scale, void* stream) {
+  if (!q || !k_cache || !v_cache || !o || !lse || !workspace) return GPT_ATTN_ERR_NULL_PTR;
+  if (B < 1 || H < 1 || Tq < 1 || L < 1 || Tq > L || Tq > ca::kDecMaxTq || H > 65535 || B > 65535)
+    return GPT_ATTN_ERR_BAD_SHAPE;
+  if (d != 32 && d != 64 && d != 128) return GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM;
+  if ((int64_t)B * L * H * d >= ((int64_t)1 << 31) || (int64_t)B * Tq * H * d >= ((int64_t)1 << 31))
+    return GPT_ATTN_ERR_TOO_LARGE;
+  int s;
+  if ((s = check_scale(scale))) return s;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(workspace, 16))
+    return GPT_ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < decode_ws_bytes(B, H, Tq, L, d)) return GPT_ATTN_ERR_BAD_SHAPE;
+  if ((s = ensure_device())) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  switch (d) {
+    case 32: return decode_impl<32>(q, k_cache, v_cache, o, lse, ws, B, H, Tq, L, scale, st);
+    case 64: return decode_impl<64>(q, k_cache, v_cache, o, lse, ws, B, H, Tq, L, scale, st);
+    default: return decode_impl<128>(q, k_cache, v_cache, o, lse, ws, B, H, Tq, L, scale, st);
+  }
 }
 
 int gpt_attn_check_doc_offsets(const int32_t* doc_offsets, int B, int T, void* stream) {

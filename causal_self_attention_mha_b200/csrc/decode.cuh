@@ -1,0 +1,209 @@
+// decode.cuh -- KV-cache decode attention on sm_100a.
+//
+// Generation appends Tq new tokens (1 in plain decoding, a few with
+// speculative drafts) to a cache of L keys and values and attends from each new
+// token to every cached position up to its own: query t sits at position
+// L - Tq + t and sees keys 0 .. L - Tq + t (the causal rule of the training
+// forward, restricted to the last Tq rows).  The pages' inference path
+// ("How to build an LLM by hand", agmtopy.github.io, section 2: nanochat's
+// engine keeps a KV cache and calls FlashAttention-3's kv-cache entry point on
+// (B, T, H, D) tensors) is what this reproduces; the cache uses that layout.
+//
+// The work is one pass over the cache, so the kernel is bound by HBM
+// bandwidth, not by arithmetic: each CTA takes one 128-key chunk of one
+// (batch, head), brings the chunk's K and V rows in by TMA (128-byte swizzle,
+// so that a thread per key row and a thread per column both read shared
+// memory without bank conflicts), and computes, for every new token, the
+// chunk's scores, their maximum, the sum of their exponentials and the
+// unnormalised weighted sum of V rows on CUDA cores (one key row or one
+// output column per thread).  A second kernel merges the chunks of each
+// (batch, head, token) in chunk order -- deterministic, no atomics.
+#pragma once
+
+#include "tiles.cuh"
+
+namespace ca {
+
+constexpr int kDecChunk = 128;   // keys per CTA (one TMA box of rows)
+constexpr int kDecThreads = 128;
+constexpr int kDecMaxTq = 16;    // new tokens per call
+
+struct DecParams {
+  const __nv_bfloat16* q;  // [B, Tq, H, D]
+  float* part_ml;          // [B, H, Tq, n_chunks, 2]: chunk max (base 2) and sum of 2^(s - max)
+  float* part_o;           // [B, H, Tq, n_chunks, D]: unnormalised sum of weights x V rows
+  int B, H, Tq, L, n_chunks;
+  float scale_log2;        // scale * log2(e)
+  uint64_t wait_limit_ns;
+};
+
+template <int D>
+struct DecLayout {
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = Tile<D>::BYTES;
+  static constexpr int Q_OFF = 2 * Tile<D>::BYTES;                 // fp32 [Tq][D], times scale*log2e
+  static constexpr int P_OFF = Q_OFF + kDecMaxTq * D * 4;          // fp32 [128] weights
+  static constexpr int RED_OFF = P_OFF + kDecChunk * 4;            // fp32 [2][4] warp partials
+  static constexpr int G = kDecThreads / D;                        // key groups in the V pass
+  static constexpr int ACC_OFF = RED_OFF + 64;                     // fp32 [G][D] group sums
+  static constexpr int BAR_OFF = ACC_OFF + G * D * 4;
+  static constexpr int MISC_OFF = BAR_OFF + 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+  static constexpr int SMEM = BYTES + 1024;
+};
+
+// Element (row r, column col) of a staged 128-row tile (the layout load_tile produces).
+template <int D>
+__device__ __forceinline__ uint32_t tile_elem_offset(int r, int col) {
+  using Tl = Tile<D>;
+  const int ch = col / Tl::BOX_COLS, cu = (col % Tl::BOX_COLS) / 8;
+  const int phys = (Tl::SW == 128) ? (cu ^ (r & 7)) : (cu ^ ((r >> 1) & 3));
+  return (uint32_t)(ch * Tl::CHUNK_BYTES + r * Tl::SW + phys * 16 + (col % 8) * 2);
+}
+
+// Block-wide reduction of one float per thread (max or sum) over the 4 warps.
+__device__ __forceinline__ float dec_block_reduce(float v, bool is_max, float* red) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < kDecThreads / 32; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  __syncthreads();  // red may be reused by the next reduction
+  return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads)
+    attn_decode_chunk_kernel(const __grid_constant__ CUtensorMap tmK,
+                             const __grid_constant__ CUtensorMap tmV, const DecParams p) {
+  using Tl = Tile<D>;
+  using L = DecLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* gsm;
+  const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
+  const uint8_t* sK = gsm + L::K_OFF;
+  const uint8_t* sV = gsm + L::V_OFF;
+  float* qs = reinterpret_cast<float*>(gsm + L::Q_OFF);
+  float* ps = reinterpret_cast<float*>(gsm + L::P_OFF);
+  float* red = reinterpret_cast<float*>(gsm + L::RED_OFF);
+  float* acc_s = reinterpret_cast<float*>(gsm + L::ACC_OFF);
+  const uint32_t bar = sbase + L::BAR_OFF;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF);
+
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {  // this chunk's 128 key and value rows of head h (rows past L read as zero)
+    mbar_arrive_expect_tx(bar, 2 * Tl::BYTES);
+#pragma unroll
+    for (int ch = 0; ch < Tl::CHUNKS; ++ch) {
+      tma_load_4d(sbase + L::K_OFF + ch * Tl::CHUNK_BYTES, &tmK, ch * Tl::BOX_COLS, h,
+                  c * kDecChunk, b, bar);
+      tma_load_4d(sbase + L::V_OFF + ch * Tl::CHUNK_BYTES, &tmV, ch * Tl::BOX_COLS, h,
+                  c * kDecChunk, b, bar);
+    }
+  }
+  // the new tokens' queries, times scale * log2(e), while the rows arrive
+  for (int i = tid; i < p.Tq * D; i += kDecThreads) {
+    const int t = i / D, col = i % D;
+    qs[i] = __bfloat162float(p.q[(((size_t)b * p.Tq + t) * p.H + h) * D + col]) * p.scale_log2;
+  }
+  const Guard g{abort_flag, p.wait_limit_ns};
+  const bool ok = wait_bounded(bar, 0, g, 1);
+  __syncthreads();  // qs complete; the outcome of the wait is uniform after this point
+  if (!ok || *abort_flag) {
+    if (tid == 0) drain_wait(bar, 0, p.wait_limit_ns);
+    return;
+  }
+
+  const int j = c * kDecChunk + tid;  // the key row this thread scores
+  const int col = tid % D, grp = tid / D;
+  constexpr int KPG = kDecChunk / L::G;  // keys per group in the V pass
+  for (int t = 0; t < p.Tq; ++t) {
+    const int last = p.L - p.Tq + t;  // query t sees keys 0 .. last
+    float s = -INFINITY;
+    if (j <= last) {
+      const float* qt = qs + t * D;
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int u = 0; u < D / 8; ++u) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(sK + tile_elem_offset<D>(tid, 8 * u));
+        const float4 q0 = *reinterpret_cast<const float4*>(qt + 8 * u);
+        const float4 q1 = *reinterpret_cast<const float4*>(qt + 8 * u + 4);
+        a0 = fmaf(bf16_lo(kv.x), q0.x, a0);
+        a1 = fmaf(bf16_hi(kv.x), q0.y, a1);
+        a0 = fmaf(bf16_lo(kv.y), q0.z, a0);
+        a1 = fmaf(bf16_hi(kv.y), q0.w, a1);
+        a0 = fmaf(bf16_lo(kv.z), q1.x, a0);
+        a1 = fmaf(bf16_hi(kv.z), q1.y, a1);
+        a0 = fmaf(bf16_lo(kv.w), q1.z, a0);
+        a1 = fmaf(bf16_hi(kv.w), q1.w, a1);
+      }
+      s = a0 + a1;
+    }
+    const float m = dec_block_reduce(s, true, red);
+    const float w = (s == -INFINITY) ? 0.f : ex2(s - m);
+    const float l = dec_block_reduce(w, false, red + 4);
+    ps[tid] = w;
+    __syncthreads();
+    // this thread's column of V, over its group's keys
+    float acc = 0.f;
+#pragma unroll 8
+    for (int k = grp * KPG; k < (grp + 1) * KPG; ++k) {
+      const uint16_t bits = *reinterpret_cast<const uint16_t*>(sV + tile_elem_offset<D>(k, col));
+      acc = fmaf(ps[k], __uint_as_float((uint32_t)bits << 16), acc);
+    }
+    const size_t row = (((size_t)b * p.H + h) * p.Tq + t) * p.n_chunks + c;
+    if (L::G > 1) {
+      acc_s[grp * D + col] = acc;
+      __syncthreads();
+      if (grp == 0) {
+        for (int gg = 1; gg < L::G; ++gg) acc += acc_s[gg * D + col];
+      }
+    }
+    if (grp == 0) p.part_o[row * D + col] = acc;
+    if (tid == 0) {
+      p.part_ml[row * 2] = m;
+      p.part_ml[row * 2 + 1] = l;
+    }
+    __syncthreads();  // ps and acc_s are rewritten for the next token
+  }
+}
+
+// Merges the chunks of one (batch, head, token) in chunk order; one thread per column.
+template <int D>
+__global__ void __launch_bounds__(D)
+    attn_decode_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
+                               __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int H,
+                               int Tq, int n_chunks) {
+  const int idx = blockIdx.x;  // ((b * H) + h) * Tq + t
+  const int t = idx % Tq, bh = idx / Tq, h = bh % H, b = bh / H;
+  const int col = threadIdx.x;
+  const float* ml = part_ml + (size_t)idx * n_chunks * 2;
+  const float* po = part_o + (size_t)idx * n_chunks * D;
+  float M = -INFINITY;
+  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, ml[2 * c]);
+  float l = 0.f, acc = 0.f;
+  for (int c = 0; c < n_chunks; ++c) {
+    const float mc = ml[2 * c];
+    if (mc == -INFINITY) continue;  // a chunk that holds no visible key
+    const float f = ex2(mc - M);
+    l = fmaf(ml[2 * c + 1], f, l);
+    acc = fmaf(po[(size_t)c * D + col], f, acc);
+  }
+  o[(((size_t)b * Tq + t) * H + h) * D + col] = __float2bfloat16_rn(acc / l);
+  if (col == 0) lse[idx] = (M + lg2(l)) * kLn2;
+}
+
+}  // namespace ca

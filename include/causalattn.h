@@ -59,6 +59,7 @@
 #ifndef CAUSALATTN_H
 #define CAUSALATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -118,6 +119,31 @@ int gpt_attn_bwd_window(const void* q, const void* k, const void* v, const void*
                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
                         float* delta_ws, int B, int H, int T, int d, float scale,
                         const int32_t* doc_offsets, int window, void* stream);
+
+/*
+ * KV-cache decode.  Generation appends Tq new tokens to a cache of L keys and
+ * values (the pages' inference engine keeps a KV cache and attends from the
+ * new tokens with FlashAttention-3's kv-cache call on (B, T, H, D) tensors:
+ * "How to build an LLM by hand", agmtopy.github.io, section 2).  New token t
+ * (0 <= t < Tq) sits at position L - Tq + t and attends to cache positions
+ * 0 .. L - Tq + t: the causal rule above, for the last Tq rows.
+ *   q:          bf16 [B, Tq, H, d]   (the new tokens' queries)
+ *   k_cache,
+ *   v_cache:    bf16 [B, L, H, d]    (positions 0 .. L-1, the new tokens' last)
+ *   o:          bf16 [B, Tq, H, d];  lse: fp32 [B, H, Tq] (natural log)
+ *   workspace:  caller-owned device memory of at least
+ *               gpt_attn_decode_workspace_size(B, H, Tq, L, d) bytes, 16-byte
+ *               aligned; its contents on entry do not matter.
+ * Limits: 1 <= Tq <= 16, Tq <= L, B and H <= 65535, B*L*H*d < 2^31.  Fails
+ * with GPT_ATTN_ERR_BAD_SHAPE for a too-small workspace.  Layout, ownership,
+ * asynchrony and error rules as above.  Split over 128-key chunks of the cache
+ * and merged in chunk order: the result is deterministic.
+ */
+size_t gpt_attn_decode_workspace_size(int B, int H, int Tq, int L, int d);
+
+int gpt_attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                    void* workspace, size_t workspace_bytes, int B, int H, int Tq, int L, int d,
+                    float scale, void* stream);
 
 /* Backward step 1: delta[b,h,i] = sum_c dout[b,h,i,c] * o[b,h,i,c] (fp32). */
 int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B, int H, int T,

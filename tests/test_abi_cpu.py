@@ -114,6 +114,29 @@ def test_window_entry_points_validate_like_the_plain_ones(lib):
             assert bw(window=w) == abi.GPT_ATTN_ERR_NO_DEVICE
 
 
+def test_decode_validation(lib):
+    ws = lib.gpt_attn_decode_workspace_size
+    assert ws(2, 4, 1, 1000, 128) == 2 * 4 * 1 * 8 * (2 + 128) * 4   # 8 chunks of 128 keys
+    assert ws(1, 1, 16, 16, 32) > 0
+    for bad in ((0, 4, 1, 100, 64), (1, 0, 1, 100, 64), (1, 1, 0, 100, 64), (1, 1, 17, 100, 64),
+                (1, 1, 5, 4, 64), (1, 1, 1, 100, 48)):
+        assert ws(*bad) == 0
+
+    def dec(q=P[0], B=1, H=2, Tq=1, L=300, d=64, wsb=1 << 20, scale=0.125):
+        return lib.gpt_attn_decode(q, P[1], P[2], P[3], P[4], P[5], wsb, B, H, Tq, L, d, scale,
+                                   None)
+    assert dec(q=None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert dec(Tq=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    assert dec(Tq=17, L=300) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    assert dec(Tq=5, L=4) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    assert dec(d=96) == abi.GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM
+    assert dec(scale=0.0) == abi.GPT_ATTN_ERR_BAD_SCALE
+    assert dec(q=P[0] + 8) == abi.GPT_ATTN_ERR_MISALIGNED
+    assert dec(wsb=16) == abi.GPT_ATTN_ERR_BAD_SHAPE        # workspace too small
+    if not torch.cuda.is_available():
+        assert dec() == abi.GPT_ATTN_ERR_NO_DEVICE
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_valid_arguments_without_a_gpu_report_no_device(lib):
     assert fwd(lib) == abi.GPT_ATTN_ERR_NO_DEVICE

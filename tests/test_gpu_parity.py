@@ -194,6 +194,58 @@ def test_window_full_size_workload(cuda_device):
     no_device_timeouts()
 
 
+# ------------------------------------------------------------ KV-cache decode
+
+def run_decode(q, kc, vc, scale):
+    dev = torch.device("cuda:0")
+    o, lse = abi.attention_decode(*(t.to(dev).contiguous() for t in (q, kc, vc)), scale)
+    torch.cuda.synchronize()
+    return o.cpu(), lse.cpu()
+
+
+def decode_inputs(B, H, Tq, L, d, seed):
+    g = torch.Generator().manual_seed(seed)
+    mk = lambda *shape: torch.randn(*shape, generator=g).to(torch.bfloat16)
+    return mk(B, Tq, H, d), mk(B, L, H, d), mk(B, L, H, d)
+
+
+@pytest.mark.parametrize("B,H,Tq,L,d", [
+    (1, 1, 1, 1, 32), (2, 3, 1, 17, 64), (1, 4, 1, 128, 128), (2, 2, 1, 129, 128),
+    (3, 2, 4, 300, 64), (1, 8, 16, 1000, 128), (2, 4, 3, 4096, 128), (1, 2, 16, 16, 32),
+    (4, 16, 1, 2048, 128),
+])
+def test_decode_parity(B, H, Tq, L, d, cuda_device):
+    """gpt_attn_decode against the fp64 decode oracle: O max-abs <= 1e-2, LSE <= 1e-3."""
+    q, kc, vc = decode_inputs(B, H, Tq, L, d, 900 + L + Tq)
+    scale = inputs.fp32_scale(d)
+    o, lse = run_decode(q, kc, vc, scale)
+    o_r, lse_r = oracle.decode_forward(q, kc, vc, scale)
+    err_o = float(np.max(np.abs(o.double().numpy() - o_r)))
+    err_l = float(np.max(np.abs(lse.double().numpy() - lse_r)))
+    print(f"decode B{B} H{H} Tq{Tq} L{L} d{d}: O {err_o:.3e} LSE {err_l:.3e}")
+    assert err_o <= O_TOL and err_l <= LSE_TOL
+    no_device_timeouts()
+
+
+def test_decode_matches_training_forward_rows(cuda_device):
+    """The decode of the last Tq tokens agrees with the training forward's last Tq rows."""
+    B, H, T, d, Tq = 2, 4, 400, 128, 5
+    q, k, v, _ = inputs.make_qkvdo(B, H, T, d, 17)
+    scale = inputs.fp32_scale(d)
+    o_full, lse_full = run_gpu(q, k, v, torch.zeros_like(q), None, scale)[:2]
+    qd = q[:, :, T - Tq:].transpose(1, 2).contiguous()
+    o, lse = run_decode(qd, k.transpose(1, 2).contiguous(), v.transpose(1, 2).contiguous(), scale)
+    assert (o.transpose(1, 2).float() - o_full[:, :, T - Tq:].float()).abs().max() <= 1e-2
+    assert (lse - lse_full[:, :, T - Tq:]).abs().max() <= 1e-3
+
+
+def test_decode_deterministic(cuda_device):
+    q, kc, vc = decode_inputs(2, 8, 2, 3000, 128, 5)
+    a = run_decode(q, kc, vc, 0.088)
+    b = run_decode(q, kc, vc, 0.088)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
 def test_host_stream_matches_device_path(cuda_device):
     """HostStream (pinned host buffers, neighbouring steps overlapped on three streams,
     two device buffer sets) gives, for every step of a sequence of different inputs,
