@@ -36,6 +36,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "causal attention fwd+bwd TFLOP/s (bf16) and % of B200 dense peak, 1 GPU"
+DECODE_METRIC = "KV-cache decode attention: GB/s of K/V cache read (bf16), 1 GPU"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.md")
 
 
@@ -233,11 +234,151 @@ def workload_config(w, parallelism):
             "l2": "not flushed: inputs Q,K,V,dO (+O) exceed the 126 MB L2"}
 
 
+def decode_config(c, parallelism):
+    return {"workload": f"decode: B={c['B']} H={c['H']} Tq={c['Tq']} L={c['L']} d={c['d']}, "
+                        "KV cache (B, L, H, d)",
+            "B": c["B"], "H": c["H"], "Tq": c["Tq"], "cache_len": c["L"], "d": c["d"],
+            "parallelism": parallelism,
+            "l2": "not flushed: the K/V cache (268 MB at decode_8k) exceeds the 126 MB L2"}
+
+
+def decode_oracle_sample(c, data, n_heads):
+    """The numpy decode oracle on the first n_heads heads of batch 0: (seconds, cache bytes)."""
+    import oracle
+    q, kc, vc = data
+    t0 = time.perf_counter()
+    oracle.decode_forward(q[:1, :, :n_heads], kc[:1, :, :n_heads], vc[:1, :, :n_heads],
+                          c["d"] ** -0.5)
+    return time.perf_counter() - t0, 2.0 * c["L"] * n_heads * c["d"] * 2
+
+
+def main_decode(args):
+    """KV-cache decode: one step = gpt_attn_decode for Tq new tokens over the whole cache."""
+    import torch
+    from causal_self_attention_mha_b200 import inputs
+    c = inputs.DECODE_WORKLOADS[args.workload]
+    B, H, Tq, L, d = c["B"], c["H"], c["Tq"], c["L"], c["d"]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    data = inputs.make_decode(B, H, Tq, L, d, c["seed"])
+    cores = len(os.sched_getaffinity(0))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        n_heads = H
+        for _ in range(args.warmup):
+            decode_oracle_sample(c, data, n_heads)
+        times, byts = [], 0.0
+        for _ in range(args.steps):
+            dt, byts = decode_oracle_sample(c, data, n_heads)
+            times.append(dt)
+        value = byts * len(times) / sum(times) / 1e9
+        print(json.dumps({
+            "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic: seeded N(0,1) bf16 q and K/V cache",
+            "config": decode_config(c, "single host process (numpy)"),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"batch 0, all {H} heads per step; CPU {cpu_model()}"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    import torch.distributed as dist
+    from causal_self_attention_mha_b200 import abi
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    q, kc, vc = (t.to(dev) for t in data)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, Tq, device=dev, dtype=torch.float32)
+    ws = torch.empty(abi.gpt_attn_decode_workspace_size(B, H, Tq, L, d), device=dev,
+                     dtype=torch.uint8)
+    scale = d ** -0.5
+    stream = torch.cuda.Stream(device=dev)
+    cache_bytes = 2.0 * B * L * H * d * 2
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            abi.gpt_attn_decode(q, kc, vc, o, lse, ws, scale, stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    sampler = ClockSampler(local)
+    t_wall0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        abi.gpt_attn_decode(q, kc, vc, o, lse, ws, scale, stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
+    status = abi.gpt_attn_device_status(clear=True)
+    # end to end: the new tokens' queries from pinned host memory in, O and LSE back out;
+    # the cache stays resident on the device, as in generation
+    qh = data[0].pin_memory()
+    oh = torch.empty(B, Tq, H, d, dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty(B, H, Tq, dtype=torch.float32).pin_memory()
+    def host_step():
+        with torch.cuda.stream(stream):
+            q.copy_(qh, non_blocking=True)
+            abi.gpt_attn_decode(q, kc, vc, o, lse, ws, scale, stream)
+            oh.copy_(o, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+    for _ in range(3):
+        host_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        host_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
+    if rank == 0:
+        pk = peaks()
+        value = world * cache_bytes / (ms * 1e-3) / 1e9
+        achieved = cache_bytes / (ms * 1e-3) / 1e9
+        line = {
+            "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) bf16 q and K/V cache",
+            "config": decode_config(c, f"replicas x{world}" if world > 1 else "single GPU"),
+            "roofline": {"kernel": "attn_decode (chunk + combine)", "bound": "hbm",
+                         "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm"], "peak_source": pk["source"],
+                         "traffic": None},
+            "e2e": {"value": world * cache_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": qh.numel() * 2,
+                    "d2h_bytes_per_step": oh.numel() * 2 + lh.numel() * 4, "ms_per_step": e2e_ms},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+            "device_status": status,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            dt, byts = decode_oracle_sample(c, data, H)
+            line["cpu_baseline"] = {"value": byts / dt / 1e9, "unit": "GB/s", "cores": 1,
+                                    "kind": "oracle", "seconds": dt,
+                                    "sample": f"batch 0 of {B}, all {H} heads; CPU {cpu_model()}"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     import torch
     from causal_self_attention_mha_b200 import inputs
 
+    if args.workload in inputs.DECODE_WORKLOADS:
+        main_decode(args)
+        return
     w = inputs.WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

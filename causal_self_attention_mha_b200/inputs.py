@@ -71,6 +71,23 @@ def make_qkvdo(B: int, H: int, T: int, d: int, seed: int):
     return tuple(out)
 
 
+def make_decode(B: int, H: int, Tq: int, L: int, d: int, seed: int):
+    """KV-cache decode inputs as CPU bf16 tensors: q [B,Tq,H,d], then the K and V caches
+    [B,L,H,d], drawn in that order from one generator."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = torch.randn(B, Tq, H, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    kc = torch.randn(B, L, H, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn(B, L, H, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    return q, kc, vc
+
+
+# KV-cache decode workloads (bench.py --workload decode_8k): one new token per step over a
+# cache of L positions, the GPT-2 / 400M head counts with a d = 128 head.
+DECODE_WORKLOADS = {
+    "decode_8k": dict(B=8, H=16, Tq=1, L=8192, d=128, seed=6),
+}
+
+
 def doc_lengths(B: int, T: int, seed: int, lo: int = DOC_MIN_LEN, hi: int = DOC_MAX_LEN) -> List[List[int]]:
     """Per-row document lengths: uniform integers in [lo, hi] until the row holds T tokens."""
     rng = random.Random(seed)
