@@ -46,8 +46,8 @@ struct DecLayout {
   static constexpr int RED_OFF = P_OFF + kDecChunk * 4;            // fp32 [2][4] warp partials
   static constexpr int G = kDecThreads / D;                        // key groups in the V pass
   static constexpr int ACC_OFF = RED_OFF + 64;                     // fp32 [G][D] group sums
-  static constexpr int BAR_OFF = ACC_OFF + G * D * 4;
-  static constexpr int MISC_OFF = BAR_OFF + 8;
+  static constexpr int BAR_OFF = ACC_OFF + G * D * 4;              // K landed, V landed
+  static constexpr int MISC_OFF = BAR_OFF + 16;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
 };
@@ -93,26 +93,29 @@ __global__ void __launch_bounds__(kDecThreads)
   float* ps = reinterpret_cast<float*>(gsm + L::P_OFF);
   float* red = reinterpret_cast<float*>(gsm + L::RED_OFF);
   float* acc_s = reinterpret_cast<float*>(gsm + L::ACC_OFF);
-  const uint32_t bar = sbase + L::BAR_OFF;
+  const uint32_t bar_k = sbase + L::BAR_OFF, bar_v = bar_k + 8u;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF);
 
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
   if (tid == 0) {
-    mbar_init(bar, 1);
+    mbar_init(bar_k, 1);
+    mbar_init(bar_v, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
   if (tid == 0) {  // this chunk's 128 key and value rows of head h (rows past L read as zero)
-    mbar_arrive_expect_tx(bar, 2 * Tl::BYTES);
+    mbar_arrive_expect_tx(bar_k, Tl::BYTES);
+    mbar_arrive_expect_tx(bar_v, Tl::BYTES);
 #pragma unroll
-    for (int ch = 0; ch < Tl::CHUNKS; ++ch) {
+    for (int ch = 0; ch < Tl::CHUNKS; ++ch)
       tma_load_4d(sbase + L::K_OFF + ch * Tl::CHUNK_BYTES, &tmK, ch * Tl::BOX_COLS, h,
-                  c * kDecChunk, b, bar);
+                  c * kDecChunk, b, bar_k);
+#pragma unroll
+    for (int ch = 0; ch < Tl::CHUNKS; ++ch)
       tma_load_4d(sbase + L::V_OFF + ch * Tl::CHUNK_BYTES, &tmV, ch * Tl::BOX_COLS, h,
-                  c * kDecChunk, b, bar);
-    }
+                  c * kDecChunk, b, bar_v);
   }
   // the new tokens' queries, times scale * log2(e), while the rows arrive
   for (int i = tid; i < p.Tq * D; i += kDecThreads) {
@@ -120,12 +123,17 @@ __global__ void __launch_bounds__(kDecThreads)
     qs[i] = __bfloat162float(p.q[(((size_t)b * p.Tq + t) * p.H + h) * D + col]) * p.scale_log2;
   }
   const Guard g{abort_flag, p.wait_limit_ns};
-  const bool ok = wait_bounded(bar, 0, g, 1);
+  // the scores need only K: V keeps landing while they are computed
+  const bool ok = wait_bounded(bar_k, 0, g, 1);
   __syncthreads();  // qs complete; the outcome of the wait is uniform after this point
   if (!ok || *abort_flag) {
-    if (tid == 0) drain_wait(bar, 0, p.wait_limit_ns);
+    if (tid == 0) {
+      drain_wait(bar_k, 0, p.wait_limit_ns);
+      drain_wait(bar_v, 0, p.wait_limit_ns);
+    }
     return;
   }
+  bool v_ready = false;
 
   const int j = c * kDecChunk + tid;  // the key row this thread scores
   const int col = tid % D, grp = tid / D;
@@ -156,6 +164,15 @@ __global__ void __launch_bounds__(kDecThreads)
     const float w = (s == -INFINITY) ? 0.f : ex2(s - m);
     const float l = dec_block_reduce(w, false, red + 4);
     ps[tid] = w;
+    if (!v_ready) {  // first token only: V must have landed before the weighted sums
+      const bool vok = wait_bounded(bar_v, 0, g, 2);
+      v_ready = true;
+      __syncthreads();
+      if (!vok || *abort_flag) {
+        if (tid == 0) drain_wait(bar_v, 0, p.wait_limit_ns);
+        return;
+      }
+    }
     __syncthreads();
     // this thread's column of V, over its group's keys
     float acc = 0.f;
