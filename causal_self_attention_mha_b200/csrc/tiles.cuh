@@ -56,14 +56,6 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m, in
     tma_load_3d(dst + c * Tile<D>::CHUNK_BYTES, m, c * Tile<D>::BOX_COLS, row0, bh, bar);
 }
 
-// L2 prefetch of the same tile (rows past T are skipped by the hardware).
-template <int D>
-__device__ __forceinline__ void prefetch_tile(const CUtensorMap* m, int row0, int bh) {
-#pragma unroll
-  for (int c = 0; c < Tile<D>::CHUNKS; ++c)
-    tma_prefetch_l2_3d(m, c * Tile<D>::BOX_COLS, row0, bh);
-}
-
 // Writes packed bf16 pairs w (columns col0 .. col0 + 2*NW - 1 of tile row r)
 // into a staged tile with the layout load_tile produces (16-byte units XORed
 // with the row inside each swizzle atom), ready for store_tile.  A warp writing
@@ -137,18 +129,6 @@ __device__ __forceinline__ uint32_t aligned_smem_base(const void* raw, uint8_t**
   const uint32_t b = (a + 1023u) & ~1023u;
   *generic = (uint8_t*)raw + (b - a);
   return b;
-}
-
-// Store 32 fp32 values (one TMEM chunk of a row), times `mul`, as 32 bf16 to global.
-__device__ __forceinline__ void store_row_chunk_bf16(__nv_bfloat16* dst, const uint32_t (&r)[32],
-                                                     float mul) {
-  uint32_t pk[16];
-#pragma unroll
-  for (int e = 0; e < 16; ++e)
-    pk[e] = pack_bf16(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int v = 0; v < 4; ++v) d4[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
 }
 
 }  // namespace ca
