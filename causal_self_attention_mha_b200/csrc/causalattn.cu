@@ -52,8 +52,14 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(ca::attn_bwd_dkdv_kernel<D>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DkdvLayout<D>::SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D>::SMEM);
+  e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D, 1>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D, 1>::SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D, 4>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D, 4>::SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D, 16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D, 16>::SMEM);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(ca::attn_bwd_dq_kernel<D>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DqLayout<D>::SMEM);
@@ -280,7 +286,16 @@ int decode_impl(const void* q, const void* kc, const void* vc, void* o, float* l
   p.scale_log2 = scale * ca::kLog2e;
   p.wait_limit_ns = kWaitLimitNs;
   dim3 grid((unsigned)p.n_chunks, (unsigned)H, (unsigned)B);
-  ca::attn_decode_chunk_kernel<D><<<grid, ca::kDecThreads, ca::DecLayout<D>::SMEM, st>>>(mk, mv, p);
+  // the smallest token capacity that holds Tq (registers and shared memory scale with it)
+  if (Tq <= 1)
+    ca::attn_decode_chunk_kernel<D, 1><<<grid, ca::kDecThreads, ca::DecLayout<D, 1>::SMEM, st>>>(
+        mk, mv, p);
+  else if (Tq <= 4)
+    ca::attn_decode_chunk_kernel<D, 4><<<grid, ca::kDecThreads, ca::DecLayout<D, 4>::SMEM, st>>>(
+        mk, mv, p);
+  else
+    ca::attn_decode_chunk_kernel<D, 16><<<grid, ca::kDecThreads, ca::DecLayout<D, 16>::SMEM, st>>>(
+        mk, mv, p);
   int s = launch_status();
   if (s) return s;
   ca::attn_decode_combine_kernel<D><<<(unsigned)(B * H * Tq), D, 0, st>>>(

@@ -37,16 +37,16 @@ struct DecParams {
   uint64_t wait_limit_ns;
 };
 
-template <int D>
+template <int D, int TQM>
 struct DecLayout {
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = Tile<D>::BYTES;
-  static constexpr int Q_OFF = 2 * Tile<D>::BYTES;                 // fp32 [Tq][D], times scale*log2e
-  static constexpr int P_OFF = Q_OFF + kDecMaxTq * D * 4;          // fp32 [128] weights
-  static constexpr int RED_OFF = P_OFF + kDecChunk * 4;            // fp32 [2][4] warp partials
+  static constexpr int Q_OFF = 2 * Tile<D>::BYTES;                 // fp32 [TQM][D], times scale*log2e
+  static constexpr int P_OFF = Q_OFF + TQM * D * 4;                // fp32 [TQM][128] weights
+  static constexpr int RED_OFF = P_OFF + TQM * kDecChunk * 4;      // fp32 [2][TQM][4] warp partials
   static constexpr int G = kDecThreads / D;                        // key groups in the V pass
-  static constexpr int ACC_OFF = RED_OFF + 64;                     // fp32 [G][D] group sums
-  static constexpr int BAR_OFF = ACC_OFF + G * D * 4;              // K landed, V landed
+  static constexpr int ACC_OFF = RED_OFF + 2 * TQM * 4 * 4;        // fp32 [G][TQM][D] group sums
+  static constexpr int BAR_OFF = ACC_OFF + (G > 1 ? G * TQM * D * 4 : 0);  // K landed, V landed
   static constexpr int MISC_OFF = BAR_OFF + 16;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
@@ -61,29 +61,37 @@ __device__ __forceinline__ uint32_t tile_elem_offset(int r, int col) {
   return (uint32_t)(ch * Tl::CHUNK_BYTES + r * Tl::SW + phys * 16 + (col % 8) * 2);
 }
 
-// Block-wide reduction of one float per thread (max or sum) over the 4 warps.
-__device__ __forceinline__ float dec_block_reduce(float v, bool is_max, float* red) {
+// Block-wide max or sum of v[t] (t < TQM) over the 4 warps; every thread gets the results.
+template <int TQM>
+__device__ __forceinline__ void dec_block_reduce(float (&v)[TQM], bool is_max, float* red) {
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float o = __shfl_xor_sync(0xffffffffu, v, off);
-    v = is_max ? fmaxf(v, o) : v + o;
-  }
+  for (int t = 0; t < TQM; ++t)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[t], off);
+      v[t] = is_max ? fmaxf(v[t], o) : v[t] + o;
+    }
   const int warp = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) red[warp] = v;
-  __syncthreads();
-  float r = red[0];
+  if ((threadIdx.x & 31) == 0) {
 #pragma unroll
-  for (int w = 1; w < kDecThreads / 32; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
-  __syncthreads();  // red may be reused by the next reduction
-  return r;
+    for (int t = 0; t < TQM; ++t) red[t * 4 + warp] = v[t];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int t = 0; t < TQM; ++t) {
+    const float4 r = *reinterpret_cast<const float4*>(red + t * 4);
+    v[t] = is_max ? fmaxf(fmaxf(r.x, r.y), fmaxf(r.z, r.w)) : (r.x + r.y) + (r.z + r.w);
+  }
 }
 
-template <int D>
+// One CTA: one 128-key chunk of one (batch, head), every new token at once: each key row
+// and each V element is read from shared memory once for all Tq tokens.
+template <int D, int TQM>
 __global__ void __launch_bounds__(kDecThreads)
     attn_decode_chunk_kernel(const __grid_constant__ CUtensorMap tmK,
                              const __grid_constant__ CUtensorMap tmV, const DecParams p) {
   using Tl = Tile<D>;
-  using L = DecLayout<D>;
+  using L = DecLayout<D, TQM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* gsm;
   const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
@@ -98,6 +106,7 @@ __global__ void __launch_bounds__(kDecThreads)
 
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
+  const int Tq = p.Tq;
   if (tid == 0) {
     mbar_init(bar_k, 1);
     mbar_init(bar_v, 1);
@@ -117,10 +126,11 @@ __global__ void __launch_bounds__(kDecThreads)
       tma_load_4d(sbase + L::V_OFF + ch * Tl::CHUNK_BYTES, &tmV, ch * Tl::BOX_COLS, h,
                   c * kDecChunk, b, bar_v);
   }
-  // the new tokens' queries, times scale * log2(e), while the rows arrive
-  for (int i = tid; i < p.Tq * D; i += kDecThreads) {
+  // the new tokens' queries, times scale * log2(e), while the rows arrive (zero past Tq)
+  for (int i = tid; i < TQM * D; i += kDecThreads) {
     const int t = i / D, col = i % D;
-    qs[i] = __bfloat162float(p.q[(((size_t)b * p.Tq + t) * p.H + h) * D + col]) * p.scale_log2;
+    qs[i] = t < Tq ? __bfloat162float(p.q[(((size_t)b * Tq + t) * p.H + h) * D + col]) * p.scale_log2
+                   : 0.f;
   }
   const Guard g{abort_flag, p.wait_limit_ns};
   // the scores need only K: V keeps landing while they are computed
@@ -133,68 +143,87 @@ __global__ void __launch_bounds__(kDecThreads)
     }
     return;
   }
-  bool v_ready = false;
 
-  const int j = c * kDecChunk + tid;  // the key row this thread scores
-  const int col = tid % D, grp = tid / D;
-  constexpr int KPG = kDecChunk / L::G;  // keys per group in the V pass
-  for (int t = 0; t < p.Tq; ++t) {
-    const int last = p.L - p.Tq + t;  // query t sees keys 0 .. last
-    float s = -INFINITY;
-    if (j <= last) {
-      const float* qt = qs + t * D;
-      float a0 = 0.f, a1 = 0.f;
+  // scores of my key row against every new token (base 2; -inf where not visible)
+  const int j = c * kDecChunk + tid;
+  float s[TQM];
 #pragma unroll
-      for (int u = 0; u < D / 8; ++u) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(sK + tile_elem_offset<D>(tid, 8 * u));
-        const float4 q0 = *reinterpret_cast<const float4*>(qt + 8 * u);
-        const float4 q1 = *reinterpret_cast<const float4*>(qt + 8 * u + 4);
-        a0 = fmaf(bf16_lo(kv.x), q0.x, a0);
-        a1 = fmaf(bf16_hi(kv.x), q0.y, a1);
-        a0 = fmaf(bf16_lo(kv.y), q0.z, a0);
-        a1 = fmaf(bf16_hi(kv.y), q0.w, a1);
-        a0 = fmaf(bf16_lo(kv.z), q1.x, a0);
-        a1 = fmaf(bf16_hi(kv.z), q1.y, a1);
-        a0 = fmaf(bf16_lo(kv.w), q1.z, a0);
-        a1 = fmaf(bf16_hi(kv.w), q1.w, a1);
-      }
-      s = a0 + a1;
+  for (int t = 0; t < TQM; ++t) s[t] = 0.f;
+#pragma unroll
+  for (int u = 0; u < D / 8; ++u) {
+    const uint4 kv = *reinterpret_cast<const uint4*>(sK + tile_elem_offset<D>(tid, 8 * u));
+    const float k8[8] = {bf16_lo(kv.x), bf16_hi(kv.x), bf16_lo(kv.y), bf16_hi(kv.y),
+                         bf16_lo(kv.z), bf16_hi(kv.z), bf16_lo(kv.w), bf16_hi(kv.w)};
+#pragma unroll
+    for (int t = 0; t < TQM; ++t) {
+      const float4 q0 = *reinterpret_cast<const float4*>(qs + t * D + 8 * u);
+      const float4 q1 = *reinterpret_cast<const float4*>(qs + t * D + 8 * u + 4);
+      float a = s[t];
+      a = fmaf(k8[0], q0.x, a);
+      a = fmaf(k8[1], q0.y, a);
+      a = fmaf(k8[2], q0.z, a);
+      a = fmaf(k8[3], q0.w, a);
+      a = fmaf(k8[4], q1.x, a);
+      a = fmaf(k8[5], q1.y, a);
+      a = fmaf(k8[6], q1.z, a);
+      a = fmaf(k8[7], q1.w, a);
+      s[t] = a;
     }
-    const float m = dec_block_reduce(s, true, red);
-    const float w = (s == -INFINITY) ? 0.f : ex2(s - m);
-    const float l = dec_block_reduce(w, false, red + 4);
-    ps[tid] = w;
-    if (!v_ready) {  // first token only: V must have landed before the weighted sums
-      const bool vok = wait_bounded(bar_v, 0, g, 2);
-      v_ready = true;
-      __syncthreads();
-      if (!vok || *abort_flag) {
-        if (tid == 0) drain_wait(bar_v, 0, p.wait_limit_ns);
-        return;
-      }
-    }
+  }
+#pragma unroll
+  for (int t = 0; t < TQM; ++t)  // query t sees keys 0 .. L - Tq + t
+    if (t >= Tq || j > p.L - Tq + t) s[t] = -INFINITY;
+  float m[TQM], w[TQM];
+#pragma unroll
+  for (int t = 0; t < TQM; ++t) m[t] = s[t];
+  dec_block_reduce<TQM>(m, true, red);
+#pragma unroll
+  for (int t = 0; t < TQM; ++t) {
+    w[t] = (s[t] == -INFINITY) ? 0.f : ex2(s[t] - m[t]);
+    ps[t * kDecChunk + tid] = w[t];
+  }
+  dec_block_reduce<TQM>(w, false, red + TQM * 4);  // w[t] now holds the chunk's sum for token t
+  // V must have landed before the weighted sums (ps is complete after the reduction's barrier)
+  {
+    const bool vok = wait_bounded(bar_v, 0, g, 2);
     __syncthreads();
-    // this thread's column of V, over its group's keys
-    float acc = 0.f;
-#pragma unroll 8
-    for (int k = grp * KPG; k < (grp + 1) * KPG; ++k) {
-      const uint16_t bits = *reinterpret_cast<const uint16_t*>(sV + tile_elem_offset<D>(k, col));
-      acc = fmaf(ps[k], __uint_as_float((uint32_t)bits << 16), acc);
+    if (!vok || *abort_flag) {
+      if (tid == 0) drain_wait(bar_v, 0, p.wait_limit_ns);
+      return;
     }
-    const size_t row = (((size_t)b * p.H + h) * p.Tq + t) * p.n_chunks + c;
-    if (L::G > 1) {
-      acc_s[grp * D + col] = acc;
-      __syncthreads();
-      if (grp == 0) {
-        for (int gg = 1; gg < L::G; ++gg) acc += acc_s[gg * D + col];
-      }
+  }
+  // my column of V over my group's keys, for every token
+  const int col = tid % D, grp = tid / D;
+  constexpr int KPG = kDecChunk / L::G;
+  float acc[TQM];
+#pragma unroll
+  for (int t = 0; t < TQM; ++t) acc[t] = 0.f;
+#pragma unroll 4
+  for (int k = grp * KPG; k < (grp + 1) * KPG; ++k) {
+    const uint16_t bits = *reinterpret_cast<const uint16_t*>(sV + tile_elem_offset<D>(k, col));
+    const float v = __uint_as_float((uint32_t)bits << 16);
+#pragma unroll
+    for (int t = 0; t < TQM; ++t) acc[t] = fmaf(ps[t * kDecChunk + k], v, acc[t]);
+  }
+  if (L::G > 1) {
+#pragma unroll
+    for (int t = 0; t < TQM; ++t) acc_s[(grp * TQM + t) * D + col] = acc[t];
+    __syncthreads();
+    if (grp == 0) {
+      for (int gg = 1; gg < L::G; ++gg)
+#pragma unroll
+        for (int t = 0; t < TQM; ++t) acc[t] += acc_s[(gg * TQM + t) * D + col];
     }
-    if (grp == 0) p.part_o[row * D + col] = acc;
+  }
+#pragma unroll
+  for (int t = 0; t < TQM; ++t) {
+    if (t >= Tq) break;
+    const size_t row = (((size_t)b * p.H + h) * Tq + t) * p.n_chunks + c;
+    if (grp == 0) p.part_o[row * D + col] = acc[t];
     if (tid == 0) {
-      p.part_ml[row * 2] = m;
-      p.part_ml[row * 2 + 1] = l;
+      p.part_ml[row * 2] = m[t];
+      p.part_ml[row * 2 + 1] = w[t];
     }
-    __syncthreads();  // ps and acc_s are rewritten for the next token
   }
 }
 
