@@ -63,12 +63,12 @@ def peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the sources of the forward / backward kernels and their launches (the decode
-    kernels, which the recorded traffic does not cover, are left out)."""
+    """Hash of the sources of the forward / backward kernels: their code, shared-memory and
+    TMEM layouts and thread counts (the host side only launches them, one CTA per SM)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_self_attention_mha_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")) and name != "decode.cuh":
+        if name in ("fwd.cuh", "bwd.cuh", "tiles.cuh", "sm100.cuh"):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
