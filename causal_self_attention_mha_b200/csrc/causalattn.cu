@@ -298,7 +298,7 @@ int decode_impl(const void* q, const void* kc, const void* vc, void* o, float* l
         mk, mv, p);
   int s = launch_status();
   if (s) return s;
-  ca::attn_decode_combine_kernel<D><<<(unsigned)(B * H * Tq), D, 0, st>>>(
+  ca::attn_decode_combine_kernel<D><<<(unsigned)(B * H * Tq), ca::kCombWarps * 32, 0, st>>>(
       p.part_ml, p.part_o, static_cast<__nv_bfloat16*>(o), lse, H, Tq, p.n_chunks);
   return launch_status();
 }

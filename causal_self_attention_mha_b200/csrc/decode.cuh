@@ -227,29 +227,71 @@ __global__ void __launch_bounds__(kDecThreads)
   }
 }
 
-// Merges the chunks of one (batch, head, token) in chunk order; one thread per column.
+// Merges the chunks of one (batch, head, token).  kCombWarps warps each fold a fixed
+// slice of the chunks (chunk order within the slice), lane l holding columns
+// l*VEC .. l*VEC + VEC - 1; the warps' results are then folded in warp order.  The
+// order is fixed, so the result is deterministic.
+constexpr int kCombWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kCombWarps * 32)
     attn_decode_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o,
                                __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int H,
                                int Tq, int n_chunks) {
+  constexpr int VEC = D / 32;  // columns per lane
+  __shared__ float sm_m[kCombWarps], sm_l[kCombWarps];
+  __shared__ float sm_o[kCombWarps][D];
   const int idx = blockIdx.x;  // ((b * H) + h) * Tq + t
   const int t = idx % Tq, bh = idx / Tq, h = bh % H, b = bh / H;
-  const int col = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* ml = part_ml + (size_t)idx * n_chunks * 2;
   const float* po = part_o + (size_t)idx * n_chunks * D;
-  float M = -INFINITY;
-  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, ml[2 * c]);
-  float l = 0.f, acc = 0.f;
-  for (int c = 0; c < n_chunks; ++c) {
+  const int per = (n_chunks + kCombWarps - 1) / kCombWarps;
+  const int c0 = warp * per, c1 = min(n_chunks, c0 + per);
+  float M = -INFINITY, l = 0.f, acc[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
+  for (int c = c0; c < c1; ++c) {
     const float mc = ml[2 * c];
     if (mc == -INFINITY) continue;  // a chunk that holds no visible key
-    const float f = ex2(mc - M);
-    l = fmaf(ml[2 * c + 1], f, l);
-    acc = fmaf(po[(size_t)c * D + col], f, acc);
+    float x[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) x[v] = po[(size_t)c * D + lane * VEC + v];
+    const float mn = fmaxf(M, mc);
+    const float fo = ex2(M - mn), fc = ex2(mc - mn);  // ex2(-inf) = 0 for the first chunk
+    l = l * fo + ml[2 * c + 1] * fc;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = acc[v] * fo + x[v] * fc;
+    M = mn;
   }
-  o[(((size_t)b * Tq + t) * H + h) * D + col] = __float2bfloat16_rn(acc / l);
-  if (col == 0) lse[idx] = (M + lg2(l)) * kLn2;
+  if (lane == 0) {
+    sm_m[warp] = M;
+    sm_l[warp] = l;
+  }
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) sm_o[warp][lane * VEC + v] = acc[v];
+  __syncthreads();
+  if (warp == 0) {
+    float Mt = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) Mt = fmaxf(Mt, sm_m[w]);
+    float lt = 0.f, ot[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) ot[v] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) {
+      if (sm_m[w] == -INFINITY) continue;
+      const float f = ex2(sm_m[w] - Mt);
+      lt = fmaf(sm_l[w], f, lt);
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) ot[v] = fmaf(sm_o[w][lane * VEC + v], f, ot[v]);
+    }
+    const float inv = 1.0f / lt;
+    __nv_bfloat16* orow = o + (((size_t)b * Tq + t) * H + h) * D;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) orow[lane * VEC + v] = __float2bfloat16_rn(ot[v] * inv);
+    if (lane == 0) lse[idx] = (Mt + lg2(lt)) * kLn2;
+  }
 }
 
 }  // namespace ca
