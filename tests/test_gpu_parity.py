@@ -5,7 +5,7 @@ Tolerances (bf16 inputs, fp32 accumulation, bf16 outputs):
   O    max |gpu - oracle|                       <= 1e-2
   LSE  max |gpu - oracle|                       <= 1e-3
   dQ, dK, dV  ||gpu - oracle||_2 / ||oracle||_2  <= 2e-2   (per tensor; ||oracle|| floored
-              at 1e-3 RMS so that exactly-zero gradients are judged in absolute terms)
+              at 1e-3 RMS so that exactly-zero gradients are measured in absolute terms)
 The full-size workloads run in the same launch configuration the benchmark
 times; for the two T = 2048, d = 128 workloads the explicit-Jacobian oracle
 backward (O(T^3) per head) is evaluated on a spread of sampled heads (every
@@ -50,7 +50,7 @@ def oracle_heads(q, k, v, do, doc, scale, heads, with_grad=True, window=None):
 
 def rel_l2(a, b):
     """||a - b|| / ||b||, with ||b|| floored at an RMS of 1e-3 per element: where the exact
-    gradient is zero (T = 1, uniform V) the GPU's fp32 rounding residue is judged absolutely."""
+    gradient is zero (T = 1, uniform V) the GPU's fp32 rounding residue is measured absolutely."""
     floor = 1e-3 * np.sqrt(b.size)
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), floor))
 
