@@ -29,24 +29,36 @@ __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16
                                                              const __nv_bfloat16* __restrict__ dout,
                                                              float* __restrict__ delta, long rows) {
   constexpr int TPR = D / 8;  // threads per row, 8 bf16 (16 bytes) each
+  constexpr int U = 4;        // independent 16-byte loads of each tensor in flight per thread
   const long total = rows * TPR;
   const long stride = (long)gridDim.x * blockDim.x;
   const int lane = threadIdx.x & 31;
   for (long base = (long)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < total;
-       base += stride) {
-    const long e = base + lane;
-    float acc = 0.f;
-    if (e < total) {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o) + e);
-      const uint4 c = __ldg(reinterpret_cast<const uint4*>(dout) + e);
-      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
+       base += U * stride) {
+    uint4 a[U], c[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long e = base + u * stride + lane;
+      if (e < total) {
+        a[u] = __ldg(reinterpret_cast<const uint4*>(o) + e);
+        c[u] = __ldg(reinterpret_cast<const uint4*>(dout) + e);
+      } else {
+        a[u] = make_uint4(0, 0, 0, 0);
+        c[u] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long e = base + u * stride + lane;
+      const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, cv[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+      float acc = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         acc += bf16_lo(av[i]) * bf16_lo(cv[i]) + bf16_hi(av[i]) * bf16_hi(cv[i]);
-    }
 #pragma unroll
-    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (e < total && (lane % TPR) == 0) delta[e / TPR] = acc;
+      for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (e < total && (lane % TPR) == 0) delta[e / TPR] = acc;
+    }
   }
 }
 
