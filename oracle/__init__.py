@@ -175,3 +175,48 @@ def decode_forward(q, k_cache, v_cache, scale: float):
                 o[b, t, h] = (w / z) @ vc[b, :n, h, :]
                 lse[b, h, t] = m + np.log(z)
     return o, lse
+
+
+# ------------------------------------------------------- RoPE + QK-norm prologue
+# "How to build an LLM by hand" (agmtopy.github.io), section 9 (gpt.py walkthrough):
+# the attention applies RoPE and then QK Norm ("x1.2") to the queries and keys.  The page
+# gives no formulas; the readings: RoPE in the rotate-half form (element i is paired with
+# i + d/2, angle = position * base^(-2i/d), base 10000), QK Norm an RMS normalisation over
+# d without learned weights (eps 1e-6) followed by the constant gain 1.2.
+
+def _rope_angles(T: int, d: int, base: float):
+    i = np.arange(d // 2, dtype=np.float64)
+    theta = base ** (-2.0 * i / d)
+    ang = np.arange(T, dtype=np.float64)[:, None] * theta[None, :]  # [T, d/2]
+    return np.cos(ang), np.sin(ang)
+
+
+def _rope(x, cos, sin, inverse=False):
+    h = x.shape[-1] // 2
+    x1, x2 = x[..., :h], x[..., h:]
+    s = -sin if inverse else sin
+    return np.concatenate([x1 * cos + x2 * s, -x1 * s + x2 * cos], axis=-1)
+
+
+def qk_prologue_forward(x, base: float = 10000.0, gain: float = 1.2, eps: float = 1e-6):
+    """z = gain * u / sqrt(mean(u^2) + eps), u = RoPE(x) at positions 0..T-1.  x: [B,H,T,d]."""
+    x = _f64(x)
+    T, d = x.shape[2], x.shape[3]
+    cos, sin = _rope_angles(T, d, base)
+    u = _rope(x, cos, sin)
+    r = np.sqrt(np.mean(u * u, axis=-1, keepdims=True) + eps)
+    return gain * u / r
+
+
+def qk_prologue_backward(x, dz, base: float = 10000.0, gain: float = 1.2, eps: float = 1e-6):
+    """dL/dx for z = qk_prologue_forward(x): through the norm, dL/du = (gain / r) *
+    (dz - u (u . dz) / (d r^2)); through the rotation, dL/dx = RoPE^T(dL/du) (the inverse
+    rotation)."""
+    x, dz = _f64(x), _f64(dz)
+    T, d = x.shape[2], x.shape[3]
+    cos, sin = _rope_angles(T, d, base)
+    u = _rope(x, cos, sin)
+    r = np.sqrt(np.mean(u * u, axis=-1, keepdims=True) + eps)
+    s = np.sum(u * dz, axis=-1, keepdims=True)
+    du = (gain / r) * (dz - u * s / (d * r * r))
+    return _rope(du, cos, sin, inverse=True)

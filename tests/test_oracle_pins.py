@@ -454,3 +454,70 @@ def test_decode_against_torch_sdpa_fp64():
     rl = torch.logsumexp(s.masked_fill(~mask, float("-inf")), dim=-1)
     assert np.max(np.abs(o - ro.transpose(1, 2).numpy())) <= 1e-12
     assert np.max(np.abs(lse - rl.numpy())) <= 1e-12
+
+
+# ------------------------------------------------------- RoPE + QK-norm prologue
+
+def torch_prologue(x, base=10000.0, gain=1.2, eps=1e-6):
+    """An independent torch float64 statement: complex-number RoPE (pairs (i, i + d/2) as
+    real and imaginary parts, multiplied by e^{i pos theta}) and torch's rms_norm."""
+    B, H, T, d = x.shape
+    h = d // 2
+    theta = base ** (-torch.arange(0, d, 2, dtype=torch.float64) / d)
+    ang = torch.arange(T, dtype=torch.float64)[:, None] * theta[None, :]
+    c = torch.complex(x[..., :h], x[..., h:]) * torch.exp(-1j * ang)
+    u = torch.cat([c.real, c.imag], dim=-1)
+    return gain * torch.nn.functional.rms_norm(u, (d,), eps=eps)
+
+
+def test_prologue_against_torch_fp64():
+    x = torch.tensor(rnd((2, 3, 50, 64), 800), dtype=torch.float64, requires_grad=True)
+    dz = rnd((2, 3, 50, 64), 801)
+    z = torch_prologue(x)
+    z.backward(torch.tensor(dz))
+    np.testing.assert_allclose(oracle.qk_prologue_forward(x.detach().numpy()), z.detach().numpy(),
+                               atol=1e-12)
+    np.testing.assert_allclose(oracle.qk_prologue_backward(x.detach().numpy(), dz),
+                               x.grad.numpy(), atol=1e-12)
+
+
+def test_prologue_position_zero_is_plain_rms_norm():
+    """Position 0 has angle 0: the output is gain * x / rms(x)."""
+    x = rnd((1, 2, 1, 32), 810)
+    z = oracle.qk_prologue_forward(x, gain=1.2)
+    np.testing.assert_allclose(z, 1.2 * x / np.sqrt(np.mean(x * x, -1, keepdims=True) + 1e-6),
+                               atol=1e-13)
+
+
+def test_prologue_rotation_keeps_rms_and_commutes_with_the_norm():
+    """Each output row has RMS gain * rms/sqrt(rms^2 + eps) (the rotation keeps the norm)."""
+    x = rnd((2, 2, 40, 128), 820)
+    z = oracle.qk_prologue_forward(x, gain=1.0, eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(z * z, -1)), 1.0, atol=1e-12)
+
+
+def test_prologue_scores_depend_on_relative_position_only():
+    """<RoPE(q)_m, RoPE(k)_n> is unchanged when both positions move by the same amount."""
+    d, T = 16, 30
+    q, k = rnd((1, 1, 1, d), 830), rnd((1, 1, 1, d), 831)
+    Q = np.repeat(q, T, axis=2)
+    K = np.repeat(k, T, axis=2)
+    zq = oracle.qk_prologue_forward(Q, gain=1.0, eps=0.0)[0, 0]
+    zk = oracle.qk_prologue_forward(K, gain=1.0, eps=0.0)[0, 0]
+    for m, n, s in ((5, 2, 7), (20, 11, 3), (9, 9, 15)):
+        np.testing.assert_allclose(zq[m] @ zk[n], zq[m + s] @ zk[n + s], atol=1e-12)
+
+
+def test_prologue_finite_differences():
+    x = rnd((1, 1, 6, 8), 840)
+    dz = rnd((1, 1, 6, 8), 841)
+    g = oracle.qk_prologue_backward(x, dz)
+    h = 1e-6
+    num = np.zeros_like(x)
+    for idx in np.ndindex(*x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += h
+        xm[idx] -= h
+        num[idx] = (np.sum(dz * oracle.qk_prologue_forward(xp)) -
+                    np.sum(dz * oracle.qk_prologue_forward(xm))) / (2 * h)
+    assert np.linalg.norm(num - g) / np.linalg.norm(num) <= 1e-6
