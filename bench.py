@@ -37,6 +37,8 @@ if ROOT not in sys.path:
 
 METRIC = "causal attention fwd+bwd TFLOP/s (bf16) and % of B200 dense peak, 1 GPU"
 DECODE_METRIC = "KV-cache decode attention: GB/s of K/V cache read (bf16), 1 GPU"
+PROLOGUE_METRIC = ("RoPE + QK-norm prologue fwd+bwd on Q and K: GB/s of algorithmic HBM traffic "
+                   "(bf16), 1 GPU")
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.md")
 
 
@@ -62,25 +64,32 @@ def peaks():
     return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
-    """Hash of the sources of the forward / backward kernels: their code, shared-memory and
-    TMEM layouts and thread counts (the host side only launches them, one CTA per SM)."""
+MAIN_KERNEL_FILES = ("fwd.cuh", "bwd.cuh", "tiles.cuh", "sm100.cuh")
+PROLOGUE_KERNEL_FILES = ("prologue.cuh", "sm100.cuh")
+PROFILE_TRAFFIC_PROLOGUE = os.path.join(ROOT, "profiles", "traffic_prologue.md")
+
+
+def kernel_source_hash(files=MAIN_KERNEL_FILES) -> str:
+    """Hash of the sources of a family of kernels (the attention forward / backward by
+    default): their code, shared-memory and TMEM layouts and thread counts (the host side
+    only launches them)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_self_attention_mha_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if name in ("fwd.cuh", "bwd.cuh", "tiles.cuh", "sm100.cuh"):
+        if name in files:
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, workload: str):
+def recorded_traffic(kernel: str, workload: str, path: str = PROFILE_TRAFFIC,
+                     files=MAIN_KERNEL_FILES):
     """DRAM bytes per launch from the committed ncu summary, if it matches the current source."""
-    if not os.path.exists(PROFILE_TRAFFIC):
+    if not os.path.exists(path):
         return None
-    text = open(PROFILE_TRAFFIC).read()
+    text = open(path).read()
     m = re.search(r"source_hash:\s*(\w+)", text)
-    if not m or m.group(1) != kernel_source_hash():
+    if not m or m.group(1) != kernel_source_hash(files):
         return None
     m = re.search(rf"^\|\s*{re.escape(kernel)}\s*\|\s*{re.escape(workload)}\s*\|\s*([0-9.eE+]+)\s*\|",
                   text, re.M)
@@ -373,6 +382,160 @@ def main_decode(args):
         dist.destroy_process_group()
 
 
+def prologue_config(c, parallelism):
+    return {"workload": f"RoPE + QK-norm prologue on Q and K: B={c['B']} H={c['H']} T={c['T']} "
+                        f"d={c['d']} (the wide_d128 attention inputs), base 10000, gain 1.2",
+            "B": c["B"], "H": c["H"], "T": c["T"], "d": c["d"], "parallelism": parallelism,
+            "l2": "not flushed: each launch touches 134-201 MB, above the 126 MB L2"}
+
+
+def prologue_oracle_sample(c, x, n_heads):
+    """The numpy oracle, forward and backward for Q and K of n_heads heads of batch 0."""
+    import oracle
+    q, k, dq_out, dk_out = (t[:1, :n_heads] for t in x)
+    t0 = time.perf_counter()
+    oracle.qk_prologue_forward(q)
+    oracle.qk_prologue_forward(k)
+    oracle.qk_prologue_backward(q, dq_out)
+    oracle.qk_prologue_backward(k, dk_out)
+    return time.perf_counter() - t0, 10.0 * n_heads * c["T"] * c["d"] * 2
+
+
+def main_prologue(args):
+    """One step = gpt_attn_rope_qknorm_fwd then gpt_attn_rope_qknorm_bwd over Q and K.
+    Algorithmic bytes: forward reads Q, K and writes Q', K' (4 tensors), backward reads Q,
+    K, dQ', dK' and writes dQ, dK (6 tensors): 10 * B*H*T*d * 2 bytes per step."""
+    import torch
+    from causal_self_attention_mha_b200 import inputs
+    c = inputs.PROLOGUE_WORKLOADS[args.workload]
+    B, H, T, d = c["B"], c["H"], c["T"], c["d"]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    x = inputs.make_prologue(B, H, T, d, c["seed"])
+    tensor_bytes = 2.0 * B * H * T * d
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        n_heads = 2
+        for _ in range(args.warmup):
+            prologue_oracle_sample(c, x, n_heads)
+        times, byts = [], 0.0
+        for _ in range(args.steps):
+            dt, byts = prologue_oracle_sample(c, x, n_heads)
+            times.append(dt)
+        value = byts * len(times) / sum(times) / 1e9
+        print(json.dumps({
+            "impl": "reference", "metric": PROLOGUE_METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic: seeded N(0,1) bf16 Q, K, dQ', dK'",
+            "config": prologue_config(c, "single host process (numpy)"),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{n_heads} of {B * H} heads per step; CPU {cpu_model()}"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    import torch.distributed as dist
+    from causal_self_attention_mha_b200 import abi
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    q, k, dqo, dko = (t.to(dev) for t in x)
+    qn, kn, dq, dk = (torch.empty_like(q) for _ in range(4))
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        abi.gpt_attn_rope_qknorm_fwd(q, k, qn, kn, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        abi.gpt_attn_rope_qknorm_bwd(q, k, dqo, dko, dq, dk, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    time.sleep(0.5)
+    t_wall0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(events[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in events) / args.steps
+    status = abi.gpt_attn_device_status(clear=True)
+    # end to end: Q, K, dQ', dK' in from pinned host memory, Q', K', dQ, dK back out
+    hin = [t.pin_memory() for t in x]
+    hout = [torch.empty(B, H, T, d, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+
+    def host_step():
+        with torch.cuda.stream(stream):
+            for dst, src in zip((q, k, dqo, dko), hin):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in zip(hout, (qn, kn, dq, dk)):
+                dst.copy_(src, non_blocking=True)
+    for _ in range(3):
+        host_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        host_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
+    if rank == 0:
+        pk = peaks()
+        step_bytes = 10.0 * tensor_bytes
+        bwd_bytes = 6.0 * tensor_bytes
+        achieved = bwd_bytes / (bwd_ms * 1e-3) / 1e9
+        line = {
+            "metric": PROLOGUE_METRIC, "value": world * step_bytes / (ms * 1e-3) / 1e9,
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic: seeded N(0,1) bf16 Q, K, dQ', dK'",
+            "config": prologue_config(c, f"replicas x{world}" if world > 1 else "single GPU"),
+            "kernel_ms": {"rope_qknorm_fwd": fwd_ms, "rope_qknorm_bwd": bwd_ms},
+            "fwd_gbs": 4.0 * tensor_bytes / (fwd_ms * 1e-3) / 1e9,
+            "roofline": {"kernel": "rope_qknorm_bwd", "bound": "hbm", "achieved": achieved,
+                         "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
+                         "peak_source": pk["source"],
+                         "traffic": recorded_traffic("rope_qknorm_bwd", args.workload,
+                                                       PROFILE_TRAFFIC_PROLOGUE,
+                                                       PROLOGUE_KERNEL_FILES)},
+            "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": int(4 * tensor_bytes),
+                    "d2h_bytes_per_step": int(4 * tensor_bytes), "ms_per_step": e2e_ms},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+            "device_status": status,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            dt, byts = prologue_oracle_sample(c, x, 8)
+            line["cpu_baseline"] = {"value": byts / dt / 1e9, "unit": "GB/s", "cores": 1,
+                                    "kind": "oracle", "seconds": dt,
+                                    "sample": f"8 of {B * H} heads; CPU {cpu_model()}"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     import torch
@@ -380,6 +543,9 @@ def main():
 
     if args.workload in inputs.DECODE_WORKLOADS:
         main_decode(args)
+        return
+    if args.workload in inputs.PROLOGUE_WORKLOADS:
+        main_prologue(args)
         return
     w = inputs.WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -32,6 +32,7 @@ GPT_ATTN_ERR_DEVICE_TIMEOUT = 9
 GPT_ATTN_ERR_NOT_IMPLEMENTED = 10
 GPT_ATTN_ERR_BAD_SCALE = 11
 GPT_ATTN_ERR_TOO_LARGE = 12
+GPT_ATTN_ERR_BAD_PARAM = 13
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -47,6 +48,8 @@ SIGNATURES = {
     "gpt_attn_decode_workspace_size": ([_i, _i, _i, _i, _i], ctypes.c_size_t),
     "gpt_attn_decode": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _i, _f, _vp],
                         _i),
+    "gpt_attn_rope_qknorm_fwd": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _f, _f, _vp], _i),
+    "gpt_attn_rope_qknorm_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _f, _f, _vp], _i),
     "gpt_attn_bwd_preprocess": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "gpt_attn_bwd_dkdv": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_bwd_dq": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
@@ -335,6 +338,81 @@ def attention_decode(q, k_cache, v_cache, scale: Optional[float] = None, stream=
                      dtype=torch.uint8)
     gpt_attn_decode(q, k_cache, v_cache, o, lse, ws, scale, stream)
     return o, lse
+
+
+def _span(t: torch.Tensor):
+    return t.data_ptr(), t.data_ptr() + t.numel() * t.element_size()
+
+
+def _same_or_disjoint(name: str, out: torch.Tensor, allowed: torch.Tensor, others) -> None:
+    """out may be exactly `allowed` (in place) but must not otherwise overlap it or `others`."""
+    lo, hi = _span(out)
+    if _span(allowed) != (lo, hi):
+        others = (allowed, *others)
+    for t in others:
+        a, b = _span(t)
+        if a < hi and lo < b:
+            raise ValueError(f"{name} overlaps another argument")
+
+
+def gpt_attn_rope_qknorm_fwd(q, k, q_out, k_out, rope_base: float = 10000.0, gain: float = 1.2,
+                             eps: float = 1e-6, stream=None) -> None:
+    """RoPE (positions 0..T-1) then RMS norm times `gain`, on q and k [B,H,T,d] in one launch.
+    q_out may be q and k_out may be k (in place)."""
+    B, H, T, d = _bhtd("q", q)
+    _bhtd("k", k, q)
+    _bhtd("q_out", q_out, q)
+    _bhtd("k_out", k_out, q)
+    _same_or_disjoint("q_out", q_out, q, (k, k_out))
+    _same_or_disjoint("k_out", k_out, k, (q, q_out))
+    _check("gpt_attn_rope_qknorm_fwd", load().gpt_attn_rope_qknorm_fwd(
+        q.data_ptr(), k.data_ptr(), q_out.data_ptr(), k_out.data_ptr(), B, H, T, d,
+        float(rope_base), float(gain), float(eps), _stream(stream)))
+
+
+def gpt_attn_rope_qknorm_bwd(q, k, dq_out, dk_out, dq, dk, rope_base: float = 10000.0,
+                             gain: float = 1.2, eps: float = 1e-6, stream=None) -> None:
+    """Gradients with respect to the prologue's inputs q, k from those with respect to its
+    outputs.  dq may be dq_out and dk may be dk_out (in place)."""
+    B, H, T, d = _bhtd("q", q)
+    for name, t in (("k", k), ("dq_out", dq_out), ("dk_out", dk_out), ("dq", dq), ("dk", dk)):
+        _bhtd(name, t, q)
+    _same_or_disjoint("dq", dq, dq_out, (q, k, dk_out, dk))
+    _same_or_disjoint("dk", dk, dk_out, (q, k, dq_out, dq))
+    _check("gpt_attn_rope_qknorm_bwd", load().gpt_attn_rope_qknorm_bwd(
+        q.data_ptr(), k.data_ptr(), dq_out.data_ptr(), dk_out.data_ptr(), dq.data_ptr(),
+        dk.data_ptr(), B, H, T, d, float(rope_base), float(gain), float(eps), _stream(stream)))
+
+
+def rope_qknorm(q, k, rope_base: float = 10000.0, gain: float = 1.2, eps: float = 1e-6,
+                stream=None):
+    """Allocates and returns (q', k') = the prologue of q and k."""
+    q_out, k_out = torch.empty_like(q), torch.empty_like(k)
+    gpt_attn_rope_qknorm_fwd(q, k, q_out, k_out, rope_base, gain, eps, stream)
+    return q_out, k_out
+
+
+class RopeQKNormFunction(torch.autograd.Function):
+    """torch.autograd wrapper of the prologue; the backward recomputes from the saved inputs."""
+
+    @staticmethod
+    def forward(ctx, q, k, rope_base, gain, eps):
+        ctx.save_for_backward(q, k)
+        ctx.args = (rope_base, gain, eps)
+        return rope_qknorm(q, k, rope_base, gain, eps)
+
+    @staticmethod
+    def backward(ctx, dq_out, dk_out):
+        q, k = ctx.saved_tensors
+        dq_out, dk_out = dq_out.contiguous(), dk_out.contiguous()
+        dq, dk = torch.empty_like(q), torch.empty_like(k)
+        gpt_attn_rope_qknorm_bwd(q, k, dq_out, dk_out, dq, dk, *ctx.args)
+        return dq, dk, None, None, None
+
+
+def rope_qk_norm(q, k, rope_base: float = 10000.0, gain: float = 1.2, eps: float = 1e-6):
+    """Autograd form: (q', k') with gradients through the library's backward kernel."""
+    return RopeQKNormFunction.apply(q, k, rope_base, gain, eps)
 
 
 class CausalSelfAttentionFunction(torch.autograd.Function):

@@ -16,6 +16,7 @@
 #include "bwd.cuh"
 #include "decode.cuh"
 #include "fwd.cuh"
+#include "prologue.cuh"
 
 namespace {
 
@@ -340,6 +341,19 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns) {
 
 int common_checks(int B, int H, int T, int d) { return check_shape(B, H, T, d); }
 
+template <int D>
+int prologue_impl(bool bwd, const ca::ProParams& p, cudaStream_t st) {
+  const int hgs = (p.H + ca::kProHeadsPerItem - 1) / ca::kProHeadsPerItem;
+  const long threads = (long)p.B * hgs * p.T * (D / 16);
+  const long blocks = (threads + ca::kProThreads - 1) / ca::kProThreads;
+  if (bwd)
+    ca::rope_qknorm_bwd_kernel<D><<<(unsigned)blocks, ca::kProThreads, 0, st>>>(p);
+  else
+    ca::rope_qknorm_fwd_kernel<D><<<(unsigned)blocks, ca::kProThreads, 0, st>>>(p);
+  return launch_status();
+}
+
+
 }  // namespace
 
 // ======================================================================== ABI
@@ -364,6 +378,7 @@ const char* gpt_attn_strerror(int s) {
     case GPT_ATTN_ERR_NOT_IMPLEMENTED: return "not implemented";
     case GPT_ATTN_ERR_BAD_SCALE: return "scale must be finite and > 0";
     case GPT_ATTN_ERR_TOO_LARGE: return "tensor too large (B*H*T*d must be < 2^31)";
+    case GPT_ATTN_ERR_BAD_PARAM: return "rope_base must be finite and > 0, gain finite, eps finite and >= 0";
     default: return "unknown status";
   }
 }
@@ -515,6 +530,53 @@ int gpt_attn_decode(const void* q, const void* k_cache, const void* v_cache, voi
     case 64: return decode_impl<64>(q, k_cache, v_cache, o, lse, ws, B, H, Tq, L, scale, st);
     default: return decode_impl<128>(q, k_cache, v_cache, o, lse, ws, B, H, Tq, L, scale, st);
   }
+}
+
+static int prologue_entry(bool bwd, const void* x0, const void* x1, const void* g0, const void* g1,
+                          void* y0, void* y1, int B, int H, int T, int d, float rope_base,
+                          float gain, float eps, void* stream) {
+  if (!x0 || !x1 || !y0 || !y1 || (bwd && (!g0 || !g1))) return GPT_ATTN_ERR_NULL_PTR;
+  int s = common_checks(B, H, T, d);
+  if (s) return s;
+  if (!std::isfinite(rope_base) || !(rope_base > 0.f) || !std::isfinite(gain) ||
+      !std::isfinite(eps) || !(eps >= 0.f))
+    return GPT_ATTN_ERR_BAD_PARAM;
+  if (!aligned(x0, 16) || !aligned(x1, 16) || !aligned(g0, 16) || !aligned(g1, 16) ||
+      !aligned(y0, 16) || !aligned(y1, 16))
+    return GPT_ATTN_ERR_MISALIGNED;
+  if ((s = ensure_device())) return s;
+  ca::ProParams p;
+  p.x0 = static_cast<const __nv_bfloat16*>(x0);
+  p.x1 = static_cast<const __nv_bfloat16*>(x1);
+  p.g0 = static_cast<const __nv_bfloat16*>(g0);
+  p.g1 = static_cast<const __nv_bfloat16*>(g1);
+  p.y0 = static_cast<__nv_bfloat16*>(y0);
+  p.y1 = static_cast<__nv_bfloat16*>(y1);
+  p.B = B;
+  p.H = H;
+  p.T = T;
+  p.log2_base = std::log2((double)rope_base);
+  p.gain = gain;
+  p.eps = eps;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 32: return prologue_impl<32>(bwd, p, st);
+    case 64: return prologue_impl<64>(bwd, p, st);
+    default: return prologue_impl<128>(bwd, p, st);
+  }
+}
+
+int gpt_attn_rope_qknorm_fwd(const void* q, const void* k, void* q_out, void* k_out, int B, int H,
+                             int T, int d, float rope_base, float gain, float eps, void* stream) {
+  return prologue_entry(false, q, k, nullptr, nullptr, q_out, k_out, B, H, T, d, rope_base, gain,
+                        eps, stream);
+}
+
+int gpt_attn_rope_qknorm_bwd(const void* q, const void* k, const void* dq_out, const void* dk_out,
+                             void* dq, void* dk, int B, int H, int T, int d, float rope_base,
+                             float gain, float eps, void* stream) {
+  return prologue_entry(true, q, k, dq_out, dk_out, dq, dk, B, H, T, d, rope_base, gain, eps,
+                        stream);
 }
 
 int gpt_attn_check_doc_offsets(const int32_t* doc_offsets, int B, int T, void* stream) {

@@ -88,6 +88,21 @@ DECODE_WORKLOADS = {
 }
 
 
+def make_prologue(B: int, H: int, T: int, d: int, seed: int):
+    """RoPE + QK-norm inputs as CPU bf16 [B,H,T,d] tensors: q and k (projections, N(0,1)),
+    then the incoming gradients dq_out and dk_out (N(0,1)), drawn in that order."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    return tuple(torch.randn(B, H, T, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
+                 for _ in range(4))
+
+
+# RoPE + QK-norm prologue workloads (bench.py --workload prologue_wide_d128): the Q and K of
+# the wide_d128 attention workload.
+PROLOGUE_WORKLOADS = {
+    "prologue_wide_d128": dict(B=4, H=16, T=2048, d=128, seed=8),
+}
+
+
 def doc_lengths(B: int, T: int, seed: int, lo: int = DOC_MIN_LEN, hi: int = DOC_MAX_LEN) -> List[List[int]]:
     """Per-row document lengths: uniform integers in [lo, hi] until the row holds T tokens."""
     rng = random.Random(seed)

@@ -81,7 +81,8 @@ typedef enum {
   GPT_ATTN_ERR_DEVICE_TIMEOUT = 9,        /* a kernel gave up on a bounded wait */
   GPT_ATTN_ERR_NOT_IMPLEMENTED = 10,
   GPT_ATTN_ERR_BAD_SCALE = 11,            /* scale not finite or <= 0 */
-  GPT_ATTN_ERR_TOO_LARGE = 12             /* a tensor exceeds 2^31 - 1 elements */
+  GPT_ATTN_ERR_TOO_LARGE = 12,            /* a tensor exceeds 2^31 - 1 elements */
+  GPT_ATTN_ERR_BAD_PARAM = 13             /* rope_base, gain or eps out of range */
 } gpt_attn_status;
 
 /*
@@ -144,6 +145,37 @@ size_t gpt_attn_decode_workspace_size(int B, int H, int Tq, int L, int d);
 int gpt_attn_decode(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                     void* workspace, size_t workspace_bytes, int B, int H, int Tq, int L, int d,
                     float scale, void* stream);
+
+/*
+ * RoPE + QK-norm prologue.  "How to build an LLM by hand" (agmtopy.github.io),
+ * section 9 (the gpt.py walkthrough): the attention applies RoPE and then QK
+ * Norm ("x1.2") to the queries and keys; the page gives no formulas.  Reading,
+ * per row x = q[b,h,t,:] or k[b,h,t,:] (t is the row's position, 0 .. T-1):
+ *   u_p       =  x_p cos(t th_p) + x_{p+d/2} sin(t th_p)      (p < d/2)
+ *   u_{p+d/2} = -x_p sin(t th_p) + x_{p+d/2} cos(t th_p),  th_p = rope_base^(-2p/d)
+ *   out       = gain * u / sqrt(mean(u^2) + eps)
+ * (RMS norm without learned weights; the page's x1.2 is `gain`.)  Q and K are
+ * processed in one launch.
+ *   q, k:          bf16 [B,H,T,d], read
+ *   q_out, k_out:  bf16 [B,H,T,d], written; may equal q / k (in place), must not
+ *                  otherwise overlap any argument.
+ * rope_base finite and > 0, gain finite, eps finite and >= 0, else
+ * GPT_ATTN_ERR_BAD_PARAM; eps = 0 on an all-zero row gives NaN, as the formula
+ * does.  Layout, ownership, alignment, asynchrony and errors as above.
+ */
+int gpt_attn_rope_qknorm_fwd(const void* q, const void* k, void* q_out, void* k_out, int B, int H,
+                             int T, int d, float rope_base, float gain, float eps, void* stream);
+
+/*
+ * Its backward: from q, k (the prologue's INPUTS) and dq_out, dk_out (gradients
+ * of the loss with respect to q_out, k_out), writes dq, dk (gradients with
+ * respect to q, k):  du = (gain/r) (dz - u <u,dz> / (d r^2)),  dx = RoPE^T du,
+ * r = sqrt(mean(u^2) + eps).  dq may equal dq_out and dk may equal dk_out (in
+ * place); no other overlap.  Parameters and errors as for the forward.
+ */
+int gpt_attn_rope_qknorm_bwd(const void* q, const void* k, const void* dq_out, const void* dk_out,
+                             void* dq, void* dk, int B, int H, int T, int d, float rope_base,
+                             float gain, float eps, void* stream);
 
 /* Backward step 1: delta[b,h,i] = sum_c dout[b,h,i,c] * o[b,h,i,c] (fp32). */
 int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B, int H, int T,

@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_strerror(lib):
     assert lib.gpt_attn_version() == 1
-    for s in range(0, 13):
+    for s in range(0, 14):
         msg = lib.gpt_attn_strerror(s)
         assert isinstance(msg, bytes) and len(msg) > 0
     assert lib.gpt_attn_strerror(999) == b"unknown status"
@@ -135,6 +135,47 @@ def test_decode_validation(lib):
     assert dec(wsb=16) == abi.GPT_ATTN_ERR_BAD_SHAPE        # workspace too small
     if not torch.cuda.is_available():
         assert dec() == abi.GPT_ATTN_ERR_NO_DEVICE
+
+
+def test_prologue_validation(lib):
+    def fwd_(q=P[0], k=P[1], qo=P[2], ko=P[3], B=1, H=2, T=64, d=64, base=10000.0, gain=1.2,
+             eps=1e-6):
+        return lib.gpt_attn_rope_qknorm_fwd(q, k, qo, ko, B, H, T, d, base, gain, eps, None)
+
+    def bwd_(dqo=P[2], dq=P[4], **kw):
+        a = dict(q=P[0], k=P[1], dko=P[3], dk=P[5], B=1, H=2, T=64, d=64, base=10000.0,
+                 gain=1.2, eps=1e-6)
+        a.update(kw)
+        return lib.gpt_attn_rope_qknorm_bwd(a["q"], a["k"], dqo, a["dko"], dq, a["dk"], a["B"],
+                                            a["H"], a["T"], a["d"], a["base"], a["gain"],
+                                            a["eps"], None)
+    for call in (fwd_, bwd_):
+        assert call(B=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
+        assert call(T=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
+        assert call(d=48) == abi.GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM
+        assert call(B=4096, H=64, T=4096, d=128) == abi.GPT_ATTN_ERR_TOO_LARGE
+        for bad in (dict(base=0.0), dict(base=-2.0), dict(base=math.inf), dict(base=math.nan),
+                    dict(gain=math.nan), dict(gain=math.inf), dict(eps=-1e-6), dict(eps=math.nan)):
+            assert call(**bad) == abi.GPT_ATTN_ERR_BAD_PARAM, bad
+        assert call(q=P[0] + 8) == abi.GPT_ATTN_ERR_MISALIGNED
+        assert call(k=None) == abi.GPT_ATTN_ERR_NULL_PTR
+        if not torch.cuda.is_available():
+            assert call() == abi.GPT_ATTN_ERR_NO_DEVICE
+            assert call(gain=-1.2, eps=0.0) == abi.GPT_ATTN_ERR_NO_DEVICE  # both are valid
+    assert fwd_(qo=None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert bwd_(dqo=None) == abi.GPT_ATTN_ERR_NULL_PTR
+    assert bwd_(dq=P[4] + 2) == abi.GPT_ATTN_ERR_MISALIGNED
+
+
+def test_prologue_binding_overlap_rule():
+    buf = torch.zeros(4 * 1024, dtype=torch.bfloat16)
+    a, b = buf[:1024], buf[1024:2048]
+    abi._same_or_disjoint("out", a, a, (b,))                 # in place: allowed
+    abi._same_or_disjoint("out", b, a, (buf[2048:3072],))    # disjoint: allowed
+    with pytest.raises(ValueError):
+        abi._same_or_disjoint("out", buf[512:1536], a, ())   # partial overlap with its input
+    with pytest.raises(ValueError):
+        abi._same_or_disjoint("out", a, a, (buf[1000:1100],))  # overlaps another argument
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")

@@ -334,3 +334,100 @@ def test_gpu_argument_errors(cuda_device):
     with pytest.raises(abi.AttnError) as e:
         abi.gpt_attn_fwd(q, q, q, q, lse, float("nan"))
     assert e.value.status == abi.GPT_ATTN_ERR_BAD_SCALE
+
+
+# ------------------------------------------------------- RoPE + QK-norm prologue
+# bf16 in, fp32 arithmetic, bf16 out: each output element is within bf16 rounding of the
+# fp64 oracle (rtol 2^-8, half an ulp at the bottom of a binade) plus a small absolute term
+# for the fp32 arithmetic and the angle (fp64 reduction, then __sincosf on [-pi, pi]).
+PRO_RTOL, PRO_ATOL = 2.0 ** -8, 2e-3
+
+
+def run_prologue(q, k, dq_out, dk_out, base=10000.0, gain=1.2, eps=1e-6, in_place=False):
+    dev = torch.device("cuda:0")
+    q, k, dq_out, dk_out = (t.to(dev).contiguous() for t in (q, k, dq_out, dk_out))
+    if in_place:
+        qo, ko = q.clone(), k.clone()
+        abi.gpt_attn_rope_qknorm_fwd(qo, ko, qo, ko, base, gain, eps)
+        dq, dk = dq_out.clone(), dk_out.clone()
+        abi.gpt_attn_rope_qknorm_bwd(q, k, dq, dk, dq, dk, base, gain, eps)
+    else:
+        qo, ko = abi.rope_qknorm(q, k, base, gain, eps)
+        dq, dk = torch.empty_like(q), torch.empty_like(k)
+        abi.gpt_attn_rope_qknorm_bwd(q, k, dq_out, dk_out, dq, dk, base, gain, eps)
+    torch.cuda.synchronize()
+    return [t.cpu().double().numpy() for t in (qo, ko, dq, dk)]
+
+
+def check_prologue(got, q, k, dq_out, dk_out, base=10000.0, gain=1.2, eps=1e-6, label=""):
+    refs = (oracle.qk_prologue_forward(q, base, gain, eps),
+            oracle.qk_prologue_forward(k, base, gain, eps),
+            oracle.qk_prologue_backward(q, dq_out, base, gain, eps),
+            oracle.qk_prologue_backward(k, dk_out, base, gain, eps))
+    for name, g, r in zip(("q'", "k'", "dq", "dk"), got, refs):
+        err = np.abs(g - r) - PRO_RTOL * np.abs(r)
+        print(f"prologue {label} {name}: max excess {float(err.max()):.2e}")
+        assert float(err.max()) <= PRO_ATOL, (name, float(err.max()))
+
+
+@pytest.mark.parametrize("B,H,T,d", [(1, 1, 1, 32), (2, 3, 37, 32), (1, 5, 130, 64),
+                                     (2, 4, 257, 128), (1, 16, 1000, 128), (3, 7, 65, 64),
+                                     (1, 1, 40000, 64)])
+def test_prologue_parity(B, H, T, d, cuda_device):
+    """Every output element of the prologue forward and backward against the fp64 oracle;
+    H not a multiple of the 4 heads a thread handles, ragged T, and positions up to 40000
+    (the angle reduction)."""
+    x = inputs.make_prologue(B, H, T, d, 700 + T + d)
+    check_prologue(run_prologue(*x), *x, label=f"B{B} H{H} T{T} d{d}")
+    no_device_timeouts()
+
+
+@pytest.mark.parametrize("base,gain,eps", [(500000.0, 1.0, 1e-5), (10.0, -0.7, 0.0)])
+def test_prologue_parameters(base, gain, eps, cuda_device):
+    x = inputs.make_prologue(2, 3, 300, 128, 77)
+    check_prologue(run_prologue(*x, base=base, gain=gain, eps=eps), *x, base=base, gain=gain,
+                   eps=eps, label=f"base {base} gain {gain} eps {eps}")
+
+
+def test_prologue_in_place_matches_out_of_place(cuda_device):
+    x = inputs.make_prologue(2, 6, 201, 64, 78)
+    a = run_prologue(*x)
+    b = run_prologue(*x, in_place=True)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+
+
+def test_prologue_full_size_workload(cuda_device):
+    """The benchmark's prologue launch (B=4, H=16, T=2048, d=128), every element."""
+    c = inputs.PROLOGUE_WORKLOADS["prologue_wide_d128"]
+    x = inputs.make_prologue(c["B"], c["H"], c["T"], c["d"], c["seed"])
+    check_prologue(run_prologue(*x), *x, label="prologue_wide_d128")
+    no_device_timeouts()
+
+
+def test_prologue_autograd_then_attention(cuda_device):
+    """rope_qk_norm then causal_attention under torch.autograd: the gradients with respect to
+    the raw q, k, v match the oracle chain (prologue forward, attention forward and
+    backward, prologue backward) on one head."""
+    B, H, T, d = 1, 2, 150, 64
+    q, k, v, do = inputs.make_qkvdo(B, H, T, d, 79)
+    scale = inputs.fp32_scale(d)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (t.to(dev).requires_grad_() for t in (q, k, v))
+    qn, kn = abi.rope_qk_norm(qd, kd)
+    o = abi.causal_attention(qn, kn, vd, scale)
+    o.backward(do.to(dev))
+    torch.cuda.synchronize()
+    qn_r = oracle.qk_prologue_forward(q)
+    kn_r = oracle.qk_prologue_forward(k)
+    # the oracle attention takes the GPU's bf16 prologue outputs, as the kernels did
+    qn_b, kn_b = (t.detach().cpu() for t in (qn, kn))
+    for a, r in ((qn_b, qn_r), (kn_b, kn_r)):
+        assert float((np.abs(a.double().numpy() - r) - PRO_RTOL * np.abs(r)).max()) <= PRO_ATOL
+    o_r, _ = oracle.attention_forward(qn_b, kn_b, v, scale)
+    dqn, dkn, dv_r = oracle.attention_backward(qn_b, kn_b, v, do, scale)
+    dq_r = oracle.qk_prologue_backward(q, dqn)
+    dk_r = oracle.qk_prologue_backward(k, dkn)
+    assert float(np.max(np.abs(o.detach().cpu().double().numpy() - o_r))) <= O_TOL
+    for g, r in ((qd.grad, dq_r), (kd.grad, dk_r), (vd.grad, dv_r)):
+        assert rel_l2(g.cpu().double().numpy(), r) <= GRAD_TOL
