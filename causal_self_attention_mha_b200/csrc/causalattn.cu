@@ -341,18 +341,30 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns) {
 
 int common_checks(int B, int H, int T, int d) { return check_shape(B, H, T, d); }
 
+// Persistent grid: the resident blocks per SM times the SMs, or fewer when the work is small.
 template <int D>
 int prologue_impl(bool bwd, const ca::ProParams& p, cudaStream_t st) {
-  const int hgs = (p.H + ca::kProHeadsPerItem - 1) / ca::kProHeadsPerItem;
-  const long threads = (long)p.B * hgs * p.T * (D / 16);
-  const long blocks = (threads + ca::kProThreads - 1) / ca::kProThreads;
+  static std::atomic<int> resident[2] = {0, 0};
+  const void* fn = bwd ? reinterpret_cast<const void*>(ca::rope_qknorm_bwd_kernel<D>)
+                       : reinterpret_cast<const void*>(ca::rope_qknorm_fwd_kernel<D>);
+  int per_sm = resident[bwd].load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, ca::kProThreads, 0) !=
+            cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    resident[bwd].store(per_sm, std::memory_order_relaxed);
+  }
+  const int hg = bwd ? ca::kProBwdHeads : ca::kProFwdHeads;
+  const long items = (long)p.B * ((p.H + hg - 1) / hg) * p.T * (D / 16);
+  long blocks = (items + ca::kProThreads - 1) / ca::kProThreads;
+  if (blocks > (long)sm_count() * per_sm) blocks = (long)sm_count() * per_sm;
   if (bwd)
     ca::rope_qknorm_bwd_kernel<D><<<(unsigned)blocks, ca::kProThreads, 0, st>>>(p);
   else
     ca::rope_qknorm_fwd_kernel<D><<<(unsigned)blocks, ca::kProThreads, 0, st>>>(p);
   return launch_status();
 }
-
 
 }  // namespace
 

@@ -14,7 +14,7 @@
 // Q and K in the same launch.  A thread owns 8 rotation pairs of a row (two 16-byte
 // chunks, elements 8c..8c+7 and d/2+8c..d/2+8c+7), so d/16 neighbouring lanes hold a row
 // and the row sums are a shuffle over those lanes.  The angles depend on t and p only: a
-// thread computes its 8 (cos, sin) once and applies them to kProHeadsPerItem heads of Q and
+// thread computes its 8 (cos, sin) once and applies them to several heads of Q and
 // of K.  The angle t * theta_p is formed and reduced to [-pi, pi] in fp64 (so positions in
 // the tens of thousands keep full fp32 phase accuracy), then __sincosf runs on the small
 // reduced argument.  Output rows may be the input rows (in place): a row is read in full
@@ -26,7 +26,8 @@
 
 namespace ca {
 
-constexpr int kProHeadsPerItem = 4;
+constexpr int kProFwdHeads = 4;  // heads per work item (sharing one set of angles)
+constexpr int kProBwdHeads = 2;
 constexpr int kProThreads = 256;
 
 struct ProParams {
@@ -81,113 +82,133 @@ __device__ __forceinline__ float row_sum(float v) {
   return v;
 }
 
-// Work item = (b, group of kProHeadsPerItem heads, t, c); consecutive threads take
-// consecutive c, then t, so a warp reads 32 / (D/16) whole consecutive rows of a head.
-template <int D>
-__device__ __forceinline__ bool pro_item(const ProParams& p, long g, int& b, int& h0, int& t,
-                                         int& c) {
-  constexpr int TPR = D / 16;
-  const int hgs = (p.H + kProHeadsPerItem - 1) / kProHeadsPerItem;
-  const long n = (long)p.B * hgs * p.T * TPR;
-  c = (int)(g % TPR);
-  long rest = g / TPR;
-  t = (int)(rest % p.T);
-  rest /= p.T;
-  h0 = (int)(rest % hgs) * kProHeadsPerItem;
-  b = (int)(rest / hgs);
-  return g < n;
+// Work item = (b, group of HG heads, t, c); consecutive items take consecutive c, then t,
+// so a warp reads 32 / (D/16) whole consecutive rows of a head.  The grid is persistent
+// (a few blocks per SM) and each warp strides over the items 32 at a time, so the angle
+// table is built once per block and there are no waves of short-lived blocks.
+template <int D, int HG>
+struct ProItems {
+  long n;   // number of items (a multiple of D/16, so every row's lane group is whole)
+  int hgs;  // head groups
+  __device__ __forceinline__ explicit ProItems(const ProParams& p)
+      : n((long)p.B * ((p.H + HG - 1) / HG) * p.T * (D / 16)), hgs((p.H + HG - 1) / HG) {}
+  __device__ __forceinline__ void decompose(const ProParams& p, long g, int& b, int& h0, int& t,
+                                            int& c) const {
+    constexpr int TPR = D / 16;
+    c = (int)(g % TPR);
+    long rest = g / TPR;
+    t = (int)(rest % p.T);
+    rest /= p.T;
+    h0 = (int)(rest % hgs) * HG;
+    b = (int)(rest / hgs);
+  }
+};
+
+__device__ __forceinline__ long warp_first_item() {
+  return (long)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
 }
 
 template <int D>
-__global__ void __launch_bounds__(kProThreads) rope_qknorm_fwd_kernel(ProParams p) {
+__global__ void __launch_bounds__(kProThreads, 2) rope_qknorm_fwd_kernel(ProParams p) {
+  constexpr int HG = kProFwdHeads;
   __shared__ double th[D / 2];
   rope_theta_table<D>(th, p.log2_base);
-  int b, h0, t, c;
-  const bool ok = pro_item<D>(p, (long)blockIdx.x * blockDim.x + threadIdx.x, b, h0, t, c);
-  if (!ok) t = 0;  // idle lanes still join the row shuffles (their groups are whole)
-  float cs[8], sn[8];
-  rope_angles<D>(th, t, c, cs, sn);
+  const ProItems<D, HG> items(p);
+  const int lane = threadIdx.x & 31;
+  const long stride = (long)gridDim.x * blockDim.x;
   const float inv_d = 1.0f / D;
-  uint4 raw[kProHeadsPerItem][2][2];  // [head][Q,K][first half, second half]
+  // the loop bound is warp-uniform: every lane joins every row shuffle
+  for (long base = warp_first_item(); base < items.n; base += stride) {
+    const long g = base + lane;
+    const bool ok = g < items.n;
+    int b = 0, h0 = 0, t = 0, c = 0;
+    if (ok) items.decompose(p, g, b, h0, t, c);
+    uint4 raw[HG][2][2];  // [head][Q,K][first half, second half]
 #pragma unroll
-  for (int i = 0; i < kProHeadsPerItem; ++i) {
-    const bool live = ok && h0 + i < p.H;
-    const long row = (((long)b * p.H + h0 + i) * p.T + t) * D;
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      const __nv_bfloat16* x = s ? p.x1 : p.x0;
-      raw[i][s][0] = live ? *reinterpret_cast<const uint4*>(x + row + 8 * c)
-                          : make_uint4(0, 0, 0, 0);
-      raw[i][s][1] = live ? *reinterpret_cast<const uint4*>(x + row + D / 2 + 8 * c)
-                          : make_uint4(0, 0, 0, 0);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kProHeadsPerItem; ++i) {
-    const bool live = ok && h0 + i < p.H;
-    const long row = (((long)b * p.H + h0 + i) * p.T + t) * D;
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      float a[8], z[8], u1[8], u2[8];
-      unpack8(raw[i][s][0], a);
-      unpack8(raw[i][s][1], z);
-      float ss = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        u1[j] = a[j] * cs[j] + z[j] * sn[j];
-        u2[j] = z[j] * cs[j] - a[j] * sn[j];
-        ss += u1[j] * u1[j] + u2[j] * u2[j];
-      }
-      ss = row_sum<D>(ss);
-      const float k = p.gain / sqrtf(ss * inv_d + p.eps);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        u1[j] *= k;
-        u2[j] *= k;
-      }
-      if (live) {
-        __nv_bfloat16* y = s ? p.y1 : p.y0;
-        *reinterpret_cast<uint4*>(y + row + 8 * c) = pack8(u1);
-        *reinterpret_cast<uint4*>(y + row + D / 2 + 8 * c) = pack8(u2);
-      }
-    }
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(kProThreads) rope_qknorm_bwd_kernel(ProParams p) {
-  __shared__ double th[D / 2];
-  rope_theta_table<D>(th, p.log2_base);
-  int b, h0, t, c;
-  const bool ok = pro_item<D>(p, (long)blockIdx.x * blockDim.x + threadIdx.x, b, h0, t, c);
-  if (!ok) t = 0;
-  float cs[8], sn[8];
-  rope_angles<D>(th, t, c, cs, sn);
-  const float inv_d = 1.0f / D;
-  constexpr int U = 2;  // heads whose loads are in flight together
-#pragma unroll
-  for (int i0 = 0; i0 < kProHeadsPerItem; i0 += U) {
-    uint4 raw[U][2][4];  // [head][Q,K][x lo, x hi, dz lo, dz hi]
-#pragma unroll
-    for (int i = 0; i < U; ++i) {
-      const bool live = ok && h0 + i0 + i < p.H;
-      const long row = (((long)b * p.H + h0 + i0 + i) * p.T + t) * D;
+    for (int i = 0; i < HG; ++i) {
+      const bool live = ok && h0 + i < p.H;
+      const long row = (((long)b * p.H + h0 + i) * p.T + t) * D;
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
         const __nv_bfloat16* x = s ? p.x1 : p.x0;
-        const __nv_bfloat16* g = s ? p.g1 : p.g0;
+        raw[i][s][0] = live ? *reinterpret_cast<const uint4*>(x + row + 8 * c)
+                            : make_uint4(0, 0, 0, 0);
+        raw[i][s][1] = live ? *reinterpret_cast<const uint4*>(x + row + D / 2 + 8 * c)
+                            : make_uint4(0, 0, 0, 0);
+      }
+    }
+    float cs[8], sn[8];
+    rope_angles<D>(th, t, c, cs, sn);  // while the loads are in flight
+#pragma unroll
+    for (int i = 0; i < HG; ++i) {
+      const bool live = ok && h0 + i < p.H;
+      const long row = (((long)b * p.H + h0 + i) * p.T + t) * D;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        float a[8], z[8], u1[8], u2[8];
+        unpack8(raw[i][s][0], a);
+        unpack8(raw[i][s][1], z);
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          u1[j] = a[j] * cs[j] + z[j] * sn[j];
+          u2[j] = z[j] * cs[j] - a[j] * sn[j];
+          ss += u1[j] * u1[j] + u2[j] * u2[j];
+        }
+        ss = row_sum<D>(ss);
+        const float k = p.gain / sqrtf(ss * inv_d + p.eps);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          u1[j] *= k;
+          u2[j] *= k;
+        }
+        if (live) {
+          __nv_bfloat16* y = s ? p.y1 : p.y0;
+          *reinterpret_cast<uint4*>(y + row + 8 * c) = pack8(u1);
+          *reinterpret_cast<uint4*>(y + row + D / 2 + 8 * c) = pack8(u2);
+        }
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kProThreads, 2) rope_qknorm_bwd_kernel(ProParams p) {
+  constexpr int HG = kProBwdHeads;
+  __shared__ double th[D / 2];
+  rope_theta_table<D>(th, p.log2_base);
+  const ProItems<D, HG> items(p);
+  const int lane = threadIdx.x & 31;
+  const long stride = (long)gridDim.x * blockDim.x;
+  const float inv_d = 1.0f / D;
+  for (long base = warp_first_item(); base < items.n; base += stride) {
+    const long g = base + lane;
+    const bool ok = g < items.n;
+    int b = 0, h0 = 0, t = 0, c = 0;
+    if (ok) items.decompose(p, g, b, h0, t, c);
+    uint4 raw[HG][2][4];  // [head][Q,K][x lo, x hi, dz lo, dz hi]
+#pragma unroll
+    for (int i = 0; i < HG; ++i) {
+      const bool live = ok && h0 + i < p.H;
+      const long row = (((long)b * p.H + h0 + i) * p.T + t) * D;
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const __nv_bfloat16* x = s ? p.x1 : p.x0;
+        const __nv_bfloat16* gz = s ? p.g1 : p.g0;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const long e = row + hh * (D / 2) + 8 * c;
           raw[i][s][hh] = live ? *reinterpret_cast<const uint4*>(x + e) : make_uint4(0, 0, 0, 0);
-          raw[i][s][2 + hh] = live ? *reinterpret_cast<const uint4*>(g + e) : make_uint4(0, 0, 0, 0);
+          raw[i][s][2 + hh] = live ? *reinterpret_cast<const uint4*>(gz + e) : make_uint4(0, 0, 0, 0);
         }
       }
     }
+    float cs[8], sn[8];
+    rope_angles<D>(th, t, c, cs, sn);
 #pragma unroll
-    for (int i = 0; i < U; ++i) {
-      const bool live = ok && h0 + i0 + i < p.H;
-      const long row = (((long)b * p.H + h0 + i0 + i) * p.T + t) * D;
+    for (int i = 0; i < HG; ++i) {
+      const bool live = ok && h0 + i < p.H;
+      const long row = (((long)b * p.H + h0 + i) * p.T + t) * D;
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
         float a[8], z[8], g1[8], g2[8], u1[8], u2[8];
