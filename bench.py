@@ -11,7 +11,8 @@ included; pairs = B*H*T*(T+1)/2 for the causal mask):
   forward 4*d*pairs, backward 10*d*pairs, step 14*d*pairs.
 
 Timing: W untimed warm-up steps, then exactly K steps between CUDA events on
-the launching stream, bracketed by barrier + synchronize; the inputs (Q, K, V,
+the launching stream, bracketed by barrier + synchronize (per-kernel events in
+every 8th step give the per-kernel launch times); the inputs (Q, K, V,
 dO = 134 MB, plus O = 34 MB) exceed the 126 MB L2, so L2 is not flushed.
 Multi-GPU (torchrun): independent replicas, one per GPU, no data-path
 collective; value = all ranks' FLOPs / max over ranks of the timed region.
@@ -52,6 +53,15 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
+
+
+# Per-kernel CUDA events go into every EVENT_EVERY-th timed step only: each timing event costs
+# the GPU a few microseconds, which would otherwise land in the step time being measured.
+EVENT_EVERY = 8
+
+
+def sampled_steps(steps: int) -> int:
+    return (steps + EVENT_EVERY - 1) // EVENT_EVERY
 
 
 def peaks():
@@ -477,21 +487,22 @@ def main_prologue(args):
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    n_sampled = sampled_steps(args.steps)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_sampled)]
     sampler = ClockSampler(local)
     time.sleep(0.5)
     t_wall0 = time.time()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
-        step(events[i])
+        step(events[i // EVENT_EVERY] if i % EVENT_EVERY == 0 else None)
     end.record(stream)
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
     ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
-    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in events) / args.steps
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in events) / n_sampled
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in events) / n_sampled
     status = abi.gpt_attn_device_status(clear=True)
     # end to end: Q, K, dQ', dK' in from pinned host memory, Q', K', dQ, dK back out
     hin = [t.pin_memory() for t in x]
@@ -621,7 +632,8 @@ def main():
     if abi.gpt_attn_device_status(clear=True) != 0:
         raise RuntimeError("a kernel reported a wait timeout during warm-up")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    n_sampled = sampled_steps(args.steps)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(n_sampled)]
     sampler = ClockSampler(local)
     time.sleep(0.5)  # let the sampler start before the timed region
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -630,7 +642,7 @@ def main():
     t_wall0 = time.time()
     start.record(stream)
     for i in range(args.steps):
-        step(events[i])
+        step(events[i // EVENT_EVERY] if i % EVENT_EVERY == 0 else None)
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -641,7 +653,7 @@ def main():
     for ev in events:
         for j in range(len(kernels)):
             per_kernel_ms[j] += ev[j].elapsed_time(ev[j + 1])
-    per_kernel_ms = [x / args.steps for x in per_kernel_ms]
+    per_kernel_ms = [x / n_sampled for x in per_kernel_ms]
     status = abi.gpt_attn_device_status(clear=True)
 
     # ---------------------------------------------- end to end, host buffers

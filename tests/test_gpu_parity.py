@@ -6,6 +6,8 @@ Tolerances (bf16 inputs, fp32 accumulation, bf16 outputs):
   LSE  max |gpu - oracle|                       <= 1e-3
   dQ, dK, dV  ||gpu - oracle||_2 / ||oracle||_2  <= 2e-2   (per tensor; ||oracle|| floored
               at 1e-3 RMS so that exactly-zero gradients are measured in absolute terms)
+  RoPE + QK-norm prologue (Q', K', dQ, dK): every element within
+              |gpu - oracle| <= 2^-8 |oracle| + 2e-3 (bf16 rounding of the output)
 The full-size workloads run in the same launch configuration the benchmark
 times; for the two T = 2048, d = 128 workloads the explicit-Jacobian oracle
 backward (O(T^3) per head) is evaluated on a spread of sampled heads (every
