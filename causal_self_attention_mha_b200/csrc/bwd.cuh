@@ -33,8 +33,6 @@ __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16
   const long total = rows * TPR;
   const long stride = (long)gridDim.x * blockDim.x;
   const int lane = threadIdx.x & 31;
-  grid_dependency_wait();  // launched as a programmatic dependent of the forward
-  grid_dependents_launch();
   for (long base = (long)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < total;
        base += U * stride) {
     uint4 a[U], c[U];
@@ -284,12 +282,6 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, p.wait_limit_ns};
-  // Programmatic dependent launch: this CTA may have started while the previous kernel in
-  // the stream was still running (its setup above overlapped that kernel's tail).  Wait for
-  // that kernel's completion and memory before touching global memory, then let the next
-  // kernel's CTAs be scheduled as soon as SMs free up.
-  grid_dependency_wait();
-  grid_dependents_launch();
 
   if (warp >= L::COMPUTE_WARPS) {
     regs_shrink<88>();
@@ -744,12 +736,6 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, p.wait_limit_ns};
-  // Programmatic dependent launch: this CTA may have started while the previous kernel in
-  // the stream was still running (its setup above overlapped that kernel's tail).  Wait for
-  // that kernel's completion and memory before touching global memory, then let the next
-  // kernel's CTAs be scheduled as soon as SMs free up.
-  grid_dependency_wait();
-  grid_dependents_launch();
 
   if (warp >= L::COMPUTE_WARPS) {
     regs_shrink<88>();

@@ -11,7 +11,6 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
-#include <utility>
 
 #include "../../include/causalattn.h"
 #include "bwd.cuh"
@@ -184,34 +183,6 @@ int launch_status() {
 }
 
 // ------------------------------------------------------------- launchers
-// Launch with programmatic stream serialization: the kernel's CTAs may be scheduled as soon
-// as the previous kernel in the stream lets them (griddepcontrol.launch_dependents) and SMs
-// are free; the kernel itself waits (griddepcontrol.wait) for that kernel's completion before
-// touching global memory.  Used for the attention forward and backward kernels, which run
-// back to back.
-template <typename... KArgs, typename... Args>
-int launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
-                     cudaStream_t st, Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(block);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    t_last_cuda_error = cudaGetErrorString(e);
-    return GPT_ATTN_ERR_LAUNCH;
-  }
-  return launch_status();
-}
-
-
 // A window of w keys (the query's own included); w <= 0 or w >= T is no window,
 // which the kernels express as w = T (the band then covers every causal key).
 int effective_window(int window, int T) { return (window <= 0 || window > T) ? T : window; }
@@ -240,8 +211,9 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
   const int sms = sm_count();
   const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
-  return launch_dependent(ca::attn_fwd_kernel<D>, grid, ca::FwdLayout<D>::THREADS,
-                          ca::FwdLayout<D>::SMEM, st, mq, mk, mv, mo, p);
+  ca::attn_fwd_kernel<D><<<grid, ca::FwdLayout<D>::THREADS, ca::FwdLayout<D>::SMEM, st>>>(
+      mq, mk, mv, mo, p);
+  return launch_status();
 }
 
 template <int D>
@@ -251,9 +223,9 @@ int delta_impl(const void* o, const void* dout, float* delta, int B, int H, int 
   const long threads = rows * (D / 8);
   long blocks = (threads + 255) / 256;
   if (blocks > 148L * 16) blocks = 148L * 16;
-  return launch_dependent(ca::attn_bwd_delta_kernel<D>, (unsigned)blocks, 256, 0, st,
-                          static_cast<const __nv_bfloat16*>(o),
-                          static_cast<const __nv_bfloat16*>(dout), delta, rows);
+  ca::attn_bwd_delta_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
+  return launch_status();
 }
 
 template <int D>
@@ -288,10 +260,12 @@ int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const
   if (!make_map<D>(&mg0, g0, BH, T) || (dkdv && !make_map<D>(&mg1, g1, BH, T)))
     return GPT_ATTN_ERR_LAUNCH;
   if (dkdv)
-    return launch_dependent(ca::attn_bwd_dkdv_kernel<D>, grid, ca::DkdvLayout<D>::THREADS,
-                            ca::DkdvLayout<D>::SMEM, st, mq, mk, mv, mdo, mg0, mg1, p);
-  return launch_dependent(ca::attn_bwd_dq_kernel<D>, grid, ca::DqLayout<D>::THREADS,
-                          ca::DqLayout<D>::SMEM, st, mq, mk, mv, mdo, mg0, p);
+    ca::attn_bwd_dkdv_kernel<D><<<grid, ca::DkdvLayout<D>::THREADS, ca::DkdvLayout<D>::SMEM, st>>>(
+        mq, mk, mv, mdo, mg0, mg1, p);
+  else
+    ca::attn_bwd_dq_kernel<D><<<grid, ca::DqLayout<D>::THREADS, ca::DqLayout<D>::SMEM, st>>>(
+        mq, mk, mv, mdo, mg0, p);
+  return launch_status();
 }
 
 template <int D>

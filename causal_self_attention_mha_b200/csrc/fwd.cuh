@@ -185,12 +185,6 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, p.wait_limit_ns};
-  // Programmatic dependent launch: this CTA may have started while the previous kernel in
-  // the stream was still running (its setup above overlapped that kernel's tail).  Wait for
-  // that kernel's completion and memory before touching global memory, then let the next
-  // kernel's CTAs be scheduled as soon as SMs free up.
-  grid_dependency_wait();
-  grid_dependents_launch();
   if (warp >= L::SOFTMAX_WARPS) {
     // third warpgroup: give registers to the softmax warpgroups, then specialise
     regs_shrink<88>();

@@ -38,17 +38,6 @@ __device__ __forceinline__ uint32_t dynamic_smem_bytes() {
   return r;
 }
 
-// Programmatic dependent launch (griddepcontrol).  wait: block until the kernels this grid
-// depends on have completed and their memory is visible (returns at once when the grid was
-// not launched as a dependent).  launch_dependents: allow the next kernel in the stream to
-// be scheduled before this grid finishes.
-__device__ __forceinline__ void grid_dependency_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void grid_dependents_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
