@@ -77,3 +77,20 @@ def test_decode_reference_arm_under_torchrun_prints_once():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
     assert rec["config"]["cache_len"] == 8192 and rec["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_prologue_reference_arm_under_torchrun_prints_once():
+    """bench.py --workload prologue_wide_d128 --impl reference: rank 0 times the prologue
+    oracle (forward and backward for Q and K of a sample of heads) and prints one line."""
+    port = free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
+           "reference", "--gpus", "2", "--steps", "1", "--warmup", "0", "--workload",
+           "prologue_wide_d128"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
+    assert rec["config"]["T"] == 2048 and rec["e2e"]["h2d_bytes_per_step"] == 0
