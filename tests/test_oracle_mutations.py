@@ -3,13 +3,17 @@
 Each case plants one mistake in a copy of the oracle's C source (a dropped
 term, a wrong sign or index, a transposed operand, an off-by-one mask, the
 wrong logarithm), compiles the copy into a temporary directory, swaps it in,
-and runs the pin tests: at least one pin must fail.  Nothing here touches the
+and runs the pin tests: at least one pin must fail.  The numpy parts (KV-cache
+decode, RoPE + QK-norm prologue) get the same treatment from a mutated copy of
+their Python source.  Nothing here touches the
 committed oracle or the GPU.
 """
+import ast
 import ctypes
 import os
 import subprocess
 
+import numpy as np
 import pytest
 
 import oracle
@@ -80,3 +84,93 @@ def test_planted_mistake_is_caught(name, tmp_path, monkeypatch):
         except AssertionError:
             caught.append(fn.__name__)
     assert caught, f"no pin caught the planted mistake {name!r}"
+
+
+# ---------------------------------------------------------- the numpy parts of the oracle
+# The KV-cache decode and the RoPE + QK-norm prologue are written in numpy inside
+# oracle/__init__.py.  Each case plants one mistake in a copy of that source, rebuilds the
+# affected functions from the copy, swaps them into the oracle module and runs the pins.
+
+
+PY_SRC = oracle.__file__
+PY_FUNCS = ("_f64", "_rope_angles", "_rope", "qk_prologue_forward", "qk_prologue_backward",
+            "decode_forward")
+
+PY_MUTATIONS = {
+    "decode_sees_one_key_too_few": ("n = L - Tq + t + 1 ", "n = L - Tq + t "),
+    "decode_sees_whole_cache": ("n = L - Tq + t + 1 ", "n = L "),
+    "decode_without_scale": ("s = scale * (kc[b, :n, h, :] @ q[b, t, h, :])",
+                             "s = (kc[b, :n, h, :] @ q[b, t, h, :])"),
+    "decode_lse_in_log2": ("lse[b, h, t] = m + np.log(z)", "lse[b, h, t] = m + np.log2(z)"),
+    "decode_unnormalised": ("o[b, t, h] = (w / z) @ vc", "o[b, t, h] = w @ vc"),
+    "decode_first_token_query": ("@ q[b, t, h, :])", "@ q[b, 0, h, :])"),
+    "rope_adjacent_pairs": ("x1, x2 = x[..., :h], x[..., h:]", "x1, x2 = x[..., 0::2], x[..., 1::2]"),
+    "rope_not_a_rotation": ("-x1 * s + x2 * cos", "x1 * s + x2 * cos"),
+    "rope_frequency_exponent": ("theta = base ** (-2.0 * i / d)", "theta = base ** (-i / d)"),
+    "rope_positions_from_one": ("ang = np.arange(T, dtype=np.float64)[:, None]",
+                                "ang = np.arange(1, T + 1, dtype=np.float64)[:, None]"),
+    "norm_without_eps": ("r = np.sqrt(np.mean(u * u, axis=-1, keepdims=True) + eps)\n    return",
+                         "r = np.sqrt(np.mean(u * u, axis=-1, keepdims=True))\n    return"),
+    "norm_sum_not_mean": ("r = np.sqrt(np.mean(u * u, axis=-1, keepdims=True) + eps)\n    return",
+                          "r = np.sqrt(np.sum(u * u, axis=-1, keepdims=True) + eps)\n    return"),
+    "forward_drops_gain": ("return gain * u / r", "return u / r"),
+    "backward_drops_projection": ("du = (gain / r) * (dz - u * s / (d * r * r))",
+                                  "du = (gain / r) * dz"),
+    "backward_projection_without_d": ("du = (gain / r) * (dz - u * s / (d * r * r))",
+                                      "du = (gain / r) * (dz - u * s / (r * r))"),
+    "backward_rotates_forward": ("return _rope(du, cos, sin, inverse=True)",
+                                 "return _rope(du, cos, sin)"),
+    "backward_drops_gain": ("du = (gain / r) * (dz", "du = (1.0 / r) * (dz"),
+}
+
+PY_PIN_TESTS = [
+    (pins.test_decode_is_the_last_rows_of_causal_attention, {"B": 1, "H": 2, "Tq": 1, "L": 1, "d": 4}),
+    (pins.test_decode_is_the_last_rows_of_causal_attention, {"B": 1, "H": 2, "Tq": 5, "L": 20, "d": 4}),
+    (pins.test_decode_single_cached_token, {}),
+    (pins.test_decode_against_torch_sdpa_fp64, {}),
+    (pins.test_prologue_against_torch_fp64, {}),
+    (pins.test_prologue_position_zero_is_plain_rms_norm, {}),
+    (pins.test_prologue_rotation_keeps_rms_and_commutes_with_the_norm, {}),
+    (pins.test_prologue_scores_depend_on_relative_position_only, {}),
+    (pins.test_prologue_finite_differences, {}),
+]
+
+
+def _mutant_functions(old, new):
+    src = open(PY_SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old!r}"
+    tree = ast.parse(src.replace(old, new))
+    keep = [n for n in tree.body if isinstance(n, ast.FunctionDef) and n.name in PY_FUNCS]
+    assert {n.name for n in keep} == set(PY_FUNCS)
+    ns = {"np": oracle.np}
+    exec(compile(ast.Module(body=keep, type_ignores=[]), "mutant_oracle", "exec"), ns)
+    return {name: ns[name] for name in PY_FUNCS}
+
+
+def test_python_mutation_anchors_are_unique():
+    src = open(PY_SRC).read()
+    for name, (old, _) in PY_MUTATIONS.items():
+        assert src.count(old) == 1, name
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTATIONS))
+def test_planted_mistake_in_numpy_oracle_is_caught(name, monkeypatch):
+    old, new = PY_MUTATIONS[name]
+    for fn_name, fn in _mutant_functions(old, new).items():
+        monkeypatch.setattr(oracle, fn_name, fn)
+    caught = []
+    for fn, kw in PY_PIN_TESTS:
+        try:
+            with np.errstate(all="ignore"):
+                fn(**kw)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(fn.__name__)
+    assert caught, f"no pin caught the planted mistake {name!r}"
+
+
+def test_unmutated_numpy_oracle_passes_every_pin(monkeypatch):
+    """The harness itself: the functions rebuilt from the unchanged source pass all pins."""
+    for fn_name, fn in _mutant_functions("def ", "def ").items():
+        monkeypatch.setattr(oracle, fn_name, fn)
+    for fn, kw in PY_PIN_TESTS:
+        fn(**kw)

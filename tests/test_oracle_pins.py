@@ -460,7 +460,7 @@ def test_decode_against_torch_sdpa_fp64():
 
 def torch_prologue(x, base=10000.0, gain=1.2, eps=1e-6):
     """An independent torch float64 statement: complex-number RoPE (pairs (i, i + d/2) as
-    real and imaginary parts, multiplied by e^{i pos theta}) and torch's rms_norm."""
+    real and imaginary parts, multiplied by e^{-i pos theta}) and torch's rms_norm."""
     B, H, T, d = x.shape
     h = d // 2
     theta = base ** (-torch.arange(0, d, 2, dtype=torch.float64) / d)
