@@ -282,8 +282,10 @@ int decode_impl(const void* q, const void* kc, const void* vc, void* o, float* l
   p.L = L;
   p.n_chunks = (L + ca::kDecChunk - 1) / ca::kDecChunk;
   const size_t rows = (size_t)B * H * Tq * p.n_chunks;
-  p.part_ml = ws;
-  p.part_o = ws + rows * 2;
+  // partial outputs first: every (row, chunk) slice of them starts on a 16-byte boundary
+  // (the merge kernel reads them as float4 / float2 vectors)
+  p.part_o = ws;
+  p.part_ml = ws + rows * D;
   p.scale_log2 = scale * ca::kLog2e;
   p.wait_limit_ns = kWaitLimitNs;
   dim3 grid((unsigned)p.n_chunks, (unsigned)H, (unsigned)B);

@@ -230,7 +230,8 @@ __global__ void __launch_bounds__(kDecThreads)
 // Merges the chunks of one (batch, head, token).  kCombWarps warps each fold a fixed
 // slice of the chunks (chunk order within the slice), lane l holding columns
 // l*VEC .. l*VEC + VEC - 1; the warps' results are then folded in warp order.  The
-// order is fixed, so the result is deterministic.
+// order is fixed, so the result is deterministic.  Every chunk's partial output is
+// finite (zero for a chunk without visible keys), so weight-zero chunks add nothing.
 constexpr int kCombWarps = 8;
 
 template <int D>
@@ -248,20 +249,47 @@ __global__ void __launch_bounds__(kCombWarps * 32)
   const float* po = part_o + (size_t)idx * n_chunks * D;
   const int per = (n_chunks + kCombWarps - 1) / kCombWarps;
   const int c0 = warp * per, c1 = min(n_chunks, c0 + per);
+  // The slice is taken 32 chunks at a time: lane j loads chunk j's (m, l), the group's
+  // maximum and weights follow from shuffles, then the group's partial outputs are loaded
+  // without waiting on one another and summed in chunk order.
   float M = -INFINITY, l = 0.f, acc[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
-  for (int c = c0; c < c1; ++c) {
-    const float mc = ml[2 * c];
-    if (mc == -INFINITY) continue;  // a chunk that holds no visible key
-    float x[VEC];
+  for (int g0 = c0; g0 < c1; g0 += 32) {
+    const int c = g0 + lane;
+    const float mc = c < c1 ? ml[2 * c] : -INFINITY;
+    const float lc = c < c1 ? ml[2 * c + 1] : 0.f;
+    float mg = mc;
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) x[v] = po[(size_t)c * D + lane * VEC + v];
-    const float mn = fmaxf(M, mc);
-    const float fo = ex2(M - mn), fc = ex2(mc - mn);  // ex2(-inf) = 0 for the first chunk
-    l = l * fo + ml[2 * c + 1] * fc;
+    for (int off = 16; off > 0; off >>= 1) mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, off));
+    if (mg == -INFINITY) continue;  // no visible key in the whole group (warp-uniform)
+    const float mn = fmaxf(M, mg);
+    const float fo = ex2(M - mn);  // ex2(-inf) = 0 before the first group
+    const float fc = (mc == -INFINITY) ? 0.f : ex2(mc - mn);
+    float lg = lc * fc;
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) acc[v] = acc[v] * fo + x[v] * fc;
+    for (int off = 16; off > 0; off >>= 1) lg += __shfl_xor_sync(0xffffffffu, lg, off);
+    l = l * fo + lg;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] *= fo;
+    const int n = min(32, c1 - g0);
+#pragma unroll 8
+    for (int j = 0; j < n; ++j) {
+      const float fj = __shfl_sync(0xffffffffu, fc, j);
+      const float* src = po + (size_t)(g0 + j) * D + lane * VEC;
+      float x[VEC];
+      if constexpr (VEC == 4) {
+        const float4 t4 = *reinterpret_cast<const float4*>(src);
+        x[0] = t4.x; x[1] = t4.y; x[2] = t4.z; x[3] = t4.w;
+      } else if constexpr (VEC == 2) {
+        const float2 t2 = *reinterpret_cast<const float2*>(src);
+        x[0] = t2.x; x[1] = t2.y;
+      } else {
+        x[0] = src[0];
+      }
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] = fmaf(x[v], fj, acc[v]);
+    }
     M = mn;
   }
   if (lane == 0) {
