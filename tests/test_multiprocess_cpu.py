@@ -36,7 +36,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_with_two_gloo_ranks():
     port = free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork: earlier tests started threads
     mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
     assert out[0] == out[1] == 5.0
 
