@@ -94,3 +94,29 @@ def test_prologue_reference_arm_under_torchrun_prints_once():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
     assert rec["config"]["T"] == 2048 and rec["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_sampled_steps_cover_the_timed_loop():
+    sys.path.insert(0, ROOT)
+    import bench
+    for steps in (1, 7, 8, 9, 2000):
+        n = bench.sampled_steps(steps)
+        sampled = [i for i in range(steps) if i % bench.EVENT_EVERY == 0]
+        assert n == len(sampled) and n >= 1
+
+
+def test_recorded_traffic_only_for_matching_sources(tmp_path):
+    """A traffic record is used only while the kernel sources hash to the recorded value."""
+    sys.path.insert(0, ROOT)
+    import bench
+    good = tmp_path / "good.md"
+    good.write_text(f"source_hash: {bench.kernel_source_hash(bench.PROLOGUE_KERNEL_FILES)}\n\n"
+                    "| kernel | workload | bytes per launch |\n|---|---|---|\n"
+                    "| rope_qknorm_bwd | prologue_wide_d128 | 1.5e+08 |\n")
+    stale = tmp_path / "stale.md"
+    stale.write_text(good.read_text().replace("source_hash: ", "source_hash: 0"))
+    args = ("rope_qknorm_bwd", "prologue_wide_d128")
+    assert bench.recorded_traffic(*args, str(good), bench.PROLOGUE_KERNEL_FILES) == 1.5e8
+    assert bench.recorded_traffic(*args, str(stale), bench.PROLOGUE_KERNEL_FILES) is None
+    assert bench.recorded_traffic("rope_qknorm_fwd", "prologue_wide_d128", str(good),
+                                  bench.PROLOGUE_KERNEL_FILES) is None
