@@ -36,11 +36,14 @@
  *
  * Ownership.  Every pointer is caller-owned DEVICE memory on the current CUDA
  * device.  The library allocates no memory; it keeps no state besides
- * per-device attribute caches and one device-side status word.
+ * per-device attribute and occupancy caches, one device-side status word and
+ * the fixed delta scratch of gpt_attn_bwd_static_ws.
  *
  * Asynchrony.  Calls validate their arguments, enqueue kernels on `stream`
  * (a cudaStream_t; NULL = the legacy default stream) and return.  Outputs are
- * valid once the stream has reached that point.  Inputs are not modified.
+ * valid once the stream has reached that point.  Inputs are not modified
+ * (except where a caller passes an input buffer as the output of a call that
+ * allows it: the RoPE + QK-norm calls work in place).
  * dq, dk, dv, o, lse, delta are fully overwritten, never accumulated into.
  *
  * Errors.  Every call returns a gpt_attn_status.  Nothing aborts, throws or
