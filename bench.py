@@ -11,8 +11,9 @@ included; pairs = B*H*T*(T+1)/2 for the causal mask):
   forward 4*d*pairs, backward 10*d*pairs, step 14*d*pairs.
 
 Timing: W untimed warm-up steps, then exactly K steps between CUDA events on
-the launching stream, bracketed by barrier + synchronize (per-kernel events in
-every 8th step give the per-kernel launch times); the inputs (Q, K, V,
+the launching stream, bracketed by barrier + synchronize, with no other events
+inside; per-kernel launch times come from a separate phase afterwards (events
+in every 4th of 64 steps, never the first); the inputs (Q, K, V,
 dO = 134 MB, plus O = 34 MB) exceed the 126 MB L2, so L2 is not flushed.
 Multi-GPU (torchrun): independent replicas, one per GPU, no data-path
 collective; value = all ranks' FLOPs / max over ranks of the timed region.
@@ -55,13 +56,64 @@ def parse():
     return ap.parse_args()
 
 
-# Per-kernel CUDA events go into every EVENT_EVERY-th timed step only: each timing event costs
-# the GPU a few microseconds, which would otherwise land in the step time being measured.
-EVENT_EVERY = 8
+# Per-kernel times come from a phase of their own after the timed region: PROFILE_STEPS steps,
+# per-kernel CUDA events in every EVENT_EVERY-th of them at offset EVENT_EVERY // 2, so that no
+# sampled step follows a synchronize (the host must be ahead of the GPU for the gaps between
+# events to be kernel time) and the events' own cost stays out of the headline.
+EVENT_EVERY = 4
+PROFILE_STEPS = 64
+KERNEL_SUM_TOL = 0.03  # the kernel times must add up to the step time within 3 %
 
 
 def sampled_steps(steps: int) -> int:
-    return (steps + EVENT_EVERY - 1) // EVENT_EVERY
+    return len(sampled_indices(steps))
+
+
+def sampled_indices(steps: int):
+    """Steps of the profile phase that carry per-kernel events (never the first)."""
+    return [i for i in range(steps) if i % EVENT_EVERY == EVENT_EVERY // 2]
+
+
+def kernel_sum_check(kernel_ms, ms_per_step: float):
+    """(ratio of the summed kernel times to the step time, warning text or None)."""
+    total = sum(kernel_ms)
+    ratio = total / ms_per_step if ms_per_step > 0 else float("nan")
+    if not abs(ratio - 1.0) <= KERNEL_SUM_TOL:
+        return ratio, (f"per-kernel times sum to {total:.4f} ms against a {ms_per_step:.4f} ms "
+                       f"step ({100 * (ratio - 1):+.1f} %): not trusted for the roofline")
+    return ratio, None
+
+
+def profile_kernels(step, stream, n_kernels: int, dev):
+    """Average duration (ms) of each of a step's n_kernels launches: PROFILE_STEPS back-to-back
+    steps, CUDA events between the launches of the sampled ones.  step(ev) records ev[j] before
+    launch j and ev[n_kernels] after the last (ev None: no events)."""
+    import torch
+    idx = set(sampled_indices(PROFILE_STEPS))
+    events = {i: [torch.cuda.Event(enable_timing=True) for _ in range(n_kernels + 1)] for i in idx}
+    torch.cuda.synchronize(dev)
+    for i in range(PROFILE_STEPS):
+        step(events.get(i))
+    torch.cuda.synchronize(dev)
+    per = [0.0] * n_kernels
+    for ev in events.values():
+        for j in range(n_kernels):
+            per[j] += ev[j].elapsed_time(ev[j + 1])
+    return [x / len(events) for x in per]
+
+
+def host_us_per_call(step, calls_per_step: int, dev, steps: int = 32) -> float:
+    """Host time to enqueue one library call (binding checks, tensor-map encoding, launch),
+    from the wall time of enqueueing `steps` steps onto an idle GPU (well below the launch-queue
+    depth, so the host never waits for the GPU)."""
+    import torch
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step(None)
+    t1 = time.perf_counter()
+    torch.cuda.synchronize(dev)
+    return 1e6 * (t1 - t0) / (steps * calls_per_step)
 
 
 def peaks():
@@ -487,22 +539,20 @@ def main_prologue(args):
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    n_sampled = sampled_steps(args.steps)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_sampled)]
     sampler = ClockSampler(local)
     time.sleep(0.5)
     t_wall0 = time.time()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for i in range(args.steps):
-        step(events[i // EVENT_EVERY] if i % EVENT_EVERY == 0 else None)
+    for _ in range(args.steps):
+        step()
     end.record(stream)
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
     ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in events) / n_sampled
-    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in events) / n_sampled
+    fwd_ms, bwd_ms = profile_kernels(step, stream, 2, dev)
+    sum_ratio, sum_warning = kernel_sum_check([fwd_ms, bwd_ms], ms)
     status = abi.gpt_attn_device_status(clear=True)
     # end to end: Q, K, dQ', dK' in from pinned host memory, Q', K', dQ, dK back out
     hin = [t.pin_memory() for t in x]
@@ -537,6 +587,7 @@ def main_prologue(args):
             "dtype": "bf16", "data": "synthetic: seeded N(0,1) bf16 Q, K, dQ', dK'",
             "config": prologue_config(c, f"replicas x{world}" if world > 1 else "single GPU"),
             "kernel_ms": {"rope_qknorm_fwd": fwd_ms, "rope_qknorm_bwd": bwd_ms},
+            "kernel_sum_vs_step": sum_ratio,
             "fwd_gbs": 4.0 * tensor_bytes / (fwd_ms * 1e-3) / 1e9,
             "roofline": {"kernel": "rope_qknorm_bwd", "bound": "hbm", "achieved": achieved,
                          "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
@@ -551,6 +602,8 @@ def main_prologue(args):
             "clocks": clocks,
             "device_status": status,
         }
+        if sum_warning:
+            line["kernel_ms_warning"] = sum_warning
         if world == 1 and not args.no_cpu_baseline:
             dt, byts = prologue_oracle_sample(c, x, 8)
             line["cpu_baseline"] = {"value": byts / dt / 1e9, "unit": "GB/s", "cores": 1,
@@ -607,7 +660,6 @@ def main():
     step_flops = 14.0 * d * pairs
     stream = torch.cuda.Stream(device=dev)
     kernels = ["attn_fwd", "attn_bwd_delta", "attn_bwd_dkdv", "attn_bwd_dq"]
-    n_ev = 5
 
     def step(ev=None):
         if ev is not None:
@@ -632,8 +684,6 @@ def main():
     if abi.gpt_attn_device_status(clear=True) != 0:
         raise RuntimeError("a kernel reported a wait timeout during warm-up")
 
-    n_sampled = sampled_steps(args.steps)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(n_sampled)]
     sampler = ClockSampler(local)
     time.sleep(0.5)  # let the sampler start before the timed region
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -641,19 +691,17 @@ def main():
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
     start.record(stream)
-    for i in range(args.steps):
-        step(events[i // EVENT_EVERY] if i % EVENT_EVERY == 0 else None)
+    for _ in range(args.steps):
+        step()
     end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
     elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
-    per_kernel_ms = [0.0] * len(kernels)
-    for ev in events:
-        for j in range(len(kernels)):
-            per_kernel_ms[j] += ev[j].elapsed_time(ev[j + 1])
-    per_kernel_ms = [x / n_sampled for x in per_kernel_ms]
+    # per-kernel durations and host cost per call, outside the timed region
+    per_kernel_ms = profile_kernels(step, stream, len(kernels), dev)
+    host_us = host_us_per_call(step, len(kernels), dev)
     status = abi.gpt_attn_device_status(clear=True)
 
     # ---------------------------------------------- end to end, host buffers
@@ -684,6 +732,7 @@ def main():
         fwd_flops, bwd_flops = 4.0 * d * pairs, 10.0 * d * pairs
         fwd_ms = per_kernel_ms[0]
         bwd_ms = sum(per_kernel_ms[1:])
+        sum_ratio, sum_warning = kernel_sum_check(per_kernel_ms, elapsed_ms / args.steps)
         # roofline of the dominant kernel (largest share of the step)
         kflops = {"attn_fwd": 4.0 * d * pairs, "attn_bwd_dkdv": 8.0 * d * pairs,
                   "attn_bwd_dq": 6.0 * d * pairs}
@@ -717,6 +766,10 @@ def main():
             "fwd_tflops": fwd_flops / (fwd_ms * 1e-3) / 1e12,
             "bwd_tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,
             "kernel_ms": dict(zip(kernels, per_kernel_ms)),
+            "kernel_ms_source": (f"{sampled_steps(PROFILE_STEPS)} sampled steps of a "
+                                 f"{PROFILE_STEPS}-step phase after the timed region"),
+            "kernel_sum_vs_step": sum_ratio,
+            "host_us_per_call": host_us,
             "roofline": roof,
             "e2e": {"value": replica_value(step_flops, world, e2e_ms), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": step_host.h2d_bytes(),
@@ -725,6 +778,8 @@ def main():
             "clocks": clocks,
             "device_status": status,
         }
+        if sum_warning:
+            line["kernel_ms_warning"] = sum_warning
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             cores = len(os.sched_getaffinity(0))

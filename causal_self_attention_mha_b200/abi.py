@@ -108,10 +108,19 @@ def version() -> int:
     return int(load().gpt_attn_version())
 
 
-def _stream(stream) -> Optional[int]:
+def _stream(stream, device: Optional[torch.device] = None) -> Optional[int]:
+    """The cudaStream_t handle to launch on.  The library launches on the CURRENT CUDA device,
+    so the tensors' device (`device`) must be the current one, and a torch stream passed in must
+    belong to it: otherwise one device's pointers would reach kernels and TMA descriptors on
+    another."""
+    if device is not None and device.index != torch.cuda.current_device():
+        raise ValueError(f"tensors are on {device} but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()}; call under torch.cuda.device({device})")
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
-    if isinstance(stream, torch.cuda.Stream):
+    if hasattr(stream, "cuda_stream"):  # torch.cuda.Stream / ExternalStream
+        if device is not None and stream.device != device:
+            raise ValueError(f"stream belongs to {stream.device}, tensors are on {device}")
         return stream.cuda_stream
     return int(stream)
 
@@ -133,17 +142,19 @@ def _bhtd(name: str, t: torch.Tensor, ref: Optional[torch.Tensor] = None):
     return tuple(t.shape)
 
 
-def _side(name: str, t: torch.Tensor, shape, dtype) -> None:
+def _side(name: str, t: torch.Tensor, shape, dtype, ref: Optional[torch.Tensor] = None) -> None:
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+    if ref is not None and t.device != ref.device:
+        raise ValueError(f"{name} is on {t.device}, q is on {ref.device}")
 
 
-def _doc_ptr(doc, B, T):
+def _doc_ptr(doc, B, T, ref=None):
     if doc is None:
         return None
-    _side("doc_offsets", doc, (B, T), torch.int32)
+    _side("doc_offsets", doc, (B, T), torch.int32, ref)
     return doc.data_ptr()
 
 
@@ -152,10 +163,10 @@ def gpt_attn_fwd(q, k, v, o, lse, scale: float, doc_offsets=None, stream=None) -
     _bhtd("k", k, q)
     _bhtd("v", v, q)
     _bhtd("o", o, q)
-    _side("lse", lse, (B, H, T), torch.float32)
+    _side("lse", lse, (B, H, T), torch.float32, q)
     _check("gpt_attn_fwd", load().gpt_attn_fwd(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, d,
-        float(scale), _doc_ptr(doc_offsets, B, T), _stream(stream)))
+        float(scale), _doc_ptr(doc_offsets, B, T, q), _stream(stream, q.device)))
 
 
 def gpt_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, scale: float, doc_offsets=None,
@@ -163,12 +174,12 @@ def gpt_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, scale: float, doc_
     B, H, T, d = _bhtd("q", q)
     for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
         _bhtd(name, t, q)
-    _side("lse", lse, (B, H, T), torch.float32)
-    _side("delta_ws", delta_ws, (B, H, T), torch.float32)
+    _side("lse", lse, (B, H, T), torch.float32, q)
+    _side("delta_ws", delta_ws, (B, H, T), torch.float32, q)
     _check("gpt_attn_bwd", load().gpt_attn_bwd(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), delta_ws.data_ptr(), B, H, T, d, float(scale),
-        _doc_ptr(doc_offsets, B, T), _stream(stream)))
+        _doc_ptr(doc_offsets, B, T, q), _stream(stream, q.device)))
 
 
 def gpt_attn_fwd_window(q, k, v, o, lse, scale: float, window: int, doc_offsets=None,
@@ -178,10 +189,10 @@ def gpt_attn_fwd_window(q, k, v, o, lse, scale: float, window: int, doc_offsets=
     _bhtd("k", k, q)
     _bhtd("v", v, q)
     _bhtd("o", o, q)
-    _side("lse", lse, (B, H, T), torch.float32)
+    _side("lse", lse, (B, H, T), torch.float32, q)
     _check("gpt_attn_fwd_window", load().gpt_attn_fwd_window(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, d,
-        float(scale), _doc_ptr(doc_offsets, B, T), int(window), _stream(stream)))
+        float(scale), _doc_ptr(doc_offsets, B, T, q), int(window), _stream(stream, q.device)))
 
 
 def gpt_attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, scale: float, window: int,
@@ -190,12 +201,12 @@ def gpt_attn_bwd_window(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, scale: floa
     B, H, T, d = _bhtd("q", q)
     for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
         _bhtd(name, t, q)
-    _side("lse", lse, (B, H, T), torch.float32)
-    _side("delta_ws", delta_ws, (B, H, T), torch.float32)
+    _side("lse", lse, (B, H, T), torch.float32, q)
+    _side("delta_ws", delta_ws, (B, H, T), torch.float32, q)
     _check("gpt_attn_bwd_window", load().gpt_attn_bwd_window(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), delta_ws.data_ptr(), B, H, T, d, float(scale),
-        _doc_ptr(doc_offsets, B, T), int(window), _stream(stream)))
+        _doc_ptr(doc_offsets, B, T, q), int(window), _stream(stream, q.device)))
 
 
 def gpt_attn_bwd_static_ws(q, k, v, o, dout, lse, dq, dk, dv, scale: float, doc_offsets=None,
@@ -205,19 +216,19 @@ def gpt_attn_bwd_static_ws(q, k, v, o, dout, lse, dq, dk, dv, scale: float, doc_
     B, H, T, d = _bhtd("q", q)
     for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
         _bhtd(name, t, q)
-    _side("lse", lse, (B, H, T), torch.float32)
+    _side("lse", lse, (B, H, T), torch.float32, q)
     _check("gpt_attn_bwd_static_ws", load().gpt_attn_bwd_static_ws(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T, d, float(scale),
-        _doc_ptr(doc_offsets, B, T), _stream(stream)))
+        _doc_ptr(doc_offsets, B, T, q), _stream(stream, q.device)))
 
 
 def gpt_attn_bwd_preprocess(o, dout, delta, stream=None) -> None:
     B, H, T, d = _bhtd("o", o)
     _bhtd("dout", dout, o)
-    _side("delta", delta, (B, H, T), torch.float32)
+    _side("delta", delta, (B, H, T), torch.float32, o)
     _check("gpt_attn_bwd_preprocess", load().gpt_attn_bwd_preprocess(
-        o.data_ptr(), dout.data_ptr(), delta.data_ptr(), B, H, T, d, _stream(stream)))
+        o.data_ptr(), dout.data_ptr(), delta.data_ptr(), B, H, T, d, _stream(stream, o.device)))
 
 
 def gpt_attn_bwd_dkdv(q, k, v, dout, lse, delta, dk, dv, scale: float, doc_offsets=None,
@@ -225,12 +236,12 @@ def gpt_attn_bwd_dkdv(q, k, v, dout, lse, delta, dk, dv, scale: float, doc_offse
     B, H, T, d = _bhtd("q", q)
     for name, t in (("k", k), ("v", v), ("dout", dout), ("dk", dk), ("dv", dv)):
         _bhtd(name, t, q)
-    _side("lse", lse, (B, H, T), torch.float32)
-    _side("delta", delta, (B, H, T), torch.float32)
+    _side("lse", lse, (B, H, T), torch.float32, q)
+    _side("delta", delta, (B, H, T), torch.float32, q)
     _check("gpt_attn_bwd_dkdv", load().gpt_attn_bwd_dkdv(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), lse.data_ptr(), delta.data_ptr(),
-        dk.data_ptr(), dv.data_ptr(), B, H, T, d, float(scale), _doc_ptr(doc_offsets, B, T),
-        _stream(stream)))
+        dk.data_ptr(), dv.data_ptr(), B, H, T, d, float(scale), _doc_ptr(doc_offsets, B, T, q),
+        _stream(stream, q.device)))
 
 
 def gpt_attn_bwd_dq(q, k, v, dout, lse, delta, dq, scale: float, doc_offsets=None,
@@ -238,11 +249,11 @@ def gpt_attn_bwd_dq(q, k, v, dout, lse, delta, dq, scale: float, doc_offsets=Non
     B, H, T, d = _bhtd("q", q)
     for name, t in (("k", k), ("v", v), ("dout", dout), ("dq", dq)):
         _bhtd(name, t, q)
-    _side("lse", lse, (B, H, T), torch.float32)
-    _side("delta", delta, (B, H, T), torch.float32)
+    _side("lse", lse, (B, H, T), torch.float32, q)
+    _side("delta", delta, (B, H, T), torch.float32, q)
     _check("gpt_attn_bwd_dq", load().gpt_attn_bwd_dq(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), lse.data_ptr(), delta.data_ptr(),
-        dq.data_ptr(), B, H, T, d, float(scale), _doc_ptr(doc_offsets, B, T), _stream(stream)))
+        dq.data_ptr(), B, H, T, d, float(scale), _doc_ptr(doc_offsets, B, T, q), _stream(stream, q.device)))
 
 
 def gpt_attn_decode_workspace_size(B: int, H: int, Tq: int, L: int, d: int) -> int:
@@ -258,13 +269,14 @@ def gpt_attn_decode(q, k_cache, v_cache, o, lse, workspace, scale: float, stream
         raise ValueError("k_cache must be [B, L, H, d] with q's B, H, d")
     _bhtd("v_cache", v_cache, k_cache)
     _bhtd("o", o, q)
-    _side("lse", lse, (B, H, Tq), torch.float32)
-    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _side("lse", lse, (B, H, Tq), torch.float32, q)
+    if (not isinstance(workspace, torch.Tensor) or not workspace.is_cuda
+            or not workspace.is_contiguous() or workspace.device != q.device):
+        raise ValueError("workspace must be a contiguous CUDA tensor on q's device")
     nbytes = workspace.numel() * workspace.element_size()
     _check("gpt_attn_decode", load().gpt_attn_decode(
         q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), o.data_ptr(), lse.data_ptr(),
-        workspace.data_ptr(), nbytes, B, H, Tq, L, d, float(scale), _stream(stream)))
+        workspace.data_ptr(), nbytes, B, H, Tq, L, d, float(scale), _stream(stream, q.device)))
 
 
 def gpt_attn_check_doc_offsets(doc_offsets, stream=None) -> bool:
@@ -273,7 +285,8 @@ def gpt_attn_check_doc_offsets(doc_offsets, stream=None) -> bool:
         raise ValueError("doc_offsets must be a [B,T] tensor")
     B, T = doc_offsets.shape
     _side("doc_offsets", doc_offsets, (B, T), torch.int32)
-    s = load().gpt_attn_check_doc_offsets(doc_offsets.data_ptr(), B, T, _stream(stream))
+    s = load().gpt_attn_check_doc_offsets(doc_offsets.data_ptr(), B, T,
+                                             _stream(stream, doc_offsets.device))
     if s == GPT_ATTN_ERR_BAD_DOC_OFFSETS:
         return False
     _check("gpt_attn_check_doc_offsets", s)
@@ -367,7 +380,7 @@ def gpt_attn_rope_qknorm_fwd(q, k, q_out, k_out, rope_base: float = 10000.0, gai
     _same_or_disjoint("k_out", k_out, k, (q, q_out))
     _check("gpt_attn_rope_qknorm_fwd", load().gpt_attn_rope_qknorm_fwd(
         q.data_ptr(), k.data_ptr(), q_out.data_ptr(), k_out.data_ptr(), B, H, T, d,
-        float(rope_base), float(gain), float(eps), _stream(stream)))
+        float(rope_base), float(gain), float(eps), _stream(stream, q.device)))
 
 
 def gpt_attn_rope_qknorm_bwd(q, k, dq_out, dk_out, dq, dk, rope_base: float = 10000.0,
@@ -381,7 +394,7 @@ def gpt_attn_rope_qknorm_bwd(q, k, dq_out, dk_out, dq, dk, rope_base: float = 10
     _same_or_disjoint("dk", dk, dk_out, (q, k, dq_out, dq))
     _check("gpt_attn_rope_qknorm_bwd", load().gpt_attn_rope_qknorm_bwd(
         q.data_ptr(), k.data_ptr(), dq_out.data_ptr(), dk_out.data_ptr(), dq.data_ptr(),
-        dk.data_ptr(), B, H, T, d, float(rope_base), float(gain), float(eps), _stream(stream)))
+        dk.data_ptr(), B, H, T, d, float(rope_base), float(gain), float(eps), _stream(stream, q.device)))
 
 
 def rope_qknorm(q, k, rope_base: float = 10000.0, gain: float = 1.2, eps: float = 1e-6,

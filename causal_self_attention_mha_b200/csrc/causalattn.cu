@@ -315,7 +315,11 @@ size_t decode_ws_bytes(int B, int H, int Tq, int L, int d) {
 }
 
 // -------------------------------------------------------- utility kernels
+// Verdict word of gpt_attn_check_doc_offsets.  One per device; every call clears it, runs the
+// checker and reads it back before returning, all under g_doc_mu, so calls from several host
+// threads (on any streams) never see one another's verdict.
 __device__ int g_doc_bad;
+std::mutex g_doc_mu;
 
 __global__ void check_doc_kernel(const int32_t* doc, int B, int T) {
   const long n = (long)B * T;
@@ -601,6 +605,7 @@ int gpt_attn_check_doc_offsets(const int32_t* doc_offsets, int B, int T, void* s
   int s = ensure_device();
   if (s) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_doc_mu);  // clear, check, read back: one call at a time
   const int zero = 0;
   if (cudaMemcpyToSymbolAsync(g_doc_bad, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) !=
       cudaSuccess) {

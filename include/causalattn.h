@@ -209,6 +209,13 @@ int gpt_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dou
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
+ *   - The array is part of the library's device code: it is reserved when
+ *     that code is loaded onto a device, which (with CUDA's default lazy
+ *     module loading) happens during the first library call of any kind on
+ *     that device -- possibly this one.  A caller whose allocator will own
+ *     every free byte of the device should make one library call (any entry
+ *     point) or set CUDA_MODULE_LOADING=EAGER before handing the device over;
+ *     after that, calls reserve nothing further.
  *   - All calls share the one array, which keeps the last call's contents
  *     (delta is rewritten in full by every call, so nothing needs clearing):
  *     calls whose work overlaps on the GPU -- two streams, two threads --
@@ -223,6 +230,10 @@ int gpt_attn_bwd_static_ws(const void* q, const void* k, const void* v, const vo
 /*
  * Checks a doc_offsets array on the device against the validity rule above.
  * Synchronises `stream`.  Returns GPT_ATTN_OK or GPT_ATTN_ERR_BAD_DOC_OFFSETS.
+ * The verdict passes through one library-owned device word per device; calls
+ * are serialised inside the library (each clears the word, runs the check and
+ * reads the word back before the next may start), so concurrent calls from
+ * several threads or streams each get their own array's verdict.
  */
 int gpt_attn_check_doc_offsets(const int32_t* doc_offsets, int B, int T, void* stream);
 

@@ -188,3 +188,18 @@ def test_binding_rejects_host_tensors(lib):
     q = torch.zeros(1, 1, 8, 32, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         abi.gpt_attn_fwd(q, q, q, q, torch.zeros(1, 1, 8), 0.1)
+
+
+def test_binding_rejects_tensors_off_the_current_device(monkeypatch):
+    """The library launches on the current CUDA device: the binding refuses tensors on another
+    device (and a stream of another device) before any pointer reaches the C ABI."""
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="current CUDA device"):
+        abi._stream(None, torch.device("cuda", 1))
+
+    class FakeStream:  # what the binding reads of a torch.cuda.Stream
+        cuda_stream = 0x1234
+        device = torch.device("cuda", 1)
+
+    with pytest.raises(ValueError, match="stream belongs to"):
+        abi._stream(FakeStream(), torch.device("cuda", 0))

@@ -96,13 +96,24 @@ def test_prologue_reference_arm_under_torchrun_prints_once():
     assert rec["config"]["T"] == 2048 and rec["e2e"]["h2d_bytes_per_step"] == 0
 
 
-def test_sampled_steps_cover_the_timed_loop():
+def test_profile_phase_samples_never_follow_a_synchronize():
+    """The per-kernel events sit in steps the host has run ahead of (never the first step of
+    the phase), and there are enough of them to average."""
     sys.path.insert(0, ROOT)
     import bench
-    for steps in (1, 7, 8, 9, 2000):
-        n = bench.sampled_steps(steps)
-        sampled = [i for i in range(steps) if i % bench.EVENT_EVERY == 0]
-        assert n == len(sampled) and n >= 1
+    idx = bench.sampled_indices(bench.PROFILE_STEPS)
+    assert 0 not in idx and len(idx) >= 10
+    assert bench.sampled_steps(bench.PROFILE_STEPS) == len(idx)
+    assert all(b - a == bench.EVENT_EVERY for a, b in zip(idx, idx[1:]))
+
+
+def test_kernel_sum_check_flags_mismatch():
+    sys.path.insert(0, ROOT)
+    import bench
+    ratio, warn = bench.kernel_sum_check([0.1, 0.02, 0.15, 0.1], 0.372)
+    assert abs(ratio - 0.37 / 0.372) < 1e-12 and warn is None
+    ratio, warn = bench.kernel_sum_check([0.1477, 0.0205, 0.1481, 0.1105], 0.3721)
+    assert ratio > 1.03 and "not trusted" in warn
 
 
 def test_recorded_traffic_only_for_matching_sources(tmp_path):

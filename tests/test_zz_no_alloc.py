@@ -29,10 +29,18 @@ def test_static_workspace_backward_matches(name, cuda_device):
     q, k, v, do, doc = (t.to(cuda_device) if t is not None else None for t in inputs.make_workload(w))
     o, lse = abi.attention_forward(q, k, v, w.scale, doc)
     ref = abi.attention_backward(q, k, v, o, lse, do, w.scale, doc)
-    for _ in range(2):
+    for call in range(2):
         got = [torch.full_like(q, float("nan")) for _ in range(3)]
+        torch.cuda.synchronize()
+        allocs0 = torch.cuda.memory_stats().get("allocation.all.allocated", 0)
+        free0 = torch.cuda.mem_get_info()[0]
         abi.gpt_attn_bwd_static_ws(q, k, v, o, do, lse, *got, w.scale, doc)
         torch.cuda.synchronize()
+        if call == 1:
+            # the first library call on a device may load the library's device code (and with it
+            # the scratch array); from then on a call allocates nothing, through torch or not
+            assert torch.cuda.memory_stats().get("allocation.all.allocated", 0) == allocs0
+            assert torch.cuda.mem_get_info()[0] == free0
         for g, r in zip(got, ref):
             assert torch.isfinite(g).all()
             assert rel_l2(g, r) <= GRAD_TOL
