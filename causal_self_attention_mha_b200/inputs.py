@@ -19,6 +19,8 @@ Recipe: torch.Generator('cpu').manual_seed(seed); fp32 randn for Q, K, V, dO in
 that order, each rounded to bf16 (round-to-nearest-even).  Document lengths for
 the packed workload come from random.Random(seed): per row, randint(64, 1024)
 (inclusive) repeatedly until the row is full; the last document is cut to fit T.
+FP8 (e4m3) inputs of a workload: Q, K, V drawn the same way from seed + 100, times 32,
+rounded to e4m3 (descale factor 1/32 each).
 """
 from __future__ import annotations
 
@@ -69,6 +71,32 @@ def make_qkvdo(B: int, H: int, T: int, d: int, seed: int):
     for _ in range(4):
         out.append(torch.randn(B, H, T, d, generator=g, dtype=torch.float32).to(torch.bfloat16))
     return tuple(out)
+
+
+# FP8 (e4m3) inputs: the stored values are FP8_MULT times N(0,1) draws (max |x| ~ 6 * 32 = 192,
+# inside e4m3's +-448), so each tensor's descale factor is 1 / FP8_MULT, a power of two.
+FP8_MULT = 32.0
+FP8_DESCALE = 1.0 / FP8_MULT
+
+
+def make_qkv_e4m3(B: int, H: int, T: int, d: int, seed: int):
+    """Q, K, V as CPU e4m3 codes (uint8 tensors [B,H,T,d]): fp32 randn from one generator, in
+    that order, times FP8_MULT, rounded by torch's float8_e4m3fn conversion.  The real values
+    are FP8_DESCALE times the codes' values."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    out = []
+    for _ in range(3):
+        x = torch.randn(B, H, T, d, generator=g, dtype=torch.float32) * FP8_MULT
+        out.append(x.to(torch.float8_e4m3fn).view(torch.uint8))
+    return tuple(out)
+
+
+def make_fp8_workload(w: Workload):
+    """(q8, k8, v8, doc_start or None) for a named workload: the workload's shapes and document
+    layout, its seed + 100 for the e4m3 draws."""
+    q8, k8, v8 = make_qkv_e4m3(w.B, w.H, w.T, w.d, w.seed + 100)
+    doc = doc_start_from_lengths(doc_lengths(w.B, w.T, w.seed), w.T) if w.doc_packed else None
+    return q8, k8, v8, doc
 
 
 def make_decode(B: int, H: int, Tq: int, L: int, d: int, seed: int):

@@ -220,3 +220,156 @@ def qk_prologue_backward(x, dz, base: float = 10000.0, gain: float = 1.2, eps: f
     s = np.sum(u * dz, axis=-1, keepdims=True)
     du = (gain / r) * (dz - u * s / (d * r * r))
     return _rope(du, cos, sin, inverse=True)
+
+
+# ------------------------------------------------------ FP8 (e4m3) attention forward
+# "How to build an LLM by hand" (agmtopy.github.io), section 5, item 4: the in-house FP8
+# training runs the forward matmuls with e4m3 operands through torch._scaled_mm (per-tensor
+# scales, higher-precision accumulation); the page lists the missing dynamic scaling as a
+# shortcoming, so scales are fixed per tensor.  Reading for the attention forward: Q, K and
+# V arrive as e4m3 codes with one fp32 descale factor each (x = descale * x8); the scores
+# are scale * (dq * dk) * Q8 K8^T, the softmax is exact, and the left operand of the second
+# product -- the attention weights -- is itself quantised to e4m3.  The weights are taken
+# relative to the row maximum (so they lie in (0, 1]) and multiplied by 2^8 before rounding,
+# so that the largest weight sits well inside e4m3's range (max 448) and weights down to
+# 2^-14 of the maximum stay normal numbers; the weighted sum is normalised by the sum of the
+# quantised weights.  The e4m3 format is the OCP 8-bit floating point "E4M3" (bias 7, no
+# infinities, S.1111.111 is NaN, largest finite 448, smallest subnormal 2^-9); rounding to it
+# is round-to-nearest-even with saturation at +-448.
+#
+# The reference output is the exact attention of the dequantised inputs (fp64).  What the
+# quantised weights may change is bounded row by row: with r_j = exp(s_j - max_k s_k) and a
+# weight error |q_j - r_j| <= e_j,
+#     O - o = sum_j (q_j - r_j)(v_j - o) / sum_j q_j,
+# so |O_c - o_c| <= sum_j e_j |v_jc - o_c| / (sum_j r_j - sum_j e_j).  Rounding 2^8 r_j c
+# (c >= 1 when the weights are taken relative to a running maximum that later grew) to e4m3
+# leaves e_j = 2^-4 r_j (normal range, half an ulp of 3 mantissa bits) or 2^-10 / 2^8 / c
+# <= 2^-18 (subnormal range, half the 2^-9 spacing); the bound uses their sum plus 2^-14 r_j
+# for the fp32 evaluation of the exponential before rounding.
+
+E4M3_MAX = 448.0
+FP8_P_SCALE = 256.0  # weights relative to the row maximum are multiplied by 2^8 before rounding
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of e4m3 codes (uint8): sign, 4 exponent bits (bias 7), 3 mantissa bits;
+    exponent field 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return sign * mag
+
+
+_E4M3_POS = None  # the 127 finite non-negative e4m3 values, ascending, and their codes
+
+
+def _e4m3_table():
+    global _E4M3_POS
+    if _E4M3_POS is None:
+        codes = np.arange(0x7F, dtype=np.uint8)  # 0x00 .. 0x7E: +0 .. 448
+        _E4M3_POS = (e4m3_decode(codes), codes)
+    return _E4M3_POS
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest e4m3 code to each float (ties to the even code, i.e. the even mantissa),
+    saturating to +-448; NaN -> 0x7F."""
+    x = np.asarray(x, dtype=np.float64)
+    vals, codes = _e4m3_table()
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(vals, a, side="left"), 0, len(vals) - 1)  # first value >= a
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - vals[lo], vals[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (codes[hi] % 2 == 0))
+    idx = np.where(pick_hi, hi, lo)
+    out = codes[idx].astype(np.uint8)
+    out = np.where((x < 0) & (out != 0), out | 0x80, out)
+    out = np.where(np.signbit(x) & (out == 0), 0x80, out)  # -0 keeps its sign
+    return np.where(np.isnan(x), 0x7F, out).astype(np.uint8)
+
+
+def e4m3_round(x) -> np.ndarray:
+    """x rounded to the nearest e4m3 value (float64)."""
+    return e4m3_decode(e4m3_encode(x))
+
+
+def _codes(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().cpu()
+        if x.dtype != torch.uint8:
+            x = x.view(torch.uint8)
+        x = x.numpy()
+    return np.asarray(x, dtype=np.uint8)
+
+
+def fp8_dequantize(x8, descale: float) -> np.ndarray:
+    """descale * value of each e4m3 code (exact in fp64)."""
+    return float(descale) * e4m3_decode(_codes(x8))
+
+
+def fp8_weight_error_bound(r: np.ndarray) -> np.ndarray:
+    """Largest |q - r| of a weight r in (0, 1] (relative to the row maximum) after rounding
+    2^8 r c to e4m3 and dividing by 2^8 c, for any c >= 1."""
+    return (2.0 ** -4 + 2.0 ** -14) * r + 2.0 ** -18
+
+
+def fp8_attention_forward(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float,
+                          scale: float, doc_start=None, window=None):
+    """Reference of the FP8 attention forward: O [B,H,T,d] and LSE [B,H,T] (exact attention of
+    the dequantised e4m3 inputs, float64) and BOUND [B,H,T,d], the largest change that
+    quantising the weights to e4m3 can make to each element of O."""
+    q = fp8_dequantize(q8, descale_q)
+    k = fp8_dequantize(k8, descale_k)
+    v = fp8_dequantize(v8, descale_v)
+    B, H, T, d = q.shape
+    doc = _doc(doc_start, B, T)
+    o = np.empty_like(q)
+    lse = np.empty((B, H, T))
+    bound = np.empty_like(q)
+    for b in range(B):
+        for h in range(H):
+            ds = doc[b:b + 1] if doc is not None else None
+            ob, lb, pb = attention_forward(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1],
+                                           v[b:b + 1, h:h + 1], scale, ds, return_probs=True,
+                                           window=window)
+            o[b, h], lse[b, h] = ob[0, 0], lb[0, 0]
+            p = pb[0, 0]                               # [T, T], rows sum to 1, zeros masked
+            r = p / p.max(axis=1, keepdims=True)       # weights relative to the row maximum
+            e = np.where(p > 0, fp8_weight_error_bound(r), 0.0)
+            den = r.sum(axis=1) - e.sum(axis=1)        # lower bound on the quantised sum
+            vb = v[b, h]
+            for i0 in range(0, T, 256):                # sum_j e_ij |v_jc - o_ic|, row blocks
+                i1 = min(T, i0 + 256)
+                dev = np.abs(vb[None, :, :] - o[b, h, i0:i1, None, :])   # [rows, T, d]
+                bound[b, h, i0:i1] = np.einsum("ij,ijc->ic", e[i0:i1], dev)
+            bound[b, h] /= den[:, None]
+    return o, lse, bound
+
+
+def fp8_attention_simulated(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float,
+                            scale: float, doc_start=None, window=None, p_scale=FP8_P_SCALE):
+    """The quantised-weight forward of the reading above, evaluated in float64 with the weights
+    taken relative to the final row maximum: q_j = e4m3(p_scale * r_j) / p_scale,
+    O = sum_j q_j v_j / sum_j q_j.  (A device kernel that takes the weights relative to a
+    running maximum rounds at other points; its result obeys the same bound.)"""
+    q = fp8_dequantize(q8, descale_q)
+    k = fp8_dequantize(k8, descale_k)
+    v = fp8_dequantize(v8, descale_v)
+    B, H, T, d = q.shape
+    doc = _doc(doc_start, B, T)
+    o = np.empty_like(q)
+    for b in range(B):
+        for h in range(H):
+            ds = doc[b:b + 1] if doc is not None else None
+            _, _, pb = attention_forward(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1],
+                                         v[b:b + 1, h:h + 1], scale, ds, return_probs=True,
+                                         window=window)
+            p = pb[0, 0]
+            r = p / p.max(axis=1, keepdims=True)
+            qw = e4m3_round(p_scale * r) / p_scale
+            o[b, h] = (qw @ v[b, h]) / qw.sum(axis=1, keepdims=True)
+    return o

@@ -174,3 +174,79 @@ def test_unmutated_numpy_oracle_passes_every_pin(monkeypatch):
         monkeypatch.setattr(oracle, fn_name, fn)
     for fn, kw in PY_PIN_TESTS:
         fn(**kw)
+
+
+# ------------------------------------------------- the FP8 (e4m3) forward oracle (numpy)
+
+from tests import test_oracle_fp8 as fp8pins  # noqa: E402
+
+FP8_FUNCS = ("e4m3_decode", "_e4m3_table", "e4m3_encode", "e4m3_round", "fp8_dequantize",
+             "fp8_weight_error_bound", "fp8_attention_forward", "fp8_attention_simulated")
+
+FP8_MUTATIONS = {
+    "e4m3_exponent_bias_8": ("np.exp2(e.astype(np.float64) - 7)", "np.exp2(e.astype(np.float64) - 8)"),
+    "e4m3_subnormal_scale": ("m / 8.0 * 2.0 ** -6", "m / 8.0 * 2.0 ** -7"),
+    "e4m3_ties_away_from_zero": ("((d_hi == d_lo) & (codes[hi] % 2 == 0))", "(d_hi == d_lo)"),
+    "dequantize_ignores_descale": ("return float(descale) * e4m3_decode", "return e4m3_decode"),
+    "weights_not_scaled_before_rounding": ("qw = e4m3_round(p_scale * r) / p_scale", "qw = e4m3_round(r)"),
+    "weights_normalised_before_rounding": ("r = p / p.max(axis=1, keepdims=True)\n            qw",
+                                           "r = p\n            qw"),
+    "simulated_exact_sum": ("o[b, h] = (qw @ v[b, h]) / qw.sum(axis=1, keepdims=True)",
+                            "o[b, h] = (qw @ v[b, h]) / r.sum(axis=1, keepdims=True)"),
+    "bound_half_an_ulp_too_small": ("(2.0 ** -4 + 2.0 ** -14) * r", "(2.0 ** -5 + 2.0 ** -14) * r"),
+    "bound_deviation_from_zero": ("np.abs(vb[None, :, :] - o[b, h, i0:i1, None, :])",
+                                  "np.abs(vb[None, :, :] + 0 * o[b, h, i0:i1, None, :])"),
+}
+
+
+def _fp8_mutant(old, new):
+    src = open(PY_SRC).read()
+    tree = ast.parse(src.replace(old, new))
+    keep = [n for n in tree.body if isinstance(n, ast.FunctionDef) and n.name in FP8_FUNCS]
+    assert {n.name for n in keep} == set(FP8_FUNCS)
+    ns = dict(vars(oracle))
+    ns["_E4M3_POS"] = None
+    exec(compile(ast.Module(body=keep, type_ignores=[]), "mutant_oracle", "exec"), ns)
+    return ns
+
+
+def _fp8_pins():
+    out = []
+    for name in dir(fp8pins):
+        fn = getattr(fp8pins, name)
+        if name.startswith("test_") and callable(fn):
+            params = fn.__code__.co_varnames[:fn.__code__.co_argcount]
+            out.append((fn, {"seed": 10} if "seed" in params else {}))
+    return out
+
+
+def test_fp8_mutation_anchors_are_unique():
+    src = open(PY_SRC).read()
+    for name, (old, _) in FP8_MUTATIONS.items():
+        assert src.count(old) == 1, name
+
+
+@pytest.mark.parametrize("name", sorted(FP8_MUTATIONS))
+def test_planted_mistake_in_fp8_oracle_is_caught(name, monkeypatch):
+    old, new = FP8_MUTATIONS[name]
+    ns = _fp8_mutant(old, new)
+    for fn_name in FP8_FUNCS:
+        monkeypatch.setattr(oracle, fn_name, ns[fn_name])
+    monkeypatch.setattr(oracle, "_E4M3_POS", None)
+    caught = []
+    for fn, kw in _fp8_pins():
+        try:
+            with np.errstate(all="ignore"):
+                fn(**kw)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(fn.__name__)
+    assert caught, f"no pin caught the planted mistake {name!r}"
+
+
+def test_unmutated_fp8_oracle_passes_every_pin(monkeypatch):
+    ns = _fp8_mutant("def ", "def ")
+    for fn_name in FP8_FUNCS:
+        monkeypatch.setattr(oracle, fn_name, ns[fn_name])
+    monkeypatch.setattr(oracle, "_E4M3_POS", None)
+    for fn, kw in _fp8_pins():
+        fn(**kw)
