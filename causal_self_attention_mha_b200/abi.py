@@ -42,6 +42,7 @@ _f = ctypes.c_float
 SIGNATURES = {
     "gpt_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
+    "gpt_attn_fwd_fp8": ([_vp, _vp, _vp, _f, _f, _f, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_fwd_window": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _i, _vp], _i),
     "gpt_attn_bwd_window": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f,
                              _vp, _i, _vp], _i),
@@ -167,6 +168,49 @@ def gpt_attn_fwd(q, k, v, o, lse, scale: float, doc_offsets=None, stream=None) -
     _check("gpt_attn_fwd", load().gpt_attn_fwd(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, d,
         float(scale), _doc_ptr(doc_offsets, B, T, q), _stream(stream, q.device)))
+
+
+def _e4m3(name: str, t: torch.Tensor, ref: Optional[torch.Tensor] = None):
+    """A contiguous [B,H,T,d] CUDA tensor of e4m3 codes (torch.float8_e4m3fn or uint8)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise ValueError(f"{name} must hold e4m3 codes (float8_e4m3fn or uint8), got {t.dtype}")
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B,H,T,d] tensor")
+    if ref is not None and (t.shape != ref.shape or t.device != ref.device):
+        raise ValueError(f"{name} must match q8: {tuple(ref.shape)} on {ref.device}")
+    return tuple(t.shape)
+
+
+def gpt_attn_fwd_fp8(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float, o, lse,
+                     scale: float, doc_offsets=None, stream=None) -> None:
+    """FP8 forward: q8, k8, v8 e4m3 codes [B,H,T,d] standing for descale * code; o bf16
+    [B,H,T,d], lse fp32 [B,H,T]."""
+    B, H, T, d = _e4m3("q8", q8)
+    _e4m3("k8", k8, q8)
+    _e4m3("v8", v8, q8)
+    _bhtd("o", o)
+    if tuple(o.shape) != (B, H, T, d) or o.device != q8.device:
+        raise ValueError(f"o must be bf16 {(B, H, T, d)} on {q8.device}")
+    _side("lse", lse, (B, H, T), torch.float32, q8)
+    _check("gpt_attn_fwd_fp8", load().gpt_attn_fwd_fp8(
+        q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(descale_q), float(descale_k),
+        float(descale_v), o.data_ptr(), lse.data_ptr(), B, H, T, d, float(scale),
+        _doc_ptr(doc_offsets, B, T, q8), _stream(stream, q8.device)))
+
+
+def attention_forward_fp8(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float,
+                          scale: Optional[float] = None, doc_offsets=None, stream=None):
+    """Allocates O [B,H,T,d] bf16 and LSE [B,H,T] fp32 and runs gpt_attn_fwd_fp8."""
+    B, H, T, d = _e4m3("q8", q8)
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty(B, H, T, d, device=q8.device, dtype=torch.bfloat16)
+    lse = torch.empty(B, H, T, device=q8.device, dtype=torch.float32)
+    gpt_attn_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, scale, doc_offsets,
+                     stream)
+    return o, lse
 
 
 def gpt_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, delta_ws, scale: float, doc_offsets=None,

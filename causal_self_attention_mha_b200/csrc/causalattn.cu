@@ -16,6 +16,7 @@
 #include "bwd.cuh"
 #include "decode.cuh"
 #include "fwd.cuh"
+#include "fwd8.cuh"
 #include "prologue.cuh"
 
 namespace {
@@ -52,6 +53,9 @@ cudaError_t set_smem_attrs() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(ca::attn_bwd_dkdv_kernel<D>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DkdvLayout<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(ca::attn_fwd_fp8_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           ca::Fwd8Layout<D>::SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D, 1>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D, 1>::SMEM);
@@ -148,6 +152,24 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int T) {
   return r == CUDA_SUCCESS;
 }
 
+// A [B*H, T, d] tensor of e4m3 codes viewed as 3-D bytes (d innermost), boxes of (d, 128 rows,
+// 1 head) with a d-byte swizzle; rows past T read as zero.
+template <int D>
+bool make_map8(CUtensorMap* m, const void* base, int BH, int T) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)T * D};
+  cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)ca::kRows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : (D == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // A [B, L, H, d] bf16 KV cache (the layout of the pages' kv-cache call) viewed as 4-D
 // (d, H, L, B) with boxes of (swizzle width, 1 head, 128 rows, 1 batch); rows past L read
 // as zero.  The staged box has the same shared-memory image as make_map's tiles.
@@ -213,6 +235,37 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
   ca::attn_fwd_kernel<D><<<grid, ca::FwdLayout<D>::THREADS, ca::FwdLayout<D>::SMEM, st>>>(
       mq, mk, mv, mo, p);
+  return launch_status();
+}
+
+template <int D>
+int fwd8_impl(const void* q8, const void* k8, const void* v8, float dsq, float dsk, float dsv,
+              void* o, float* lse, int B, int H, int T, float scale, const int32_t* doc,
+              cudaStream_t st) {
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map8<D>(&mq, q8, BH, T) || !make_map8<D>(&mk, k8, BH, T) ||
+      !make_map8<D>(&mv, v8, BH, T) || !make_map<D>(&mo, o, BH, T))
+    return GPT_ATTN_ERR_LAUNCH;
+  ca::Fwd8Params p8;
+  ca::FwdParams& p = p8.f;
+  p.doc = doc;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.H = H;
+  p.T = T;
+  p.BH = BH;
+  p.n_qt = (T + ca::kRows - 1) / ca::kRows;
+  p.n_pairs = (p.n_qt + 1) / 2;
+  p.n_items = p.n_pairs * BH;
+  p.scale_log2 = (float)((double)scale * dsq * dsk * 1.4426950408889634);
+  p.window = T;
+  p.wait_limit_ns = kWaitLimitNs;
+  p8.descale_v = dsv;
+  const int sms = sm_count();
+  const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
+  ca::attn_fwd_fp8_kernel<D><<<grid, ca::Fwd8Layout<D>::THREADS, ca::Fwd8Layout<D>::SMEM, st>>>(
+      mq, mk, mv, mo, p8);
   return launch_status();
 }
 
@@ -396,7 +449,9 @@ const char* gpt_attn_strerror(int s) {
     case GPT_ATTN_ERR_NOT_IMPLEMENTED: return "not implemented";
     case GPT_ATTN_ERR_BAD_SCALE: return "scale must be finite and > 0";
     case GPT_ATTN_ERR_TOO_LARGE: return "tensor too large (B*H*T*d must be < 2^31)";
-    case GPT_ATTN_ERR_BAD_PARAM: return "rope_base must be finite and > 0, gain finite, eps finite and >= 0";
+    case GPT_ATTN_ERR_BAD_PARAM:
+      return "bad parameter: rope_base must be finite and > 0, gain finite, eps finite and >= 0; "
+             "FP8 descale factors finite and > 0";
     default: return "unknown status";
   }
 }
@@ -429,6 +484,36 @@ int gpt_attn_fwd_window(const void* q, const void* k, const void* v, void* o, fl
                         int H, int T, int d, float scale, const int32_t* doc_offsets, int window,
                         void* stream) {
   return fwd_entry(q, k, v, o, lse, B, H, T, d, scale, doc_offsets, window, stream);
+}
+
+int gpt_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, float descale_q,
+                     float descale_k, float descale_v, void* o, float* lse, int B, int H, int T,
+                     int d, float scale, const int32_t* doc_offsets, void* stream) {
+  if (!q8 || !k8 || !v8 || !o || !lse) return GPT_ATTN_ERR_NULL_PTR;
+  int s = common_checks(B, H, T, d);
+  if (s) return s;
+  if ((s = check_scale(scale))) return s;
+  for (float ds : {descale_q, descale_k, descale_v})
+    if (!std::isfinite(ds) || !(ds > 0.f)) return GPT_ATTN_ERR_BAD_PARAM;
+  // the combined score scale must stay a finite, non-zero fp32 number
+  const double sl = (double)scale * descale_q * descale_k;
+  if (!(sl > 1e-30) || !(sl < 1e30)) return GPT_ATTN_ERR_BAD_PARAM;
+  if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(doc_offsets, 4))
+    return GPT_ATTN_ERR_MISALIGNED;
+  if ((s = ensure_device())) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 32:
+      return fwd8_impl<32>(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, H, T, scale,
+                           doc_offsets, st);
+    case 64:
+      return fwd8_impl<64>(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, H, T, scale,
+                           doc_offsets, st);
+    default:
+      return fwd8_impl<128>(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, B, H, T, scale,
+                            doc_offsets, st);
+  }
 }
 
 int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B, int H, int T,

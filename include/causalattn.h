@@ -85,7 +85,7 @@ typedef enum {
   GPT_ATTN_ERR_NOT_IMPLEMENTED = 10,
   GPT_ATTN_ERR_BAD_SCALE = 11,            /* scale not finite or <= 0 */
   GPT_ATTN_ERR_TOO_LARGE = 12,            /* a tensor exceeds 2^31 - 1 elements */
-  GPT_ATTN_ERR_BAD_PARAM = 13             /* rope_base, gain or eps out of range */
+  GPT_ATTN_ERR_BAD_PARAM = 13             /* rope_base, gain, eps or an FP8 descale out of range */
 } gpt_attn_status;
 
 /*
@@ -123,6 +123,34 @@ int gpt_attn_bwd_window(const void* q, const void* k, const void* v, const void*
                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
                         float* delta_ws, int B, int H, int T, int d, float scale,
                         const int32_t* doc_offsets, int window, void* stream);
+
+/*
+ * FP8 (e4m3) forward.  "How to build an LLM by hand" (agmtopy.github.io),
+ * section 5, item 4: the in-house FP8 training runs the forward matmuls with
+ * e4m3 operands through torch._scaled_mm, one fixed scale per tensor (the page
+ * notes that dynamic scaling is missing).  Reading for this forward: q8, k8, v8
+ * hold e4m3 codes (OCP E4M3: bias 7, no infinities, largest finite 448) of
+ * layout [B,H,T,d], one byte per element, standing for descale_q * q8,
+ * descale_k * k8, descale_v * v8.  Both products of the attention take e4m3
+ * operands, so the attention weights are rounded to e4m3 too:
+ *     S  = scale * descale_q * descale_k * Q8 K8^T   (fp32 accumulation)
+ *     r  = exp(S - rowmax S)                          (masks as for gpt_attn_fwd)
+ *     W8 = e4m3(2^8 * r)                              (round to nearest even)
+ *     o  = descale_v * (W8 V8) / rowsum(W8)           (bf16 [B,H,T,d])
+ *     lse = rowmax S + log rowsum(r)                  (fp32 [B,H,T], natural log)
+ * The weights are rounded relative to each row's final maximum (the kernel
+ * makes two passes over the keys).  o therefore differs from the exact
+ * attention of the dequantised inputs by at most
+ *     sum_j e_j |v_j - o_exact| / (sum_j r_j - sum_j e_j),
+ *     e_j = (2^-4 + 2^-14) r_j + 2^-18,
+ * plus bf16 rounding of o.  Causal or document-causal (doc_offsets) masks; no
+ * window.  descale_q, descale_k, descale_v must be finite and > 0
+ * (GPT_ATTN_ERR_BAD_PARAM otherwise); q8, k8, v8 and o 16-byte aligned.
+ * Ownership, asynchrony and errors as for gpt_attn_fwd.
+ */
+int gpt_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, float descale_q,
+                     float descale_k, float descale_v, void* o, float* lse, int B, int H, int T,
+                     int d, float scale, const int32_t* doc_offsets, void* stream);
 
 /*
  * KV-cache decode.  Generation appends Tq new tokens to a cache of L keys and

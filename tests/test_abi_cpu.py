@@ -203,3 +203,20 @@ def test_binding_rejects_tensors_off_the_current_device(monkeypatch):
 
     with pytest.raises(ValueError, match="stream belongs to"):
         abi._stream(FakeStream(), torch.device("cuda", 0))
+
+
+def test_fp8_forward_argument_errors(lib):
+    def f8(q=P[0], k=P[1], v=P[2], dq=0.03, dk=0.03, dv=0.03, o=P[3], lse=P[4], B=1, H=2, T=64,
+           d=64, scale=0.125, doc=None):
+        return lib.gpt_attn_fwd_fp8(q, k, v, dq, dk, dv, o, lse, B, H, T, d, scale, doc, None)
+    for name in ("q", "k", "v", "o", "lse"):
+        assert f8(**{name: None}) == abi.GPT_ATTN_ERR_NULL_PTR, name
+    for name in ("dq", "dk", "dv"):
+        for bad in (0.0, -1.0, math.inf, math.nan):
+            assert f8(**{name: bad}) == abi.GPT_ATTN_ERR_BAD_PARAM, (name, bad)
+    assert f8(dq=1e-20, dk=1e-20) == abi.GPT_ATTN_ERR_BAD_PARAM  # combined scale underflows
+    assert f8(scale=0.0) == abi.GPT_ATTN_ERR_BAD_SCALE
+    assert f8(d=96) == abi.GPT_ATTN_ERR_UNSUPPORTED_HEAD_DIM
+    assert f8(T=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
+    assert f8(q=P[0] + 8) == abi.GPT_ATTN_ERR_MISALIGNED
+    assert f8(lse=P[4] + 2) == abi.GPT_ATTN_ERR_MISALIGNED
