@@ -614,6 +614,170 @@ def main_prologue(args):
         dist.destroy_process_group()
 
 
+FP8_METRIC = "causal attention FP8 (e4m3) forward TFLOP/s and % of B200 dense FP8 peak, 1 GPU"
+FP8_OVER_BF16 = 2.0  # nominal dense fp8 / bf16 tensor rate (4.5 / 2.25 PFLOP/s)
+
+
+def fp8_oracle_sample(w, data, n_heads: int):
+    """The FP8 oracle (exact attention of the dequantised inputs, the rounding bound and the
+    rounded-weight forward) on the first n_heads heads: (seconds, algorithmic flops)."""
+    import oracle
+    from causal_self_attention_mha_b200 import inputs
+    q8, k8, v8, doc = data
+    sel = [(i // w.H, i % w.H) for i in range(n_heads)]
+    t0 = time.perf_counter()
+    for b, h in sel:
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        ds = doc[b:b + 1] if doc is not None else None
+        oracle.fp8_attention_forward(sl(q8), sl(k8), sl(v8), inputs.FP8_DESCALE,
+                                     inputs.FP8_DESCALE, inputs.FP8_DESCALE, w.scale, ds)
+        oracle.fp8_attention_simulated(sl(q8), sl(k8), sl(v8), inputs.FP8_DESCALE,
+                                       inputs.FP8_DESCALE, inputs.FP8_DESCALE, w.scale, ds)
+    dt = time.perf_counter() - t0
+    pairs = sum(inputs.visible_pairs(1, 1, w.T, doc[b:b + 1] if doc is not None else None)
+                for b, _ in sel)
+    return dt, 4.0 * w.d * pairs
+
+
+def main_fp8(args):
+    """FP8 forward: one step = gpt_attn_fwd_fp8 over the workload (e4m3 Q, K, V resident)."""
+    import torch
+    from causal_self_attention_mha_b200 import inputs
+    w = inputs.FP8_WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    data = inputs.make_fp8_workload(w)
+    q8, k8, v8, doc = data
+    pairs = inputs.visible_pairs(w.B, w.H, w.T, doc)
+    step_flops = 4.0 * w.d * pairs
+    cfg = workload_config(w, "single GPU")
+    cfg["workload"] = f"FP8 forward, {cfg['workload']}; e4m3 Q, K, V (32 x N(0,1)), descale 1/32"
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cores = len(os.sched_getaffinity(0))
+        import oracle
+        oracle.set_threads(cores)
+        for _ in range(args.warmup):
+            fp8_oracle_sample(w, data, 1)
+        times, fl = [], 0.0
+        for _ in range(args.steps):
+            dt, fl = fp8_oracle_sample(w, data, 1)
+            times.append(dt)
+        value = fl * len(times) / sum(times) / 1e12
+        print(json.dumps({
+            "impl": "reference", "metric": FP8_METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic: seeded e4m3 Q, K, V", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"1 of {w.B * w.H} heads per step; CPU {cpu_model()}"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    import torch.distributed as dist
+    from causal_self_attention_mha_b200 import abi
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    qd, kd, vd = (t.to(dev) for t in (q8, k8, v8))
+    docd = doc.to(dev) if doc is not None else None
+    o = torch.empty(w.B, w.H, w.T, w.d, device=dev, dtype=torch.bfloat16)
+    lse = torch.empty(w.B, w.H, w.T, device=dev, dtype=torch.float32)
+    ds = inputs.FP8_DESCALE
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        abi.gpt_attn_fwd_fp8(qd, kd, vd, ds, ds, ds, o, lse, w.scale, docd, stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    sampler = ClockSampler(local)
+    time.sleep(0.5)
+    t_wall0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
+    (kernel_ms,) = profile_kernels(step, stream, 1, dev)
+    host_us = host_us_per_call(step, 1, dev)
+    status = abi.gpt_attn_device_status(clear=True)
+    # end to end: e4m3 Q, K, V in from pinned host memory, O and LSE back out, every step
+    hin = [t.pin_memory() for t in (q8, k8, v8)]
+    oh = torch.empty(w.B, w.H, w.T, w.d, dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty(w.B, w.H, w.T, dtype=torch.float32).pin_memory()
+
+    def host_step():
+        with torch.cuda.stream(stream):
+            for dst, src in zip((qd, kd, vd), hin):
+                dst.copy_(src, non_blocking=True)
+            step()
+            oh.copy_(o, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+    for _ in range(3):
+        host_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        host_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
+    if rank == 0:
+        pk = peaks()
+        capped = bool(clocks) and "sw_power_cap" in (clocks.get("reasons") or [])
+        kind = "burst" if (ms * args.steps < 2000.0 and not capped) else "sustained"
+        peak = FP8_OVER_BF16 * (pk["bf16"] if kind == "burst" else pk["bf16_sustained"])
+        achieved = step_flops / (kernel_ms * 1e-3) / 1e12
+        value = world * step_flops / (ms * 1e-3) / 1e12
+        cfg["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
+        line = {
+            "metric": FP8_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+            "data": "synthetic: seeded e4m3 Q, K, V", "config": cfg,
+            "pct_of_peak": 100.0 * (value / world) / peak, "peak_tflops": peak,
+            "kernel_ms": {"attn_fwd_fp8": kernel_ms}, "host_us_per_call": host_us,
+            "roofline": {"kernel": "attn_fwd_fp8", "bound": "tensor", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{pk['source']} ({kind} bf16 GEMM) x {FP8_OVER_BF16} "
+                                        "(nominal fp8/bf16 ratio)",
+                         "traffic": None},
+            "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": 3 * q8.numel(),
+                    "d2h_bytes_per_step": oh.numel() * 2 + lh.numel() * 4, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps, "clocks": clocks, "device_status": status,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            cores = len(os.sched_getaffinity(0))
+            import oracle
+            oracle.set_threads(cores)
+            dt, fl = fp8_oracle_sample(w, data, 2)
+            line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
+                                    "kind": "oracle", "seconds": dt,
+                                    "sample": f"2 of {w.B * w.H} heads; CPU {cpu_model()}"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     import torch
@@ -624,6 +788,9 @@ def main():
         return
     if args.workload in inputs.PROLOGUE_WORKLOADS:
         main_prologue(args)
+        return
+    if args.workload in inputs.FP8_WORKLOADS:
+        main_fp8(args)
         return
     w = inputs.WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))

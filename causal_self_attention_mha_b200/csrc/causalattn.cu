@@ -134,10 +134,49 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded descriptors are cached per host thread: a descriptor is a pure function of its kind,
+// head dim, base address and extents, which together form the key, so a hit is always valid
+// (also after the memory was freed and reallocated).  Small and round-robin: a training step
+// touches about a dozen distinct tensors.
+struct MapKey {
+  const void* base;
+  int kind, d, e0, e1, e2;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && kind == o.kind && d == o.d && e0 == o.e0 && e1 == o.e1 && e2 == o.e2;
+  }
+};
+constexpr int kMapCache = 32;
+struct MapCache {
+  MapKey key[kMapCache];
+  CUtensorMap map[kMapCache];
+  bool used[kMapCache] = {};
+  int next = 0;
+};
+thread_local MapCache t_maps;
+
+template <class F>
+bool cached_map(CUtensorMap* m, const MapKey& k, F encode) {
+  MapCache& c = t_maps;
+  for (int i = 0; i < kMapCache; ++i)
+    if (c.used[i] && c.key[i] == k) {
+      *m = c.map[i];
+      return true;
+    }
+  if (!encode(m)) return false;
+  const int i = c.next;
+  c.next = (c.next + 1) % kMapCache;
+  c.key[i] = k;
+  c.map[i] = *m;
+  c.used[i] = true;
+  return true;
+}
+
+enum MapKind { kMapBf16 = 1, kMapE4m3 = 2, kMapCacheKV = 3 };
+
 // A [B*H, T, d] bf16 tensor viewed as 3-D (d innermost), boxes of
 // (swizzle width, 128 rows, 1 head); rows past T read as zero.
 template <int D>
-bool make_map(CUtensorMap* m, const void* base, int BH, int T) {
+bool encode_map(CUtensorMap* m, const void* base, int BH, int T) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   using Tl = ca::Tile<D>;
@@ -152,10 +191,16 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int T) {
   return r == CUDA_SUCCESS;
 }
 
+template <int D>
+bool make_map(CUtensorMap* m, const void* base, int BH, int T) {
+  return cached_map(m, MapKey{base, kMapBf16, D, BH, T, 0},
+                    [&](CUtensorMap* out) { return encode_map<D>(out, base, BH, T); });
+}
+
 // A [B*H, T, d] tensor of e4m3 codes viewed as 3-D bytes (d innermost), boxes of (d, 128 rows,
 // 1 head) with a d-byte swizzle; rows past T read as zero.
 template <int D>
-bool make_map8(CUtensorMap* m, const void* base, int BH, int T) {
+bool encode_map8(CUtensorMap* m, const void* base, int BH, int T) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
@@ -170,11 +215,17 @@ bool make_map8(CUtensorMap* m, const void* base, int BH, int T) {
   return r == CUDA_SUCCESS;
 }
 
+template <int D>
+bool make_map8(CUtensorMap* m, const void* base, int BH, int T) {
+  return cached_map(m, MapKey{base, kMapE4m3, D, BH, T, 0},
+                    [&](CUtensorMap* out) { return encode_map8<D>(out, base, BH, T); });
+}
+
 // A [B, L, H, d] bf16 KV cache (the layout of the pages' kv-cache call) viewed as 4-D
 // (d, H, L, B) with boxes of (swizzle width, 1 head, 128 rows, 1 batch); rows past L read
 // as zero.  The staged box has the same shared-memory image as make_map's tiles.
 template <int D>
-bool make_cache_map(CUtensorMap* m, const void* base, int B, int L, int H) {
+bool encode_cache_map(CUtensorMap* m, const void* base, int B, int L, int H) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   using Tl = ca::Tile<D>;
@@ -187,6 +238,12 @@ bool make_cache_map(CUtensorMap* m, const void* base, int B, int L, int H) {
                    Tl::SW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+template <int D>
+bool make_cache_map(CUtensorMap* m, const void* base, int B, int L, int H) {
+  return cached_map(m, MapKey{base, kMapCacheKV, D, B, L, H},
+                    [&](CUtensorMap* out) { return encode_cache_map<D>(out, base, B, L, H); });
 }
 
 int sm_count() {

@@ -99,6 +99,10 @@ def make_fp8_workload(w: Workload):
     return q8, k8, v8, doc
 
 
+# FP8 forward workloads (bench.py --workload fp8_<name>): the attention workloads' shapes.
+FP8_WORKLOADS = {f"fp8_{name}": w for name, w in WORKLOADS.items()}
+
+
 def make_decode(B: int, H: int, Tq: int, L: int, d: int, seed: int):
     """KV-cache decode inputs as CPU bf16 tensors: q [B,Tq,H,d], then the K and V caches
     [B,L,H,d], drawn in that order from one generator."""
