@@ -12,6 +12,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import threading
 from typing import Optional
 
 import torch
@@ -54,6 +55,8 @@ SIGNATURES = {
     "gpt_attn_bwd_preprocess": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "gpt_attn_bwd_dkdv": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_bwd_dq": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
+    "gpt_attn_bwd_dq_delta": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp],
+                              _i),
     "gpt_attn_bwd_static_ws": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp], _i),
     "gpt_attn_check_doc_offsets": ([_vp, _i, _i, _vp], _i),
     "gpt_attn_device_status": ([ctypes.POINTER(ctypes.c_uint), _i], _i),
@@ -78,9 +81,15 @@ class AttnError(RuntimeError):
         super().__init__(f"{fn} failed: status {status} ({strerror(status)}{detail})")
 
 
+_tls = threading.local()  # prepare(): a per-thread recorder that stands in for the library
+
+
 def load(path: Optional[str] = None) -> ctypes.CDLL:
     """Load libcausalattn.so (raises if it is missing: there is no fallback)."""
     global _lib
+    rec = getattr(_tls, "recorder", None)
+    if rec is not None and path is None:
+        return rec
     if _lib is None or path is not None:
         p = path or LIB_PATH
         if not os.path.exists(p):
@@ -300,6 +309,20 @@ def gpt_attn_bwd_dq(q, k, v, dout, lse, delta, dq, scale: float, doc_offsets=Non
         dq.data_ptr(), B, H, T, d, float(scale), _doc_ptr(doc_offsets, B, T, q), _stream(stream, q.device)))
 
 
+def gpt_attn_bwd_dq_delta(q, k, v, o, dout, lse, delta_out, dq, scale: float, doc_offsets=None,
+                          stream=None) -> None:
+    """dQ, computing delta = rowsum(dout * o) on the way into delta_out (for gpt_attn_bwd_dkdv)."""
+    B, H, T, d = _bhtd("q", q)
+    for name, t in (("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq)):
+        _bhtd(name, t, q)
+    _side("lse", lse, (B, H, T), torch.float32, q)
+    _side("delta_out", delta_out, (B, H, T), torch.float32, q)
+    _check("gpt_attn_bwd_dq_delta", load().gpt_attn_bwd_dq_delta(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+        delta_out.data_ptr(), dq.data_ptr(), B, H, T, d, float(scale),
+        _doc_ptr(doc_offsets, B, T, q), _stream(stream, q.device)))
+
+
 def gpt_attn_decode_workspace_size(B: int, H: int, Tq: int, L: int, d: int) -> int:
     return int(load().gpt_attn_decode_workspace_size(B, H, Tq, L, d))
 
@@ -346,6 +369,61 @@ def gpt_attn_device_status(clear: bool = False) -> int:
 def gpt_attn_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
     """Runs the bounded-wait self-test; returns the raw status (DEVICE_TIMEOUT expected)."""
     return int(load().gpt_attn_selftest_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+# ------------------------------------------------------------ prepared calls
+
+class PreparedCall:
+    """One library call whose arguments were checked and marshalled once: calling it re-issues
+    the C call with the same device pointers, sizes and stream (a few microseconds of host time
+    instead of the binding's per-call checks).  The tensors must stay alive and unmoved (they
+    are referenced here); their contents may change between calls."""
+
+    def __init__(self, name: str, args, keep):
+        self._fn = getattr(load(), name)
+        self._name = name
+        # converted to ctypes values once, so a call does not convert Python numbers again
+        self._args = tuple(t(a) if a is not None else None
+                           for t, a in zip(SIGNATURES[name][0], args))
+        self._keep = keep  # the tensors whose pointers are in _args
+
+    def __call__(self) -> None:
+        st = self._fn(*self._args)
+        if st:
+            raise AttnError(self._name, st)
+
+
+def _capture(fn, *a, **kw):
+    """Runs fn's checks and argument marshalling without calling the library: returns the
+    (name, args) it would pass to the C function."""
+    captured = {}
+
+    class _Recorder:
+        def __getattr__(self, name):
+            def rec(*args):
+                if "call" in captured:
+                    raise ValueError("prepare() needs a function that makes one library call")
+                captured["call"] = (name, args)
+                return GPT_ATTN_OK
+            return rec
+    load()  # the real library must be there: a prepared call will use it
+    _tls.recorder = _Recorder()
+    try:
+        fn(*a, **kw)
+    finally:
+        _tls.recorder = None
+    if "call" not in captured:
+        raise ValueError("prepare() needs a function that makes one library call")
+    return captured["call"]
+
+
+def prepare(fn, *args, **kwargs) -> PreparedCall:
+    """prepare(gpt_attn_fwd, q, k, v, o, lse, scale, ...) -> a PreparedCall re-issuing that call.
+    Works for every binding function that makes exactly one library call."""
+    name, cargs = _capture(fn, *args, **kwargs)
+    keep = [x for x in args if isinstance(x, torch.Tensor)]
+    keep += [x for x in kwargs.values() if isinstance(x, torch.Tensor)]
+    return PreparedCall(name, cargs, keep)
 
 
 # ------------------------------------------------------------ conveniences

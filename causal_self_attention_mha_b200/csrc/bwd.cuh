@@ -66,6 +66,7 @@ struct BwdParams {
   const int32_t* doc;     // [B, T] or nullptr
   const float* lse;       // [B, H, T] natural log
   const float* delta;     // [B, H, T]
+  float* delta_out;       // dq kernel with delta fused: where it writes delta [B, H, T]
   __nv_bfloat16* g0;      // dK (dkdv kernel) or dQ (dq kernel)   [B, H, T, D]
   __nv_bfloat16* g1;      // dV (dkdv kernel) or unused
   int H, T, BH, n_t;      // n_t = number of 128-row tiles along T
@@ -629,18 +630,44 @@ struct DqLayout {
   static constexpr int DO_OFF = Q_OFF + Tile<D>::BYTES;
   static constexpr int K_OFF = DO_OFF + Tile<D>::BYTES;           // + s * BYTES
   static constexpr int V_OFF = K_OFF + STK * Tile<D>::BYTES;      // + s * BYTES
-  static constexpr int BAR_OFF = V_OFF + STV * Tile<D>::BYTES;
+  static constexpr int DPART_OFF = V_OFF + STV * Tile<D>::BYTES;  // [2][128] partial deltas
+  static constexpr int BAR_OFF = DPART_OFF + 2 * kRows * 4;
   // barriers: qdo_full qdo_empty | k_full[STK] k_empty[STK] | v_full[STV] v_empty[STV] |
-  //           s_full[2] dp_full dp_read ds_full | acc_done acc_free drain | stg_full stg_free
-  static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 5 + 3 + 2;
+  //           s_full[2] dp_full dp_read ds_full | acc_done acc_free drain | stg_full stg_free |
+  //           dpart_full
+  static constexpr int NBAR = 2 + 2 * STK + 2 * STV + 5 + 3 + 2 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
+  static_assert(SMEM <= kMaxDynSmem, "dQ shared-memory layout");
   static constexpr int COMPUTE_WARPS = 8;
   static constexpr int THREADS = 384;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 256, T_DQ = 384;
 };
+
+// Reads this thread's half of row r of a staged tile (columns [half*D/2, (half+1)*D/2), the
+// layout load_tile produces) and returns sum_c a_rc * b_rc over them, in fp32.
+template <int D>
+__device__ __forceinline__ float tile_half_row_dot(const uint8_t* a, const uint8_t* b, int r,
+                                                   int half) {
+  using Tl = Tile<D>;
+  float acc = 0.f;
+#pragma unroll
+  for (int u = 0; u < D / 16; ++u) {
+    const int col = half * (D / 2) + 8 * u;
+    const int ch = col / Tl::BOX_COLS, cu = (col % Tl::BOX_COLS) / 8;
+    const int phys = (Tl::SW == 128) ? (cu ^ (r & 7)) : (cu ^ ((r >> 1) & 3));
+    const int off = ch * Tl::CHUNK_BYTES + r * Tl::SW + phys * 16;
+    const uint4 x = *reinterpret_cast<const uint4*>(a + off);
+    const uint4 y = *reinterpret_cast<const uint4*>(b + off);
+    const uint32_t xv[4] = {x.x, x.y, x.z, x.w}, yv[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      acc += bf16_lo(xv[i]) * bf16_lo(yv[i]) + bf16_hi(xv[i]) * bf16_hi(yv[i]);
+  }
+  return acc;
+}
 
 struct DqItem {
   int qt, bh, b, q0, kv_lo, n;  // query tile, head, batch, first row, key tiles [kv_lo, kv_lo+n)
@@ -665,16 +692,24 @@ __device__ __forceinline__ DqItem dq_item(const BwdParams& p, int w) {
   return I;
 }
 
-template <int D>
+// kDelta: the kernel also computes delta = rowsum(dO o O) for its query tile (O staged through
+// the K ring: one extra ring element at the start of every item), uses it, and writes it to
+// p.delta_out for the dK/dV kernel; otherwise it reads delta from p.delta.
+template <int D, bool kDelta>
 __global__ void __launch_bounds__(384, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmdO,
-                       const __grid_constant__ CUtensorMap tmdQ, const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmdQ,
+                       const __grid_constant__ CUtensorMap tmO, const BwdParams p) {
   using Tl = Tile<D>;
   using L = DqLayout<D>;
   constexpr int STK = L::STK, STV = L::STV;
+  // K-ring elements of item li: [O (kDelta)] [its n key tiles] [dQ staging]; with gk key tiles
+  // before the item, its first element is gk + li * PER_ITEM
+  constexpr int E = kDelta ? 1 : 0;
+  constexpr int PER_ITEM = 1 + E;
   constexpr int kProducerWarp = L::COMPUTE_WARPS, kMmaWarp = L::COMPUTE_WARPS + 1;
   constexpr int kStoreWarp = L::COMPUTE_WARPS + 2;
   extern __shared__ uint8_t smem_raw[];
@@ -696,6 +731,8 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t stg_full = xb + 56u;  // the staged dQ tile is complete
   const uint32_t stg_free = xb + 64u;  // ... and its store has read it
   const uint32_t dp_read = xb + 72u;   // dP(t) is in the element-wise warps' registers
+  const uint32_t dpart_full = xb + 80u;  // every warp's partial delta is in shared memory
+  float* dpart = reinterpret_cast<float*>(gsm + L::DPART_OFF);  // [2][128]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
 
@@ -707,7 +744,9 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(stg_full, L::COMPUTE_WARPS);
     mbar_init(stg_free, 1);
     mbar_init(qdo_full, 1);
-    mbar_init(qdo_empty, 1);
+    // Q / dO may be replaced once the item's last S / dP MMAs are done and, with the delta
+    // fused, once the element-wise warps have read dO for it
+    mbar_init(qdo_empty, kDelta ? 2 : 1);
     for (int s = 0; s < STK; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
@@ -724,6 +763,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(acc_done, 1);
     mbar_init(acc_free, L::COMPUTE_WARPS);
     mbar_init(drain, 1);
+    mbar_init(dpart_full, L::COMPUTE_WARPS);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -762,14 +802,15 @@ __global__ void __launch_bounds__(384, 1)
       const int NS = isK ? STK : STV;
       const CUtensorMap* tm = isK ? &tmK : &tmV;
       tma_prefetch_desc(tm);
+      if (kDelta && isK) tma_prefetch_desc(&tmO);
       int gk = 0;
       bool ok = true;
       for (int k_ = 0; ok && k_ * dw < p.n_items; ++k_) {
         const int w = snake_item(k_, w0, dw, p.n_items);
         if (w < 0) break;  // past the last item: no later round has one either
         const DqItem I = dq_item(p, w);
-        // the K ring carries one more element per item: the slot that stages dQ
-        const int n_el = isK ? I.n + 1 : I.n;
+        // the K ring carries PER_ITEM more elements per item: O (kDelta) and the dQ stage
+        const int n_el = isK ? I.n + PER_ITEM : I.n;
         for (int it = 0; it < n_el; ++it) {
           const int s = gk % NS, u = gk / NS;
           const uint32_t full = isK ? k_full(s) : v_full(s);
@@ -777,9 +818,13 @@ __global__ void __launch_bounds__(384, 1)
             ok = false;
             break;
           }
-          if (it < I.n) {
+          const int kt = isK ? it - E : it;  // key tile of this element
+          if (isK && kDelta && it == 0) {
             mbar_arrive_expect_tx(full, Tl::BYTES);
-            load_tile<D>(isK ? sK(s) : sV(s), tm, (I.kv_lo + it) * kRows, I.bh, full);
+            load_tile<D>(sK(s), &tmO, I.q0, I.bh, full);  // the item's O tile
+          } else if (kt < I.n) {
+            mbar_arrive_expect_tx(full, Tl::BYTES);
+            load_tile<D>(isK ? sK(s) : sV(s), tm, (I.kv_lo + kt) * kRows, I.bh, full);
           } else {
             mbar_arrive(full);  // hand the slot to the epilogue
           }
@@ -801,10 +846,12 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t kIdG = idesc_bf16_f32(128, D, true);     // dQ: N = d, B (K) is MN-major
       const uint32_t tDP = tmem + L::T_DP, tdQ = tmem + L::T_DQ;
       int li = 0, gk = 0;
-      // key tile t of item li is element t + li of the K ring (one staging slot per earlier item)
+      // key tile t (counted over all items) of item li is element t + li * PER_ITEM + E of the
+      // K ring (the extra elements of earlier items, and this item's O)
       auto issue_s = [&](int t) -> bool {  // S(t) = Q K_t^T into buffer t & 1
-        const int s = (t + li) % STK;
-        if (!wait_bounded(k_full(s), ((t + li) / STK) & 1, g, 3)) return false;
+        const int el = t + li * PER_ITEM + E;
+        const int s = el % STK;
+        if (!wait_bounded(k_full(s), (el / STK) & 1, g, 3)) return false;
         tc_fence_after();
         const uint32_t tS = tmem + L::T_S + 128u * (uint32_t)(t & 1);
 #pragma unroll
@@ -847,7 +894,7 @@ __global__ void __launch_bounds__(384, 1)
           if (it == 0 && li >= 1 && !wait_bounded(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
           if (!wait_bounded(ds_full, t & 1, g, 5)) { ok = false; break; }
           tc_fence_after();
-          const int s = (t + li) % STK;
+          const int s = (t + li * PER_ITEM + E) % STK;
           const uint32_t tdS = tmem + L::T_S + 128u * (uint32_t)(t & 1);  // dS(t) over S(t)
 #pragma unroll
           for (int kk = 0; kk < kRows / 16; ++kk)
@@ -876,7 +923,7 @@ __global__ void __launch_bounds__(384, 1)
         if (w < 0) break;  // past the last item: no later round has one either
         const DqItem I = dq_item(p, w);
         gk += I.n;
-        const int s = (gk + li) % STK;  // the item's staging slot
+        const int s = (gk + li * PER_ITEM + E) % STK;  // the item's staging slot
         if (!wait_bounded(stg_full, li & 1, g, 10)) break;
         store_tile<D>(&tmdQ, sK(s), I.q0, I.bh);
         bulk_commit();
@@ -906,7 +953,33 @@ __global__ void __launch_bounds__(384, 1)
       const int r = I.q0 + rl;  // query position owned by this thread
       // rows past T: -LSE = -inf makes every weight zero
       const float nlse2 = (r < T) ? -p.lse[(size_t)I.bh * T + r] * kLog2e : -INFINITY;
-      const float ndlt = (r < T) ? -p.delta[(size_t)I.bh * T + r] : 0.f;
+      float ndlt;
+      if (kDelta) {
+        // delta of my row from the staged O tile and dO: each of the two warps on these lanes
+        // sums half of the columns; both add the two halves in the same order
+        const int eo = gk + li * PER_ITEM;  // the item's O element of the K ring
+        if (!wait_bounded_warp(k_full(eo % STK), (eo / STK) & 1, g, 13) ||
+            !wait_bounded_warp(qdo_full, li & 1, g, 13)) {
+          ok = false;
+          break;
+        }
+        dpart[cs * kRows + rl] = tile_half_row_dot<D>(gsm + L::K_OFF + (eo % STK) * Tl::BYTES,
+                                                      gsm + L::DO_OFF, rl, cs);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dpart_full);
+        if (!wait_bounded_warp(dpart_full, li & 1, g, 13)) { ok = false; break; }
+        // every warp has read O and dO: O's slot goes back to the K ring, and dO may be
+        // replaced once the MMAs are done with it as well
+        if (warp == 0 && lane == 0) {
+          mbar_arrive(k_empty(eo % STK));
+          mbar_arrive(qdo_empty);
+        }
+        const float dlt = dpart[rl] + dpart[kRows + rl];
+        if (cs == 0 && r < T) p.delta_out[(size_t)I.bh * T + r] = dlt;
+        ndlt = (r < T) ? -dlt : 0.f;
+      } else {
+        ndlt = (r < T) ? -p.delta[(size_t)I.bh * T + r] : 0.f;
+      }
       // first visible key of this row: its document start or the window's start
       int ds = p.doc ? p.doc[(size_t)I.b * T + (r < T ? r : T - 1)] : 0;
       ds = ds > r - p.window + 1 ? ds : r - p.window + 1;
@@ -980,7 +1053,7 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) mbar_arrive(acc_free);
         // the K-ring slot after this item's key tiles stages the tile, once the
         // producer has handed it over and the previous item's store has been read
-        const int ks = gk + li;
+        const int ks = gk + li * PER_ITEM + E;
         if (!wait_bounded_warp(k_full(ks % STK), (ks / STK) & 1, g, 11) ||
             (li > 0 && !wait_bounded_warp(stg_free, (li - 1) & 1, g, 12))) {
           ok = false;

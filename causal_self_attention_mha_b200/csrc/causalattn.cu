@@ -9,6 +9,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <cstdio>
 #include <cstdint>
 #include <mutex>
 
@@ -66,7 +67,10 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D, 16>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D, 16>::SMEM);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(ca::attn_bwd_dq_kernel<D>,
+  e = cudaFuncSetAttribute(ca::attn_bwd_dq_kernel<D, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DqLayout<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(ca::attn_bwd_dq_kernel<D, false>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DqLayout<D>::SMEM);
 }
 
@@ -80,6 +84,18 @@ int ensure_device() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return GPT_ATTN_ERR_NO_DEVICE;
+  }
+  // The runtime binds a device's primary context to a host thread lazily; descriptor encoding
+  // (a driver call) needs it bound, and the first library call on a thread (torch's autograd
+  // engine calls the backward from a worker thread of its own) may come before anything else
+  // has bound it.  cudaSetDevice binds it; once per thread and device.
+  thread_local int t_bound_dev = -1;
+  if (t_bound_dev != dev) {
+    if (cudaSetDevice(dev) != cudaSuccess) {
+      cudaGetLastError();
+      return GPT_ATTN_ERR_NO_DEVICE;
+    }
+    t_bound_dev = dev;
   }
   int st = g_dev_state[dev].load(std::memory_order_acquire);
   if (st == 0) {
@@ -134,10 +150,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Encoded descriptors are cached per host thread: a descriptor is a pure function of its kind,
-// head dim, base address and extents, which together form the key, so a hit is always valid
-// (also after the memory was freed and reallocated).  Small and round-robin: a training step
-// touches about a dozen distinct tensors.
+// Encoded descriptors are cached: a descriptor is a pure function of its kind, head dim, base
+// address and extents, which together form the key, so a hit is always valid (also after the
+// memory was freed and reallocated).  Small and round-robin (a training step touches about a
+// dozen distinct tensors); one cache for all host threads, under a mutex.
 struct MapKey {
   const void* base;
   int kind, d, e0, e1, e2;
@@ -149,14 +165,19 @@ constexpr int kMapCache = 32;
 struct MapCache {
   MapKey key[kMapCache];
   CUtensorMap map[kMapCache];
-  bool used[kMapCache] = {};
-  int next = 0;
+  bool used[kMapCache];
+  int next;
 };
-thread_local MapCache t_maps;
+MapCache g_maps;  // zero-initialised: no entry used
+std::mutex g_maps_mu;
+
+thread_local const char* t_last_cuda_error = "no error";
+thread_local char t_encode_error[96];
 
 template <class F>
 bool cached_map(CUtensorMap* m, const MapKey& k, F encode) {
-  MapCache& c = t_maps;
+  std::lock_guard<std::mutex> lock(g_maps_mu);
+  MapCache& c = g_maps;
   for (int i = 0; i < kMapCache; ++i)
     if (c.used[i] && c.key[i] == k) {
       *m = c.map[i];
@@ -173,12 +194,24 @@ bool cached_map(CUtensorMap* m, const MapKey& k, F encode) {
 
 enum MapKind { kMapBf16 = 1, kMapE4m3 = 2, kMapCacheKV = 3 };
 
+// True on success; otherwise records the driver's code for gpt_attn_last_cuda_error.
+bool encode_ok(CUresult r) {
+  if (r == CUDA_SUCCESS) return true;
+  snprintf(t_encode_error, sizeof(t_encode_error), "cuTensorMapEncodeTiled failed with CUresult %d",
+           (int)r);
+  t_last_cuda_error = t_encode_error;
+  return false;
+}
+
 // A [B*H, T, d] bf16 tensor viewed as 3-D (d innermost), boxes of
 // (swizzle width, 128 rows, 1 head); rows past T read as zero.
 template <int D>
 bool encode_map(CUtensorMap* m, const void* base, int BH, int T) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    t_last_cuda_error = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
   using Tl = ca::Tile<D>;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
@@ -188,7 +221,7 @@ bool encode_map(CUtensorMap* m, const void* base, int BH, int T) {
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    Tl::SW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_ok(r);
 }
 
 template <int D>
@@ -212,7 +245,7 @@ bool encode_map8(CUtensorMap* m, const void* base, int BH, int T) {
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_ok(r);
 }
 
 template <int D>
@@ -237,7 +270,7 @@ bool encode_cache_map(CUtensorMap* m, const void* base, int B, int L, int H) {
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    Tl::SW == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_ok(r);
 }
 
 template <int D>
@@ -251,8 +284,6 @@ int sm_count() {
   cudaGetDevice(&dev);
   return (dev >= 0 && dev < kMaxDevices && g_sm_count[dev] > 0) ? g_sm_count[dev] : 148;
 }
-
-thread_local const char* t_last_cuda_error = "no error";
 
 int launch_status() {
   cudaError_t e = cudaGetLastError();
@@ -338,10 +369,13 @@ int delta_impl(const void* o, const void* dout, float* delta, int B, int H, int 
   return launch_status();
 }
 
+// dkdv: the dK/dV kernel (g0 = dK, g1 = dV); otherwise the dQ kernel (g0 = dQ), which with
+// o != nullptr also computes delta from o and dout and writes it to delta_out.
 template <int D>
 int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const void* dout,
                    const float* lse, const float* delta, void* g0, void* g1, int B, int H, int T,
-                   float scale, const int32_t* doc, int window, cudaStream_t st) {
+                   float scale, const int32_t* doc, int window, cudaStream_t st,
+                   const void* o = nullptr, float* delta_out = nullptr) {
   const int BH = B * H;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map<D>(&mq, q, BH, T) || !make_map<D>(&mk, k, BH, T) || !make_map<D>(&mv, v, BH, T) ||
@@ -351,6 +385,7 @@ int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const
   p.doc = doc;
   p.lse = lse;
   p.delta = delta;
+  p.delta_out = delta_out;
   p.g0 = static_cast<__nv_bfloat16*>(g0);
   p.g1 = static_cast<__nv_bfloat16*>(g1);
   p.H = H;
@@ -366,15 +401,19 @@ int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const
   const int sms = sm_count();
   const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
   // outputs leave through TMA stores of whole tiles (rows past T are dropped)
-  CUtensorMap mg0, mg1;
-  if (!make_map<D>(&mg0, g0, BH, T) || (dkdv && !make_map<D>(&mg1, g1, BH, T)))
+  CUtensorMap mg0, mg1, mo;
+  if (!make_map<D>(&mg0, g0, BH, T) || (dkdv && !make_map<D>(&mg1, g1, BH, T)) ||
+      (o && !make_map<D>(&mo, o, BH, T)))
     return GPT_ATTN_ERR_LAUNCH;
   if (dkdv)
     ca::attn_bwd_dkdv_kernel<D><<<grid, ca::DkdvLayout<D>::THREADS, ca::DkdvLayout<D>::SMEM, st>>>(
         mq, mk, mv, mdo, mg0, mg1, p);
-  else
-    ca::attn_bwd_dq_kernel<D><<<grid, ca::DqLayout<D>::THREADS, ca::DqLayout<D>::SMEM, st>>>(
-        mq, mk, mv, mdo, mg0, p);
+  else if (o)
+    ca::attn_bwd_dq_kernel<D, true><<<grid, ca::DqLayout<D>::THREADS, ca::DqLayout<D>::SMEM, st>>>(
+        mq, mk, mv, mdo, mg0, mo, p);
+  else  // the O map is not read without the fused delta: any valid map will do
+    ca::attn_bwd_dq_kernel<D, false><<<grid, ca::DqLayout<D>::THREADS, ca::DqLayout<D>::SMEM, st>>>(
+        mq, mk, mv, mdo, mg0, mq, p);
   return launch_status();
 }
 
@@ -588,27 +627,33 @@ int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B
   }
 }
 
+// With o != nullptr (dQ step only) delta is not read but computed from o and dout and written
+// to delta_out; otherwise delta is an input.
 static int bwd_step(bool dkdv, const void* q, const void* k, const void* v, const void* dout,
                     const float* lse, const float* delta, void* g0, void* g1, int B, int H, int T,
-                    int d, float scale, const int32_t* doc, int window, void* stream) {
-  if (!q || !k || !v || !dout || !lse || !delta || !g0 || (dkdv && !g1))
+                    int d, float scale, const int32_t* doc, int window, void* stream,
+                    const void* o = nullptr, float* delta_out = nullptr) {
+  if (!q || !k || !v || !dout || !lse || !g0 || (dkdv && !g1) || (o ? !delta_out : !delta))
     return GPT_ATTN_ERR_NULL_PTR;
   int s = common_checks(B, H, T, d);
   if (s) return s;
   if ((s = check_scale(scale))) return s;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dout, 16) ||
       !aligned(g0, 16) || (dkdv && !aligned(g1, 16)) || !aligned(lse, 4) || !aligned(delta, 4) ||
-      !aligned(doc, 4))
+      !aligned(doc, 4) || !aligned(o, 16) || !aligned(delta_out, 4))
     return GPT_ATTN_ERR_MISALIGNED;
   if ((s = ensure_device())) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d) {
     case 32:
-      return bwd_tiled_impl<32>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, window, st);
+      return bwd_tiled_impl<32>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc,
+                                window, st, o, delta_out);
     case 64:
-      return bwd_tiled_impl<64>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, window, st);
+      return bwd_tiled_impl<64>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc,
+                                window, st, o, delta_out);
     default:
-      return bwd_tiled_impl<128>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc, window, st);
+      return bwd_tiled_impl<128>(dkdv, q, k, v, dout, lse, delta, g0, g1, B, H, T, scale, doc,
+                                 window, st, o, delta_out);
   }
 }
 
@@ -623,6 +668,15 @@ int gpt_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dou
                     float scale, const int32_t* doc_offsets, void* stream) {
   return bwd_step(false, q, k, v, dout, lse, delta, dq, nullptr, B, H, T, d, scale, doc_offsets, 0,
                   stream);
+}
+
+int gpt_attn_bwd_dq_delta(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, float* delta_out, void* dq, int B,
+                          int H, int T, int d, float scale, const int32_t* doc_offsets,
+                          void* stream) {
+  if (!o) return GPT_ATTN_ERR_NULL_PTR;
+  return bwd_step(false, q, k, v, dout, lse, nullptr, dq, nullptr, B, H, T, d, scale, doc_offsets,
+                  0, stream, o, delta_out);
 }
 
 static int bwd_entry(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -640,11 +694,11 @@ static int bwd_entry(const void* q, const void* k, const void* v, const void* o,
       !aligned(lse, 4) || !aligned(delta_ws, 4) || !aligned(doc_offsets, 4))
     return GPT_ATTN_ERR_MISALIGNED;
   if ((s = ensure_device())) return s;
-  if ((s = gpt_attn_bwd_preprocess(o, dout, delta_ws, B, H, T, d, stream))) return s;
-  if ((s = bwd_step(true, q, k, v, dout, lse, delta_ws, dk, dv, B, H, T, d, scale, doc_offsets,
-                    window, stream)))
+  // dQ first: it also computes delta (into delta_ws), which dK/dV then reads
+  if ((s = bwd_step(false, q, k, v, dout, lse, nullptr, dq, nullptr, B, H, T, d, scale,
+                    doc_offsets, window, stream, o, delta_ws)))
     return s;
-  return bwd_step(false, q, k, v, dout, lse, delta_ws, dq, nullptr, B, H, T, d, scale, doc_offsets,
+  return bwd_step(true, q, k, v, dout, lse, delta_ws, dk, dv, B, H, T, d, scale, doc_offsets,
                   window, stream);
 }
 
@@ -861,10 +915,11 @@ extern "C" int gpt_attn_bwd_static_ws(const void* q, const void* k, const void* 
   if ((s = ensure_device())) return s;
   float* delta = nullptr;
   if ((s = static_delta_ptr(&delta))) return s;
-  // delta is fully rewritten by the first step, so nothing needs clearing first
-  if ((s = gpt_attn_bwd_preprocess(o, dout, delta, B, H, T, d, stream))) return s;
-  if ((s = gpt_attn_bwd_dkdv(q, k, v, dout, lse, delta, dk, dv, B, H, T, d, scale, doc_offsets,
-                             stream)))
+  // delta is fully rewritten by the first step (dQ, which computes it), so nothing needs
+  // clearing first
+  if ((s = gpt_attn_bwd_dq_delta(q, k, v, o, dout, lse, delta, dq, B, H, T, d, scale, doc_offsets,
+                                 stream)))
     return s;
-  return gpt_attn_bwd_dq(q, k, v, dout, lse, delta, dq, B, H, T, d, scale, doc_offsets, stream);
+  return gpt_attn_bwd_dkdv(q, k, v, dout, lse, delta, dk, dv, B, H, T, d, scale, doc_offsets,
+                           stream);
 }

@@ -35,7 +35,8 @@
  * lse, delta: contiguous fp32 [B, H, T].
  *
  * Ownership.  Every pointer is caller-owned DEVICE memory on the current CUDA
- * device.  The library allocates no memory; it keeps no state besides
+ * device (its primary context, which the first call on each host thread binds
+ * to that thread if nothing has yet).  The library allocates no memory; it keeps no state besides
  * per-device attribute and occupancy caches, one device-side status word and
  * the fixed delta scratch of gpt_attn_bwd_static_ws.
  *
@@ -98,7 +99,8 @@ int gpt_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  * Backward.  Reads q, k, v, o, dout [B,H,T,d] and lse [B,H,T] (the forward's
  * outputs); writes dq, dk, dv [B,H,T,d].  delta_ws is a caller-provided fp32
  * [B,H,T] workspace that receives delta = rowsum(dout o o).  Equivalent to
- * gpt_attn_bwd_preprocess, then gpt_attn_bwd_dkdv, then gpt_attn_bwd_dq.
+ * gpt_attn_bwd_dq_delta (which computes delta into delta_ws), then
+ * gpt_attn_bwd_dkdv.
  */
 int gpt_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                  const float* lse, void* dq, void* dk, void* dv, float* delta_ws, int B, int H,
@@ -216,6 +218,17 @@ int gpt_attn_bwd_preprocess(const void* o, const void* dout, float* delta, int B
 int gpt_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
                       const float* lse, const float* delta, void* dk, void* dv, int B, int H,
                       int T, int d, float scale, const int32_t* doc_offsets, void* stream);
+
+/*
+ * Backward step 3, without a separate delta step: dq [B,H,T,d] from q, k, v,
+ * dout and lse, computing delta = rowsum(dout o o) from o and dout on the way
+ * and writing it to delta_out (fp32 [B,H,T]) for gpt_attn_bwd_dkdv.  Same
+ * result as gpt_attn_bwd_preprocess followed by gpt_attn_bwd_dq.
+ */
+int gpt_attn_bwd_dq_delta(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, float* delta_out, void* dq, int B,
+                          int H, int T, int d, float scale, const int32_t* doc_offsets,
+                          void* stream);
 
 /* Backward step 3: dq [B,H,T,d] from q, k, v, dout, lse and delta. */
 int gpt_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout,

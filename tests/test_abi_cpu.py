@@ -220,3 +220,43 @@ def test_fp8_forward_argument_errors(lib):
     assert f8(T=0) == abi.GPT_ATTN_ERR_BAD_SHAPE
     assert f8(q=P[0] + 8) == abi.GPT_ATTN_ERR_MISALIGNED
     assert f8(lse=P[4] + 2) == abi.GPT_ATTN_ERR_MISALIGNED
+
+
+def test_prepare_records_the_marshalled_call(lib, monkeypatch):
+    """prepare() runs the binding's checks and marshalling once, without calling the library,
+    and keeps exactly the arguments the binding would pass."""
+    calls = []
+
+    class FakeFn:
+        def __init__(self, name):
+            self.name = name
+
+        def __call__(self, *args):
+            calls.append((self.name, args))
+            return 0
+
+    class FakeLib:
+        def __getattr__(self, name):
+            return FakeFn(name)
+
+    def fake_fwd(q, scale, stream=None):  # a binding-shaped function: checks, then one call
+        if scale <= 0:
+            raise ValueError("scale")
+        abi._check("gpt_attn_fwd", abi.load().gpt_attn_fwd(
+            0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 1, 2, 64, 64, float(scale), None, 0))
+
+    pc = abi.prepare(fake_fwd, None, 0.125)
+    assert pc._name == "gpt_attn_fwd" and len(pc._args) == 12
+    assert pc._args[9].value == 0.125 and pc._args[10] is None
+    monkeypatch.setattr(pc, "_fn", FakeFn("gpt_attn_fwd"))
+    pc()
+    pc()
+    assert len(calls) == 2 and calls[0][1][9].value == 0.125
+    with pytest.raises(ValueError):
+        abi.prepare(fake_fwd, None, -1.0)  # the checks run at prepare time
+
+    def two_calls():
+        abi.load().gpt_attn_version()
+        abi.load().gpt_attn_version()
+    with pytest.raises(ValueError, match="one library call"):
+        abi.prepare(two_calls)

@@ -423,3 +423,82 @@ def test_prologue_autograd_then_attention(cuda_device):
     assert float(np.max(np.abs(o.detach().cpu().double().numpy() - o_r))) <= O_TOL
     for g, r in ((qd.grad, dq_r), (kd.grad, dk_r), (vd.grad, dv_r)):
         assert rel_l2(g.cpu().double().numpy(), r) <= GRAD_TOL
+
+
+# ----------------------------------------------- dQ with delta fused into it
+
+@pytest.mark.parametrize("T,d,with_doc", [(1, 32, False), (200, 64, True), (300, 128, False),
+                                          (1024, 128, True)])
+def test_dq_step_computes_delta(T, d, with_doc, cuda_device):
+    """gpt_attn_bwd_dq_delta writes delta = rowsum(dO * O) (checked in fp64 from the same bf16
+    O and dO) and gives the dQ of gpt_attn_bwd_preprocess + gpt_attn_bwd_dq up to the order of
+    the fp32 additions in delta."""
+    B, H = 2, 3
+    q, k, v, do = (t.to(cuda_device) for t in inputs.make_qkvdo(B, H, T, d, 800 + T + d))
+    doc = inputs.random_doc_start(B, T, 9 + T, 20, 200).to(cuda_device) if with_doc else None
+    scale = inputs.fp32_scale(d)
+    o, lse = abi.attention_forward(q, k, v, scale, doc)
+    delta_f = torch.full((B, H, T), float("nan"), device=cuda_device)
+    dq_f = torch.empty_like(q)
+    abi.gpt_attn_bwd_dq_delta(q, k, v, o, do, lse, delta_f, dq_f, scale, doc)
+    delta_s = torch.empty_like(delta_f)
+    dq_s = torch.empty_like(q)
+    abi.gpt_attn_bwd_preprocess(o, do, delta_s)
+    abi.gpt_attn_bwd_dq(q, k, v, do, lse, delta_s, dq_s, scale, doc)
+    torch.cuda.synchronize()
+    ref = (o.double() * do.double()).sum(-1)
+    mag = (o.double() * do.double()).abs().sum(-1)
+    assert torch.all((delta_f.double() - ref).abs() <= 1e-6 * mag + 1e-6)
+    assert rel_l2(dq_f.double().cpu().numpy(), dq_s.double().cpu().numpy()) <= 1e-3
+    no_device_timeouts()
+
+
+def test_prepared_calls_match_direct_calls(cuda_device):
+    """abi.prepare: the checked-once call re-issued gives bit-identical results."""
+    B, H, T, d = 2, 3, 333, 64
+    q, k, v, do = (t.to(cuda_device) for t in inputs.make_qkvdo(B, H, T, d, 901))
+    scale = inputs.fp32_scale(d)
+    o, lse = abi.attention_forward(q, k, v, scale)
+    o2, lse2 = torch.empty_like(o), torch.empty_like(lse)
+    fwd = abi.prepare(abi.gpt_attn_fwd, q, k, v, o2, lse2, scale)
+    dq, dk, dv = abi.attention_backward(q, k, v, o, lse, do, scale)
+    dq2, dk2, dv2 = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    delta = torch.empty_like(lse)
+    bwd = abi.prepare(abi.gpt_attn_bwd, q, k, v, o, do, lse, dq2, dk2, dv2, delta, scale)
+    for _ in range(2):
+        fwd()
+        bwd()
+        torch.cuda.synchronize()
+        assert torch.equal(o2, o) and torch.equal(lse2, lse)
+        assert torch.equal(dq2, dq) and torch.equal(dk2, dk) and torch.equal(dv2, dv)
+    no_device_timeouts()
+
+
+def test_calls_from_another_host_thread(cuda_device):
+    """Library calls from a second host thread (as torch's autograd engine makes them) give the
+    results of the same calls from the main thread, bit for bit."""
+    import threading
+    B, H, T, d = 1, 2, 200, 64
+    q, k, v, do = (t.to(cuda_device) for t in inputs.make_qkvdo(B, H, T, d, 902))
+    scale = inputs.fp32_scale(d)
+    o, lse = abi.attention_forward(q, k, v, scale)
+    ref = abi.attention_backward(q, k, v, o, lse, do, scale)
+    torch.cuda.synchronize()
+    out, err = {}, []
+
+    def work():
+        try:
+            torch.cuda.set_device(cuda_device)
+            o2, lse2 = abi.attention_forward(q, k, v, scale)
+            out["g"] = abi.attention_backward(q, k, v, o2, lse2, do, scale)
+            out["f"] = (o2, lse2)
+            torch.cuda.synchronize()
+        except Exception as e:  # reported on the main thread
+            err.append(e)
+    th = threading.Thread(target=work)
+    th.start()
+    th.join()
+    assert not err, err
+    assert torch.equal(out["f"][0], o) and torch.equal(out["f"][1], lse)
+    for a, b in zip(out["g"], ref):
+        assert torch.equal(a, b)
