@@ -286,11 +286,8 @@ __global__ void __launch_bounds__(384, 1)
         const int w = snake_item(k_, w0, dw, p.n_items);
         if (w < 0) break;  // past the last item: no later round has one either
         const FwdItem I = fwd_item(p, w);
-        for (int x = 0; x < 2; ++x) {
-          if (x == 1 && !I.hasB) continue;
-          if (!wait_bounded(q_full(x), nq[x] & 1, g, 2)) { ok = false; break; }
-          ++nq[x];
-        }
+        // each slot's Q is waited for right before its first S: B's Q can only be loaded once
+        // B's last S of the previous item has read the old one, a key tile later than A's
         for (int j = I.j_lo; ok && j <= I.j_hi; ++j, ++gk, ++gv) {
           const int sk = gk % STK;
           if (!wait_bounded(k_full(sk), (gk / STK) & 1, g, 3)) { ok = false; break; }
@@ -299,6 +296,10 @@ __global__ void __launch_bounds__(384, 1)
           auto step = [&](int x, bool act) -> bool {
             if (pend_t[x] >= 0 && !issue_pv(x)) return false;
             if (!act) return true;
+            if (j == I.lo[x]) {  // first S of this query tile: its Q must have landed
+              if (!wait_bounded(q_full(x), nq[x] & 1, g, 2)) return false;
+              ++nq[x];
+            }
             tc_fence_after();
             const uint32_t tS = tmem + 128u * x;
 #pragma unroll
