@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "fwd.cuh"
 #include "fwd8.cuh"
+#include "fwd_pair.cuh"
 #include "prologue.cuh"
 
 namespace {
@@ -45,6 +46,27 @@ int check_scale(float scale) {
 std::mutex g_mu;
 std::atomic<int> g_dev_state[kMaxDevices];  // 0 unknown, 1 ready, 2 wrong arch, 3 setup failed
 int g_sm_count[kMaxDevices];                // multiprocessors per device (persistent grids)
+int g_pair_clusters[kMaxDevices];           // co-resident CTA pairs of the pair forward kernel
+
+// Shared-memory opt-in of the CTA-pair forward kernel and how many of its pairs fit at once.
+cudaError_t setup_pair_kernel(int dev) {
+  cudaError_t e = cudaFuncSetAttribute(ca::attn_fwd_pair_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       ca::PairLayout::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (unsigned)(g_sm_count[dev] / 2));
+  cfg.blockDim = dim3(ca::PairLayout::THREADS);
+  cfg.dynamicSmemBytes = ca::PairLayout::SMEM;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (void*)ca::attn_fwd_pair_kernel, &cfg) != cudaSuccess ||
+      n < 1) {
+    cudaGetLastError();
+    n = g_sm_count[dev] / 2;
+  }
+  g_pair_clusters[dev] = n;
+  return cudaSuccess;
+}
 
 template <int D>
 cudaError_t set_smem_attrs() {
@@ -114,7 +136,7 @@ int ensure_device() {
       if (major != 10 || minor != 0) {
         st = 2;
       } else if (set_smem_attrs<32>() != cudaSuccess || set_smem_attrs<64>() != cudaSuccess ||
-                 set_smem_attrs<128>() != cudaSuccess) {
+                 set_smem_attrs<128>() != cudaSuccess || setup_pair_kernel(dev) != cudaSuccess) {
         cudaGetLastError();
         st = 3;
       } else {
@@ -192,7 +214,7 @@ bool cached_map(CUtensorMap* m, const MapKey& k, F encode) {
   return true;
 }
 
-enum MapKind { kMapBf16 = 1, kMapE4m3 = 2, kMapCacheKV = 3 };
+enum MapKind { kMapBf16 = 1, kMapE4m3 = 2, kMapCacheKV = 3, kMapBf16Half = 4 };
 
 // True on success; otherwise records the driver's code for gpt_attn_last_cuda_error.
 bool encode_ok(CUresult r) {
@@ -206,7 +228,7 @@ bool encode_ok(CUresult r) {
 // A [B*H, T, d] bf16 tensor viewed as 3-D (d innermost), boxes of
 // (swizzle width, 128 rows, 1 head); rows past T read as zero.
 template <int D>
-bool encode_map(CUtensorMap* m, const void* base, int BH, int T) {
+bool encode_map(CUtensorMap* m, const void* base, int BH, int T, int box_rows = ca::kRows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) {
     t_last_cuda_error = "cuTensorMapEncodeTiled is not available from the driver";
@@ -215,7 +237,7 @@ bool encode_map(CUtensorMap* m, const void* base, int BH, int T) {
   using Tl = ca::Tile<D>;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
-  cuuint32_t box[3] = {(cuuint32_t)Tl::BOX_COLS, (cuuint32_t)ca::kRows, 1};
+  cuuint32_t box[3] = {(cuuint32_t)Tl::BOX_COLS, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -228,6 +250,13 @@ template <int D>
 bool make_map(CUtensorMap* m, const void* base, int BH, int T) {
   return cached_map(m, MapKey{base, kMapBf16, D, BH, T, 0},
                     [&](CUtensorMap* out) { return encode_map<D>(out, base, BH, T); });
+}
+
+// The same view with boxes of 64 rows: each CTA of a pair loads half of a 128-row tile.
+template <int D>
+bool make_half_map(CUtensorMap* m, const void* base, int BH, int T) {
+  return cached_map(m, MapKey{base, kMapBf16Half, D, BH, T, 0},
+                    [&](CUtensorMap* out) { return encode_map<D>(out, base, BH, T, 64); });
 }
 
 // A [B*H, T, d] tensor of e4m3 codes viewed as 3-D bytes (d innermost), boxes of (d, 128 rows,
@@ -285,6 +314,12 @@ int sm_count() {
   return (dev >= 0 && dev < kMaxDevices && g_sm_count[dev] > 0) ? g_sm_count[dev] : 148;
 }
 
+int pair_clusters() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return (dev >= 0 && dev < kMaxDevices && g_pair_clusters[dev] > 0) ? g_pair_clusters[dev] : 74;
+}
+
 int launch_status() {
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) return GPT_ATTN_OK;
@@ -318,6 +353,16 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.scale_log2 = scale * ca::kLog2e;
   p.window = effective_window(window, T);
   p.wait_limit_ns = kWaitLimitNs;
+  if (D == 128) {
+    // CTA pairs: each pair walks items, each CTA of it one query tile of the item
+    CUtensorMap mkh;
+    if (!make_half_map<D>(&mkh, k, BH, T)) return GPT_ATTN_ERR_LAUNCH;
+    const int pairs = pair_clusters();
+    const unsigned grid = 2u * (unsigned)(p.n_items < pairs ? p.n_items : pairs);
+    ca::attn_fwd_pair_kernel<<<grid, ca::PairLayout::THREADS, ca::PairLayout::SMEM, st>>>(
+        mq, mkh, mv, mo, p);
+    return launch_status();
+  }
   // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
   const int sms = sm_count();
   const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
