@@ -133,6 +133,29 @@ __device__ __forceinline__ bool wait_pair_warp(uint32_t bar, uint32_t parity, co
   return __all_sync(0xffffffffu, wait_pair(bar, parity, pg, site));
 }
 
+// 2^x for a pair of x <= 0 on the FMA pipe: x = n + f with n = round(x) (clamped at -125) and
+// f in [-1/2, 1/2]; 2^f from a cubic fitted for least maximum relative error on that interval
+// (Lawson's iteratively reweighted least squares; max relative error 7.5e-5, far below the
+// 2^-9 of the bf16 weights it feeds), and n added into the exponent field.  Below 2^-125 the
+// result is 2^-125 times 2^f instead of the exact value (or 0 for -inf): weights that small
+// change no sum, and no output, by more than 1e-37.
+constexpr int kExp2FmaPhase = 0;  // pairs e with e % 4 == this take the FMA path
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+  const float2 x = f2split(x2);
+  const uint64_t xc = f2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer
+  const uint64_t t = fadd2(xc, f2(kRound, kRound));
+  const uint64_t n = fadd2(t, f2(-kRound, -kRound));
+  const uint64_t fr = ffma2(n, f2(-1.f, -1.f), xc);
+  uint64_t q = ffma2(f2(0.05517166f, 0.05517166f), fr, f2(0.24261112f, 0.24261112f));
+  q = ffma2(q, fr, f2(0.69326099f, 0.69326099f));
+  q = ffma2(q, fr, f2(0.99992807f, 0.99992807f));
+  const float2 qf = f2split(q), tf = f2split(t);
+  // the low bits of t hold n in two's complement: shifted into the exponent field they add n
+  return f2(__uint_as_float(__float_as_uint(qf.x) + (__float_as_uint(tf.x) << 23)),
+            __uint_as_float(__float_as_uint(qf.y) + (__float_as_uint(tf.y) << 23)));
+}
+
 struct PairLayout {
   static constexpr int D = 128;
   static constexpr int QB = kRows * D * 2;          // own Q tile: 32 KB (2 swizzle chunks)
@@ -249,8 +272,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 
   if (warp >= 8) {
     // third warpgroup: give registers to the softmax warpgroups, then specialise
-    // (launched at 168 per thread: 2 * 128 * 192 + 128 * 120 = 384 * 168)
-    regs_shrink<120>();
+    // (launched at 168 per thread: 2 * 128 * 184 + 128 * 136 = 384 * 168)
+    regs_shrink<136>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {  // Q (double-buffered by item) and the K ring (own halves)
@@ -429,7 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     __syncwarp();
   }
   } else {
-    regs_grow<192>();
+    regs_grow<184>();
     // ------------------------------------------------------ softmax warps
     // Control flow is the same in both warps of a row quarter whatever happens (the named
     // barrier of the two must be reached by both equally often): a failed wait only clears
@@ -608,9 +631,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
               uint32_t pk[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
-                const float2 xx =
-                    f2split(ffma2(f2u(sr[c][2 * e], sr[c][2 * e + 1]), sl2x2, nmu2));
-                const float p0 = ex2(xx.x), p1 = ex2(xx.y);
+                const uint64_t x2 = ffma2(f2u(sr[c][2 * e], sr[c][2 * e + 1]), sl2x2, nmu2);
+                float p0, p1;
+                if ((e & 3) == kExp2FmaPhase) {
+                  // a quarter of the exponentials on the FMA pipe (the MUFU pipe is the
+                  // softmax's bottleneck)
+                  const float2 pe = f2split(exp2_fma2(x2));
+                  p0 = pe.x;
+                  p1 = pe.y;
+                } else {
+                  const float2 xx = f2split(x2);
+                  p0 = ex2(xx.x);
+                  p1 = ex2(xx.y);
+                }
                 const uint32_t v = pack_bf16(p0, p1);
                 acc_l[e & 1] = fadd2(acc_l[e & 1], f2(p0, p1));
                 acc_lr[e & 1] = fadd2(acc_lr[e & 1], bf16x2_to_f2(v));
