@@ -126,7 +126,7 @@ def peaks():
     return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
 
 
-MAIN_KERNEL_FILES = ("fwd.cuh", "bwd.cuh", "tiles.cuh", "sm100.cuh")
+MAIN_KERNEL_FILES = ("fwd.cuh", "fwd_pair.cuh", "bwd.cuh", "tiles.cuh", "sm100.cuh")
 PROLOGUE_KERNEL_FILES = ("prologue.cuh", "sm100.cuh")
 PROFILE_TRAFFIC_PROLOGUE = os.path.join(ROOT, "profiles", "traffic_prologue.md")
 
