@@ -18,7 +18,9 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libcausalattn.so")
+# CAUSALATTN_LIBRARY selects another build of the same library (e.g. libcausalattn_debug.so,
+# whose kernels check every TMA coordinate and computed global index on the device).
+LIB_PATH = os.environ.get("CAUSALATTN_LIBRARY") or os.path.join(_HERE, "libcausalattn.so")
 
 GPT_ATTN_OK = 0
 GPT_ATTN_ERR_NULL_PTR = 1

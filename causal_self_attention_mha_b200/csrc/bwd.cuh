@@ -170,7 +170,7 @@ __device__ __forceinline__ DkdvItem dkdv_item(const BwdParams& p, int w) {
     int lo = c_last + 1, hi = p.T;  // first r in (c_last, T) with drow[r] > c_last, else T
     while (lo < hi) {
       const int mid = lo + ((hi - lo) >> 1);
-      if (drow[mid] > c_last) hi = mid; else lo = mid + 1;
+      if (ld_chk(drow, (size_t)mid, (size_t)p.T) > c_last) hi = mid; else lo = mid + 1;
     }
     i_hi = (lo - 1) / kRows;
     i_hi = i_hi < I.jt ? I.jt : (i_hi > p.n_t - 1 ? p.n_t - 1 : i_hi);
@@ -329,8 +329,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int k = 0; k < kRows / 32; ++k) {
           const int rl = lane + 32 * k, r = r0 + rl;
           if (r < T) {  // stored negated: -LSE*log2(e) and -delta
-            lse2[rl] = -p.lse[(size_t)I.bh * T + r] * kLog2e;
-            dl[rl] = -p.delta[(size_t)I.bh * T + r];
+            lse2[rl] = -ld_chk(p.lse, (size_t)I.bh * T + r, (size_t)p.BH * T) * kLog2e;
+            dl[rl] = -ld_chk(p.delta, (size_t)I.bh * T + r, (size_t)p.BH * T);
           } else {  // rows past the end: every weight is zero
             lse2[rl] = -INFINITY;
             dl[rl] = 0.f;
@@ -474,7 +474,7 @@ __global__ void __launch_bounds__(384, 1)
         const int rb = 64 * cs;                       // first query row (in the tile) of my columns
         const int r0 = (I.i_lo + it) * kRows + rb;    // its position
         // document start of my last query row (read before the wait hides its latency)
-        const int dlast = (drow && r0 + 63 < T) ? __ldg(drow + r0 + 63) : 0;
+        const int dlast = (drow && r0 + 63 < T) ? ldg_chk(drow, (size_t)(r0 + 63), (size_t)T) : 0;
         if (!wait_bounded_warp(st_full, t & 1, g, 7) ||
             !wait_bounded_warp(vec_full(sd), (t / DST) & 1, g, 7)) {
           ok = false;
@@ -496,8 +496,8 @@ __global__ void __launch_bounds__(384, 1)
           int n_vis;  // rows r0 .. r0 + n_vis - 1 are in c's document or an earlier one, and < T
           if (drow) {
             const int ra = r0 + lane, rbb = r0 + 32 + lane;
-            const int da = ra < T ? __ldg(drow + ra) : 0x7fffffff;
-            const int db = rbb < T ? __ldg(drow + rbb) : 0x7fffffff;
+            const int da = ra < T ? ldg_chk(drow, (size_t)ra, (size_t)T) : 0x7fffffff;
+            const int db = rbb < T ? ldg_chk(drow, (size_t)rbb, (size_t)T) : 0x7fffffff;
             n_vis = rows_in_doc_prefix(da, db, c);
           } else {
             n_vis = T - r0 < 0 ? 0 : (T - r0 > 64 ? 64 : T - r0);
@@ -683,7 +683,7 @@ __device__ __forceinline__ DqItem dq_item(const BwdParams& p, int w) {
   // no key before the tile's first row's document start or window start is visible
   int first = I.q0 - p.window + 1;
   if (p.doc) {
-    const int ds = p.doc[(size_t)I.b * p.T + I.q0];
+    const int ds = ld_chk(p.doc, (size_t)I.b * p.T + I.q0, (size_t)(p.BH / p.H) * p.T);
     first = first > ds ? first : ds;
   }
   const int lo = first < 0 ? 0 : first / kRows;
@@ -952,7 +952,8 @@ __global__ void __launch_bounds__(384, 1)
       const DqItem I = dq_item(p, w);
       const int r = I.q0 + rl;  // query position owned by this thread
       // rows past T: -LSE = -inf makes every weight zero
-      const float nlse2 = (r < T) ? -p.lse[(size_t)I.bh * T + r] * kLog2e : -INFINITY;
+      const float nlse2 =
+          (r < T) ? -ld_chk(p.lse, (size_t)I.bh * T + r, (size_t)p.BH * T) * kLog2e : -INFINITY;
       float ndlt;
       if (kDelta) {
         // delta of my row from the staged O tile and dO: each of the two warps on these lanes
@@ -975,13 +976,15 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(qdo_empty);
         }
         const float dlt = dpart[rl] + dpart[kRows + rl];
-        if (cs == 0 && r < T) p.delta_out[(size_t)I.bh * T + r] = dlt;
+        if (cs == 0 && r < T) st_chk(p.delta_out, (size_t)I.bh * T + r, (size_t)p.BH * T, dlt);
         ndlt = (r < T) ? -dlt : 0.f;
       } else {
-        ndlt = (r < T) ? -p.delta[(size_t)I.bh * T + r] : 0.f;
+        ndlt = (r < T) ? -ld_chk(p.delta, (size_t)I.bh * T + r, (size_t)p.BH * T) : 0.f;
       }
       // first visible key of this row: its document start or the window's start
-      int ds = p.doc ? p.doc[(size_t)I.b * T + (r < T ? r : T - 1)] : 0;
+      int ds = p.doc ? ld_chk(p.doc, (size_t)I.b * T + (r < T ? r : T - 1),
+                              (size_t)(p.BH / p.H) * T)
+                     : 0;
       ds = ds > r - p.window + 1 ? ds : r - p.window + 1;
       const uint64_t nlse2x2 = f2(nlse2, nlse2), ndltx2 = f2(ndlt, ndlt);
       for (int it = 0; it < I.n; ++it, ++gk) {

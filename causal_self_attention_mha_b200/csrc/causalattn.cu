@@ -6,6 +6,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <cmath>
@@ -25,6 +26,15 @@ namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 constexpr int kMaxDevices = 64;
+
+// An NVTX range around each kernel launch, named after the kernel, for timelines taken with
+// nsys or `ncu --nvtx`; with no tool attached a push and a pop cost a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // ------------------------------------------------------------ validation
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -353,12 +363,15 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.scale_log2 = scale * ca::kLog2e;
   p.window = effective_window(window, T);
   p.wait_limit_ns = kWaitLimitNs;
-  if (D == 128) {
-    // CTA pairs: each pair walks items, each CTA of it one query tile of the item
+  if (D == 128 && p.window >= T) {
+    // CTA pairs: each pair walks items, each CTA of it one query tile of the item.  Both CTAs
+    // walk the union of the two tiles' key ranges, so with a sliding window (ranges offset by
+    // a tile) the single-CTA kernel, whose two tiles each walk their own range, is faster.
     CUtensorMap mkh;
     if (!make_half_map<D>(&mkh, k, BH, T)) return GPT_ATTN_ERR_LAUNCH;
     const int pairs = pair_clusters();
     const unsigned grid = 2u * (unsigned)(p.n_items < pairs ? p.n_items : pairs);
+    NvtxRange nvtx("attn_fwd_pair");
     ca::attn_fwd_pair_kernel<<<grid, ca::PairLayout::THREADS, ca::PairLayout::SMEM, st>>>(
         mq, mkh, mv, mo, p);
     return launch_status();
@@ -366,6 +379,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   // persistent: one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
   const int sms = sm_count();
   const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
+  NvtxRange nvtx("attn_fwd");
   ca::attn_fwd_kernel<D><<<grid, ca::FwdLayout<D>::THREADS, ca::FwdLayout<D>::SMEM, st>>>(
       mq, mk, mv, mo, p);
   return launch_status();
@@ -397,6 +411,7 @@ int fwd8_impl(const void* q8, const void* k8, const void* v8, float dsq, float d
   p8.descale_v = dsv;
   const int sms = sm_count();
   const unsigned grid = (unsigned)(p.n_items < sms ? p.n_items : sms);
+  NvtxRange nvtx("attn_fwd_fp8");
   ca::attn_fwd_fp8_kernel<D><<<grid, ca::Fwd8Layout<D>::THREADS, ca::Fwd8Layout<D>::SMEM, st>>>(
       mq, mk, mv, mo, p8);
   return launch_status();
@@ -409,6 +424,7 @@ int delta_impl(const void* o, const void* dout, float* delta, int B, int H, int 
   const long threads = rows * (D / 8);
   long blocks = (threads + 255) / 256;
   if (blocks > 148L * 16) blocks = 148L * 16;
+  NvtxRange nvtx("attn_bwd_delta");
   ca::attn_bwd_delta_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), delta, rows);
   return launch_status();
@@ -450,6 +466,7 @@ int bwd_tiled_impl(bool dkdv, const void* q, const void* k, const void* v, const
   if (!make_map<D>(&mg0, g0, BH, T) || (dkdv && !make_map<D>(&mg1, g1, BH, T)) ||
       (o && !make_map<D>(&mo, o, BH, T)))
     return GPT_ATTN_ERR_LAUNCH;
+  NvtxRange nvtx(dkdv ? "attn_bwd_dkdv" : (o ? "attn_bwd_dq_delta" : "attn_bwd_dq"));
   if (dkdv)
     ca::attn_bwd_dkdv_kernel<D><<<grid, ca::DkdvLayout<D>::THREADS, ca::DkdvLayout<D>::SMEM, st>>>(
         mq, mk, mv, mdo, mg0, mg1, p);
@@ -484,6 +501,8 @@ int decode_impl(const void* q, const void* kc, const void* vc, void* o, float* l
   p.wait_limit_ns = kWaitLimitNs;
   dim3 grid((unsigned)p.n_chunks, (unsigned)H, (unsigned)B);
   // the smallest token capacity that holds Tq (registers and shared memory scale with it)
+  {
+  NvtxRange nvtx("attn_decode_chunk");
   if (Tq <= 1)
     ca::attn_decode_chunk_kernel<D, 1><<<grid, ca::kDecThreads, ca::DecLayout<D, 1>::SMEM, st>>>(
         mk, mv, p);
@@ -493,8 +512,10 @@ int decode_impl(const void* q, const void* kc, const void* vc, void* o, float* l
   else
     ca::attn_decode_chunk_kernel<D, 16><<<grid, ca::kDecThreads, ca::DecLayout<D, 16>::SMEM, st>>>(
         mk, mv, p);
+  }
   int s = launch_status();
   if (s) return s;
+  NvtxRange nvtx("attn_decode_combine");
   ca::attn_decode_combine_kernel<D><<<(unsigned)(B * H * Tq), ca::kCombWarps * 32, 0, st>>>(
       p.part_ml, p.part_o, static_cast<__nv_bfloat16*>(o), lse, H, Tq, p.n_chunks);
   return launch_status();
@@ -559,6 +580,7 @@ int prologue_impl(bool bwd, const ca::ProParams& p, cudaStream_t st) {
   const long items = (long)p.B * ((p.H + hg - 1) / hg) * p.T * (D / 16);
   long blocks = (items + ca::kProThreads - 1) / ca::kProThreads;
   if (blocks > (long)sm_count() * per_sm) blocks = (long)sm_count() * per_sm;
+  NvtxRange nvtx(bwd ? "rope_qknorm_bwd" : "rope_qknorm_fwd");
   if (bwd)
     ca::rope_qknorm_bwd_kernel<D><<<(unsigned)blocks, ca::kProThreads, 0, st>>>(p);
   else

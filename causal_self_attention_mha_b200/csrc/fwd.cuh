@@ -102,7 +102,7 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& p, int w) {
       const int q0 = I.qt[x] * kRows;
       int first = q0 - p.window + 1;
       if (p.doc) {
-        const int ds = p.doc[(size_t)I.b * p.T + q0];
+        const int ds = ld_chk(p.doc, (size_t)I.b * p.T + q0, (size_t)(p.BH / p.H) * p.T);
         first = first > ds ? first : ds;
       }
       lo = first < 0 ? 0 : first / kRows;
@@ -375,7 +375,9 @@ __global__ void __launch_bounds__(384, 1)
       if (x == 1 && !I.hasB) continue;
       const int row = I.qt[x] * kRows + rl;
       // first visible key of this row: its document start or the window's start
-      int ds = p.doc ? p.doc[(size_t)I.b * T + (row < T ? row : T - 1)] : 0;
+      int ds = p.doc ? ld_chk(p.doc, (size_t)I.b * T + (row < T ? row : T - 1),
+                              (size_t)(p.BH / p.H) * T)
+                     : 0;
       ds = ds > row - p.window + 1 ? ds : row - p.window + 1;
       float m = -INFINITY;
       // acc_l: sum of the fp32 weights (for the LSE); acc_lr: sum of the bf16-rounded weights
@@ -484,7 +486,7 @@ __global__ void __launch_bounds__(384, 1)
           lr += bq.x + bq.y;
         }
         const float mu = (m == -INFINITY) ? 0.f : m;
-        if (row < T) p.lse[(size_t)I.bh * T + row] = (mu + lg2(l)) * kLn2;
+        if (row < T) st_chk(p.lse, (size_t)I.bh * T + row, (size_t)p.BH * T, (mu + lg2(l)) * kLn2);
         const float inv = 1.0f / lr;
         // the row, normalised, as packed bf16: up to two waves of 64 columns, loads in flight together
         uint32_t wo[D / 2];

@@ -360,7 +360,9 @@ __global__ void __launch_bounds__(384, 1)
       if (x == 1 && !I.hasB) continue;
       if (!ok) continue;
       const int row = I.qt[x] * kRows + rl;
-      int ds = p.doc ? p.doc[(size_t)I.b * T + (row < T ? row : T - 1)] : 0;
+      int ds = p.doc ? ld_chk(p.doc, (size_t)I.b * T + (row < T ? row : T - 1),
+                              (size_t)(p.BH / p.H) * T)
+                     : 0;
       ds = ds > row - p.window + 1 ? ds : row - p.window + 1;
       const int n = I.hi[x] - I.lo[x] + 1;
       // S of this thread's row for key tile c0, masked; returns false on a failed wait
@@ -439,7 +441,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         const float lq = (acc_q[0] + acc_q[1]) + (acc_q[2] + acc_q[3]);
         // l sums 2^8 * exp(S - m): LSE = m + log2(l) - 8, in base 2, to natural log
-        if (row < T) p.lse[(size_t)I.bh * T + row] = (m + lg2(l) - 8.0f) * kLn2;
+        if (row < T)
+          st_chk(p.lse, (size_t)I.bh * T + row, (size_t)p.BH * T, (m + lg2(l) - 8.0f) * kLn2);
         const float mul = p8.descale_v / lq;
         uint32_t wo[D / 2];
 #pragma unroll

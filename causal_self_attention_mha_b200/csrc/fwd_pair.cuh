@@ -74,6 +74,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
 // the pair (rank 0's).  c0 * 2 bytes is a multiple of 16.
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* m, int c0, int c1,
                                                  int c2, uint32_t bar_cluster) {
+  if (!tma_coords_ok(c0, c2)) return;
   asm volatile(
       "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
@@ -133,28 +134,8 @@ __device__ __forceinline__ bool wait_pair_warp(uint32_t bar, uint32_t parity, co
   return __all_sync(0xffffffffu, wait_pair(bar, parity, pg, site));
 }
 
-// 2^x for a pair of x <= 0 on the FMA pipe: x = n + f with n = round(x) (clamped at -125) and
-// f in [-1/2, 1/2]; 2^f from a cubic fitted for least maximum relative error on that interval
-// (Lawson's iteratively reweighted least squares; max relative error 7.5e-5, far below the
-// 2^-9 of the bf16 weights it feeds), and n added into the exponent field.  Below 2^-125 the
-// result is 2^-125 times 2^f instead of the exact value (or 0 for -inf): weights that small
-// change no sum, and no output, by more than 1e-37.
-constexpr int kExp2FmaPhase = 0;  // pairs e with e % 4 == this take the FMA path
-__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
-  const float2 x = f2split(x2);
-  const uint64_t xc = f2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
-  constexpr float kRound = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer
-  const uint64_t t = fadd2(xc, f2(kRound, kRound));
-  const uint64_t n = fadd2(t, f2(-kRound, -kRound));
-  const uint64_t fr = ffma2(n, f2(-1.f, -1.f), xc);
-  uint64_t q = ffma2(f2(0.05517166f, 0.05517166f), fr, f2(0.24261112f, 0.24261112f));
-  q = ffma2(q, fr, f2(0.69326099f, 0.69326099f));
-  q = ffma2(q, fr, f2(0.99992807f, 0.99992807f));
-  const float2 qf = f2split(q), tf = f2split(t);
-  // the low bits of t hold n in two's complement: shifted into the exponent field they add n
-  return f2(__uint_as_float(__float_as_uint(qf.x) + (__float_as_uint(tf.x) << 23)),
-            __uint_as_float(__float_as_uint(qf.y) + (__float_as_uint(tf.y) << 23)));
-}
+// softmax pairs e with e % 4 == this evaluate their exponentials with exp2_fma2
+constexpr int kExp2FmaPhase = 0;
 
 struct PairLayout {
   static constexpr int D = 128;
@@ -495,7 +476,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       l += xl;
       lr += xlr;
       const float mu = (m == -INFINITY) ? 0.f : m;
-      if (h == 0 && row < T) p.lse[(size_t)bh * T + row] = (mu + lg2(l)) * kLn2;
+      if (h == 0 && row < T)
+        st_chk(p.lse, (size_t)bh * T + row, (size_t)p.BH * T, (mu + lg2(l)) * kLn2);
       const float inv = 1.0f / lr;
       const uint32_t tO = tO0 + 128u * (uint32_t)(k & 1);
       uint32_t wo[32];
@@ -533,7 +515,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       const FwdItem I = fwd_item(p, w);
       const int row = (rank ? I.qt[1] : I.qt[0]) * kRows + rl;
       const uint32_t tO = tO0 + 128u * (uint32_t)(k_ & 1);
-      int ds = p.doc ? p.doc[(size_t)I.b * T + (row < T ? row : T - 1)] : 0;
+      int ds = p.doc ? ld_chk(p.doc, (size_t)I.b * T + (row < T ? row : T - 1),
+                              (size_t)(p.BH / p.H) * T)
+                     : 0;
       ds = ds > row - p.window + 1 ? ds : row - p.window + 1;
       // rows of this quarter: the first and last visible key over its 32 rows (a tile outside
       // every row's range of visible keys gets zero weights without exponentials); the same

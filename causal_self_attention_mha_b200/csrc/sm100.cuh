@@ -19,6 +19,7 @@ namespace ca {
 enum : unsigned {
   kStatusTimeout = 1u << 31,
   kStatusSmem = 1u << 30,  // a kernel's shared-memory layout did not fit what it was given
+  kStatusBounds = 1u << 29,  // (debug builds) a checked index or TMA coordinate was out of range
 };
 
 __device__ unsigned int g_status;
@@ -28,6 +29,40 @@ __device__ __forceinline__ void report_timeout(unsigned site) {
 }
 
 __device__ __forceinline__ void report_smem_shortfall() { atomicOr(&g_status, kStatusSmem); }
+
+// Debug builds (compiled with CA_DEBUG_CHECKS): the kernels check every TMA coordinate and
+// every global index they compute on the device; a failed check sets kStatusBounds and the
+// access is skipped (a load reads 0, a TMA copy is not issued, so its waiter times out and
+// reports) instead of trapping.  In release builds the checks compile to nothing.
+#ifdef CA_DEBUG_CHECKS
+__device__ __forceinline__ bool dbg_ok(bool ok) {
+  if (!ok) atomicOr(&g_status, kStatusBounds);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool dbg_ok(bool) { return true; }
+#endif
+
+// a[i] of an array of n elements (i computed by the kernel), checked in debug builds.
+template <class T>
+__device__ __forceinline__ T ld_chk(const T* a, size_t i, size_t n) {
+  return dbg_ok(i < n) ? a[i] : T(0);
+}
+template <class T>
+__device__ __forceinline__ T ldg_chk(const T* a, size_t i, size_t n) {
+  return dbg_ok(i < n) ? __ldg(a + i) : T(0);
+}
+template <class T>
+__device__ __forceinline__ void st_chk(T* a, size_t i, size_t n, T v) {
+  if (dbg_ok(i < n)) a[i] = v;
+}
+
+// The innermost coordinate of a tiled TMA copy must start on a 16-byte boundary: every copy
+// here moves 16-bit (bf16) or 8-bit (e4m3, at x = 0) elements, so x is a multiple of 8; a
+// store never starts at a negative coordinate.
+__device__ __forceinline__ bool tma_coords_ok(int c0, int c_outer) {
+  return dbg_ok(c0 >= 0 && (c0 & 7) == 0 && c_outer >= 0);
+}
 
 // Opt-in limit of dynamic shared memory per block (227 KB).
 constexpr int kMaxDynSmem = 232448;
@@ -124,6 +159,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
 // 16 here (c0 is 0 or a multiple of the 32/64-element swizzle width).
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, int c0, int c1,
                                             int c2, uint32_t bar) {
+  if (!tma_coords_ok(c0, c2)) return;
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
@@ -134,6 +170,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
 // 4-D tiled load, as above (c0 * 2 bytes a multiple of 16).
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, int c0, int c1,
                                             int c2, int c3, uint32_t bar) {
+  if (!tma_coords_ok(c0, c1 | c3)) return;
   asm volatile(
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
@@ -145,6 +182,7 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, 
 // written).  Completion is tracked per thread with bulk groups.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t src, int c0, int c1,
                                              int c2) {
+  if (!tma_coords_ok(c0, c1 | c2)) return;
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(m)),
                "r"(src), "r"(c0), "r"(c1), "r"(c2)
@@ -375,6 +413,28 @@ __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+// 2^x for a pair of x < 126 on the FMA pipe: x = n + f with n = round(x) (clamped at -125) and
+// f in [-1/2, 1/2]; 2^f from a cubic fitted for least maximum relative error on that interval
+// (Lawson's iteratively reweighted least squares; max relative error 7.5e-5, far below the
+// 2^-9 of the bf16 weights it feeds), and n added into the exponent field.  Below 2^-125 the
+// result is 2^-125 times 2^f instead of the exact value (or 0 for -inf): weights that small
+// change no sum, and no output, by more than 1e-37.
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+  const float2 x = f2split(x2);
+  const uint64_t xc = f2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer
+  const uint64_t t = fadd2(xc, f2(kRound, kRound));
+  const uint64_t n = fadd2(t, f2(-kRound, -kRound));
+  const uint64_t fr = ffma2(n, f2(-1.f, -1.f), xc);
+  uint64_t q = ffma2(f2(0.05517166f, 0.05517166f), fr, f2(0.24261112f, 0.24261112f));
+  q = ffma2(q, fr, f2(0.69326099f, 0.69326099f));
+  q = ffma2(q, fr, f2(0.99992807f, 0.99992807f));
+  const float2 qf = f2split(q), tf = f2split(t);
+  // the low bits of t hold n in two's complement: shifted into the exponent field they add n
+  return f2(__uint_as_float(__float_as_uint(qf.x) + (__float_as_uint(tf.x) << 23)),
+            __uint_as_float(__float_as_uint(qf.y) + (__float_as_uint(tf.y) << 23)));
+}
+
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

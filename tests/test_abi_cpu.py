@@ -260,3 +260,20 @@ def test_prepare_records_the_marshalled_call(lib, monkeypatch):
         abi.load().gpt_attn_version()
     with pytest.raises(ValueError, match="one library call"):
         abi.prepare(two_calls)
+
+
+def test_debug_checks_library_exports_every_symbol(lib):
+    """libcausalattn_debug.so (the same sources with device-side bounds checks) is a drop-in
+    replacement: it exports every declared entry point, and its validation behaves alike."""
+    path = build.build(debug=True)
+    dbg = abi.load(path)  # sets argtypes for every declared symbol (raises if one is missing)
+    assert dbg.gpt_attn_version() == lib.gpt_attn_version()
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+    assert dbg.gpt_attn_strerror(-1) == lib.gpt_attn_strerror(-1)
+
+
+def test_debug_build_command_defines_the_checks():
+    cmd = build.nvcc_command("out.so", debug=True)
+    assert "-DCA_DEBUG_CHECKS" in cmd and "arch=compute_100a,code=sm_100a" in cmd
+    assert "-DCA_DEBUG_CHECKS" not in build.nvcc_command("out.so")
