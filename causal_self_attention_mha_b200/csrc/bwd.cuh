@@ -104,8 +104,9 @@ __device__ __forceinline__ void tmem_half_row_bf16(uint32_t tacc, int half, floa
 // chain.  384 threads = three warpgroups: warpgroups 0-1 are the element-wise
 // warps (warp w owns TMEM lanes 32*(w%4).. and columns 64*(w/4).. of each
 // tile), the third holds the TMA producer and the single MMA-issuing thread;
-// registers are rebalanced with setmaxnreg (168 at launch; 208 for the
-// element-wise warpgroups, 88 for the third).  An element-wise thread keeps its
+// registers are rebalanced with setmaxnreg (168 at launch; dQ: 208 for the
+// element-wise warpgroups, 88 for the third; dK/dV: 192 and 120, where the third
+// warpgroup's MMA issuer needs more).  An element-wise thread keeps its
 // 64 fp32 P values in registers while it waits for dP.  P and dS go back to
 // TMEM as packed bf16 over the first half of the columns the same warp has
 // just read, and feed the gradient MMAs as their A operand.  At an item
@@ -285,7 +286,7 @@ __global__ void __launch_bounds__(384, 1)
   const Guard g{abort_flag, p.wait_limit_ns};
 
   if (warp >= L::COMPUTE_WARPS) {
-    regs_shrink<88>();
+    regs_shrink<120>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t tdV = tmem + L::T_DV, tdK = tmem + L::T_DK;
       auto issue_st = [&](int t) -> bool {  // S^T = K Q_t^T
         const int s = t % QST;
-        if (!wait_bounded(q_full(s), (t / QST) & 1, g, 3)) return false;
+        if (!wait_bounded_fast(q_full(s), (t / QST) & 1, g, 3)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       auto issue_dpt = [&](int t) -> bool {  // dP^T = V dO_t^T
         const int s = t % DST;
-        if (!wait_bounded(do_full(s), (t / DST) & 1, g, 3)) return false;
+        if (!wait_bounded_fast(do_full(s), (t / DST) & 1, g, 3)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
@@ -385,17 +386,17 @@ __global__ void __launch_bounds__(384, 1)
         const int w = snake_item(k_, w0, dw, p.n_items);
         if (w < 0) break;  // past the last item: no later round has one either
         const DkdvItem I = dkdv_item(p, w);
-        if (!wait_bounded(kv_full, li & 1, g, 2)) break;
+        if (!wait_bounded_fast(kv_full, li & 1, g, 2)) break;
         if (!issue_st(gq) || !issue_dpt(gq)) break;
         if (I.n == 1) tc_commit(kv_empty);  // K, V of this item no longer read after these
         for (int it = 0; it < I.n; ++it, ++gq) {
           const int t = gq, sq = t % QST, sd = t % DST;
           // dV += P^T dO: the first one of an item overwrites dV, so the previous
           // item's epilogue must have read it
-          if (it == 0 && li >= 1 && !wait_bounded(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
+          if (it == 0 && li >= 1 && !wait_bounded_fast(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
           // half h holds query rows 64c + 32h + [0, 32) of the tile, c = 0, 1: K-steps 4c + 2h + {0, 1}
           for (int h = 0; h < 2; ++h) {
-            if (!wait_bounded(p_ready(h), t & 1, g, 5)) { ok = false; break; }
+            if (!wait_bounded_fast(p_ready(h), t & 1, g, 5)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(384, 1)
           const bool more = it + 1 < I.n;
           // S^T of the next query tile, behind dV(t) in the stream
           if (more && !issue_st(t + 1)) { ok = false; break; }
-          if (!wait_bounded(ds_ready, t & 1, g, 6)) { ok = false; break; }
+          if (!wait_bounded_fast(ds_ready, t & 1, g, 6)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kRows / 16; ++kk)
@@ -453,7 +454,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   }
   } else {
-    regs_grow<208>();
+    regs_grow<192>();
     // ------------------------------------------- P^T / dS^T (thread = key row)
     const int qd = warp & 3, cs = warp >> 2;
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
@@ -851,7 +852,7 @@ __global__ void __launch_bounds__(384, 1)
       auto issue_s = [&](int t) -> bool {  // S(t) = Q K_t^T into buffer t & 1
         const int el = t + li * PER_ITEM + E;
         const int s = el % STK;
-        if (!wait_bounded(k_full(s), (el / STK) & 1, g, 3)) return false;
+        if (!wait_bounded_fast(k_full(s), (el / STK) & 1, g, 3)) return false;
         tc_fence_after();
         const uint32_t tS = tmem + L::T_S + 128u * (uint32_t)(t & 1);
 #pragma unroll
@@ -862,7 +863,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       auto issue_dp = [&](int t) -> bool {  // dP(t) = dO V_t^T
         const int s = t % STV;
-        if (!wait_bounded(v_full(s), (t / STV) & 1, g, 3)) return false;
+        if (!wait_bounded_fast(v_full(s), (t / STV) & 1, g, 3)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
@@ -876,10 +877,10 @@ __global__ void __launch_bounds__(384, 1)
         const int w = snake_item(k_, w0, dw, p.n_items);
         if (w < 0) break;  // past the last item: no later round has one either
         const DqItem I = dq_item(p, w);
-        if (!wait_bounded(qdo_full, li & 1, g, 2)) break;
+        if (!wait_bounded_fast(qdo_full, li & 1, g, 2)) break;
         const int t0 = gk;
         // dP(t0) overwrites dP(t0 - 1): the element-wise warps must have loaded it
-        if (t0 > 0 && !wait_bounded(dp_read, (t0 - 1) & 1, g, 9)) break;
+        if (t0 > 0 && !wait_bounded_fast(dp_read, (t0 - 1) & 1, g, 9)) break;
         ok = issue_s(t0) && issue_dp(t0);
         if (ok && I.n == 1) tc_commit(qdo_empty);  // Q, dO of this item no longer read
         if (ok && I.n > 1) ok = issue_s(t0 + 1);
@@ -887,12 +888,12 @@ __global__ void __launch_bounds__(384, 1)
           const int t = t0 + it;
           // dP of the next key tile as soon as dP(t) has been read out of TMEM
           if (it + 1 < I.n) {
-            if (!wait_bounded(dp_read, t & 1, g, 9) || !issue_dp(t + 1)) { ok = false; break; }
+            if (!wait_bounded_fast(dp_read, t & 1, g, 9) || !issue_dp(t + 1)) { ok = false; break; }
             if (it + 2 == I.n) tc_commit(qdo_empty);  // that was the item's last S / dP
           }
           // the first dQ MMA of an item overwrites dQ: the previous epilogue must have read it
-          if (it == 0 && li >= 1 && !wait_bounded(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
-          if (!wait_bounded(ds_full, t & 1, g, 5)) { ok = false; break; }
+          if (it == 0 && li >= 1 && !wait_bounded_fast(acc_free, (li - 1) & 1, g, 4)) { ok = false; break; }
+          if (!wait_bounded_fast(ds_full, t & 1, g, 5)) { ok = false; break; }
           tc_fence_after();
           const int s = (t + li * PER_ITEM + E) % STK;
           const uint32_t tdS = tmem + L::T_S + 128u * (uint32_t)(t & 1);  // dS(t) over S(t)

@@ -266,11 +266,11 @@ __global__ void __launch_bounds__(384, 1)
       bool pend_first[2] = {false, false}, pend_rel[2] = {false, false};
       auto issue_pv = [&](int x) -> bool {
         const int tp = pend_t[x];
-        if (pend_first[x] && nq[x] >= 2 && !wait_bounded(o_free(x), (nq[x] - 2) & 1, g, 4))
+        if (pend_first[x] && nq[x] >= 2 && !wait_bounded_fast(o_free(x), (nq[x] - 2) & 1, g, 4))
           return false;  // the previous item's epilogue must have read O_x
-        if (!wait_bounded(p_full(x), tp & 1, g, 5)) return false;
+        if (!wait_bounded_fast(p_full(x), tp & 1, g, 5)) return false;
         const int sv = pend_v[x] % STV;
-        if (!wait_bounded(v_full(sv), (pend_v[x] / STV) & 1, g, 6)) return false;
+        if (!wait_bounded_fast(v_full(sv), (pend_v[x] / STV) & 1, g, 6)) return false;
         tc_fence_after();
         const uint32_t sVs = sV + sv * Tl::BYTES;
         const uint32_t tP = tmem + 128u * x, tO = tmem + 256u + x * D;
@@ -290,14 +290,14 @@ __global__ void __launch_bounds__(384, 1)
         // B's last S of the previous item has read the old one, a key tile later than A's
         for (int j = I.j_lo; ok && j <= I.j_hi; ++j, ++gk, ++gv) {
           const int sk = gk % STK;
-          if (!wait_bounded(k_full(sk), (gk / STK) & 1, g, 3)) { ok = false; break; }
+          if (!wait_bounded_fast(k_full(sk), (gk / STK) & 1, g, 3)) { ok = false; break; }
           const bool actB = I.hasB && j >= I.lo[1] && j <= I.hi[1];
           // slot x: the pending PV of x (previous key tile), then S_x for this key tile
           auto step = [&](int x, bool act) -> bool {
             if (pend_t[x] >= 0 && !issue_pv(x)) return false;
             if (!act) return true;
             if (j == I.lo[x]) {  // first S of this query tile: its Q must have landed
-              if (!wait_bounded(q_full(x), nq[x] & 1, g, 2)) return false;
+              if (!wait_bounded_fast(q_full(x), nq[x] & 1, g, 2)) return false;
               ++nq[x];
             }
             tc_fence_after();

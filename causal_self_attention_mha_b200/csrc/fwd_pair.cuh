@@ -129,6 +129,12 @@ __device__ __forceinline__ bool wait_pair(uint32_t bar, uint32_t parity, const P
   return false;
 }
 
+// The MMA-issuing thread's wait: the phase is tested once before the (sleeping) bounded wait.
+__device__ __forceinline__ bool wait_pair_fast(uint32_t bar, uint32_t parity, const PairGuard& pg,
+                                               unsigned site) {
+  return mbar_test(bar, parity) || wait_pair(bar, parity, pg, site);
+}
+
 __device__ __forceinline__ bool wait_pair_warp(uint32_t bar, uint32_t parity, const PairGuard& pg,
                                                unsigned site) {
   return __all_sync(0xffffffffu, wait_pair(bar, parity, pg, site));
@@ -338,8 +344,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       // in the in-order MMA stream and overwrites P(t) only after PV(t) has read it
       auto issue_s = [&]() -> bool {
         const int b = st & 1, qb = sk & 1;
-        if (sj == 0 && !wait_pair(q_full(qb), (sk >> 1) & 1, g, 2)) return false;
-        if (!wait_pair(k_full(ks), kph, g, 3)) return false;
+        if (sj == 0 && !wait_pair_fast(q_full(qb), (sk >> 1) & 1, g, 2)) return false;
+        if (!wait_pair_fast(k_full(ks), kph, g, 3)) return false;
         tc_fence_after();
         const uint64_t a0 = dQ + (uint64_t)((qb * L::QB) >> 4);
         const uint64_t b0 = dK + (uint64_t)((ks * L::KB) >> 4);
@@ -371,11 +377,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         const bool first_pv = (pj == 0), last_pv = (pj == pn - 1);
         // O buffer pk & 1 is overwritten by item pk's first PV: the epilogue of item pk - 2
         // must have read it
-        if (first_pv && pk >= 2 && !wait_pair(o_free(pk & 1), ((pk >> 1) - 1) & 1, g, 4)) {
+        if (first_pv && pk >= 2 && !wait_pair_fast(o_free(pk & 1), ((pk >> 1) - 1) & 1, g, 4)) {
           ok = false;
           break;
         }
-        if (!wait_pair(p_full(b), (pt >> 1) & 1, g, 5) || !wait_pair(v_full(vs), vph, g, 6)) {
+        if (!wait_pair_fast(p_full(b), (pt >> 1) & 1, g, 5) || !wait_pair_fast(v_full(vs), vph, g, 6)) {
           ok = false;
           break;
         }
