@@ -114,9 +114,12 @@ def make_decode(B: int, H: int, Tq: int, L: int, d: int, seed: int):
 
 
 # KV-cache decode workloads (bench.py --workload decode_8k): one new token per step over a
-# cache of L positions, the GPT-2 / 400M head counts with a d = 128 head.
+# cache of L positions, the GPT-2 / 400M head counts with a d = 128 head; the _tq variants
+# append 4 or 16 tokens per step (speculative drafts).
 DECODE_WORKLOADS = {
     "decode_8k": dict(B=8, H=16, Tq=1, L=8192, d=128, seed=6),
+    "decode_8k_tq4": dict(B=8, H=16, Tq=4, L=8192, d=128, seed=6),
+    "decode_8k_tq16": dict(B=8, H=16, Tq=16, L=8192, d=128, seed=6),
 }
 
 
