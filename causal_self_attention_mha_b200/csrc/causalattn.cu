@@ -504,13 +504,13 @@ int decode_impl(const void* q, const void* kc, const void* vc, void* o, float* l
   {
   NvtxRange nvtx("attn_decode_chunk");
   if (Tq <= 1)
-    ca::attn_decode_chunk_kernel<D, 1><<<grid, ca::kDecThreads, ca::DecLayout<D, 1>::SMEM, st>>>(
+    ca::attn_decode_chunk_kernel<D, 1><<<grid, ca::dec_threads<1>(), ca::DecLayout<D, 1>::SMEM, st>>>(
         mk, mv, p);
   else if (Tq <= 4)
-    ca::attn_decode_chunk_kernel<D, 4><<<grid, ca::kDecThreads, ca::DecLayout<D, 4>::SMEM, st>>>(
+    ca::attn_decode_chunk_kernel<D, 4><<<grid, ca::dec_threads<4>(), ca::DecLayout<D, 4>::SMEM, st>>>(
         mk, mv, p);
   else
-    ca::attn_decode_chunk_kernel<D, 16><<<grid, ca::kDecThreads, ca::DecLayout<D, 16>::SMEM, st>>>(
+    ca::attn_decode_chunk_kernel<D, 16><<<grid, ca::dec_threads<16>(), ca::DecLayout<D, 16>::SMEM, st>>>(
         mk, mv, p);
   }
   int s = launch_status();

@@ -26,6 +26,11 @@ namespace ca {
 
 constexpr int kDecChunk = 128;   // keys per CTA (one TMA box of rows)
 constexpr int kDecThreads = 128;
+// Threads of a chunk CTA: one token, a thread per key row; several tokens, two threads per key
+// row (each taking half of the tokens in the score pass) -- the multi-token path is bound by
+// shared-memory and L1 latency, and twice the warps hide twice as much of it.
+template <int TQM>
+constexpr int dec_threads() { return TQM > 1 ? 2 * kDecThreads : kDecThreads; }
 constexpr int kDecMaxTq = 16;    // new tokens per call
 
 struct DecParams {
@@ -43,8 +48,9 @@ struct DecLayout {
   static constexpr int V_OFF = Tile<D>::BYTES;
   static constexpr int Q_OFF = 2 * Tile<D>::BYTES;                 // fp32 [TQM][D], times scale*log2e
   static constexpr int P_OFF = Q_OFF + TQM * D * 4;                // fp32 [TQM][128] weights
+  static constexpr int NT = dec_threads<TQM>();
   static constexpr int RED_OFF = P_OFF + TQM * kDecChunk * 4;      // fp32 [2][TQM][4] warp partials
-  static constexpr int G = kDecThreads / D;                        // key groups in the V pass
+  static constexpr int G = NT / D;                                 // key groups in the V pass
   static constexpr int ACC_OFF = RED_OFF + 2 * TQM * 4 * 4;        // fp32 [G][TQM][D] group sums
   static constexpr int BAR_OFF = ACC_OFF + (G > 1 ? G * TQM * D * 4 : 0);  // K landed, V landed
   static constexpr int MISC_OFF = BAR_OFF + 16;
@@ -61,7 +67,8 @@ __device__ __forceinline__ uint32_t tile_elem_offset(int r, int col) {
   return (uint32_t)(ch * Tl::CHUNK_BYTES + r * Tl::SW + phys * 16 + (col % 8) * 2);
 }
 
-// Block-wide max or sum of v[t] (t < TQM) over the 4 warps; every thread gets the results.
+// Max or sum of v[t] (t < TQM) over the 4 warps of this thread's group of 128 threads (the
+// group's own slice of `red`); every thread of the group gets the results.
 template <int TQM>
 __device__ __forceinline__ void dec_block_reduce(float (&v)[TQM], bool is_max, float* red) {
 #pragma unroll
@@ -71,7 +78,7 @@ __device__ __forceinline__ void dec_block_reduce(float (&v)[TQM], bool is_max, f
       const float o = __shfl_xor_sync(0xffffffffu, v[t], off);
       v[t] = is_max ? fmaxf(v[t], o) : v[t] + o;
     }
-  const int warp = threadIdx.x >> 5;
+  const int warp = (threadIdx.x >> 5) & 3;
   if ((threadIdx.x & 31) == 0) {
 #pragma unroll
     for (int t = 0; t < TQM; ++t) red[t * 4 + warp] = v[t];
@@ -87,7 +94,7 @@ __device__ __forceinline__ void dec_block_reduce(float (&v)[TQM], bool is_max, f
 // One CTA: one 128-key chunk of one (batch, head), every new token at once: each key row
 // and each V element is read from shared memory once for all Tq tokens.
 template <int D, int TQM>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(dec_threads<TQM>())
     attn_decode_chunk_kernel(const __grid_constant__ CUtensorMap tmK,
                              const __grid_constant__ CUtensorMap tmV, const DecParams p) {
   using Tl = Tile<D>;
@@ -127,7 +134,7 @@ __global__ void __launch_bounds__(kDecThreads)
                   c * kDecChunk, b, bar_v);
   }
   // the new tokens' queries, times scale * log2(e), while the rows arrive (zero past Tq)
-  for (int i = tid; i < TQM * D; i += kDecThreads) {
+  for (int i = tid; i < TQM * D; i += L::NT) {
     const int t = i / D, col = i % D;
     qs[i] = t < Tq ? __bfloat162float(p.q[(((size_t)b * Tq + t) * p.H + h) * D + col]) * p.scale_log2
                    : 0.f;
@@ -144,21 +151,24 @@ __global__ void __launch_bounds__(kDecThreads)
     return;
   }
 
-  // scores of my key row against every new token (base 2; -inf where not visible)
-  const int j = c * kDecChunk + tid;
-  float s[TQM];
+  // scores of my key row against my half of the new tokens (base 2; -inf where not visible)
+  constexpr int TH = TQM / (L::NT / kDecChunk);  // tokens per score thread
+  const int kr = tid % kDecChunk, th = tid / kDecChunk;
+  const int j = c * kDecChunk + kr;
+  float s[TH];
 #pragma unroll
-  for (int t = 0; t < TQM; ++t) s[t] = 0.f;
+  for (int i = 0; i < TH; ++i) s[i] = 0.f;
 #pragma unroll
   for (int u = 0; u < D / 8; ++u) {
-    const uint4 kv = *reinterpret_cast<const uint4*>(sK + tile_elem_offset<D>(tid, 8 * u));
+    const uint4 kv = *reinterpret_cast<const uint4*>(sK + tile_elem_offset<D>(kr, 8 * u));
     const float k8[8] = {bf16_lo(kv.x), bf16_hi(kv.x), bf16_lo(kv.y), bf16_hi(kv.y),
                          bf16_lo(kv.z), bf16_hi(kv.z), bf16_lo(kv.w), bf16_hi(kv.w)};
 #pragma unroll
-    for (int t = 0; t < TQM; ++t) {
+    for (int i = 0; i < TH; ++i) {
+      const int t = th * TH + i;
       const float4 q0 = *reinterpret_cast<const float4*>(qs + t * D + 8 * u);
       const float4 q1 = *reinterpret_cast<const float4*>(qs + t * D + 8 * u + 4);
-      float a = s[t];
+      float a = s[i];
       a = fmaf(k8[0], q0.x, a);
       a = fmaf(k8[1], q0.y, a);
       a = fmaf(k8[2], q0.z, a);
@@ -167,22 +177,25 @@ __global__ void __launch_bounds__(kDecThreads)
       a = fmaf(k8[5], q1.y, a);
       a = fmaf(k8[6], q1.z, a);
       a = fmaf(k8[7], q1.w, a);
-      s[t] = a;
+      s[i] = a;
     }
   }
 #pragma unroll
-  for (int t = 0; t < TQM; ++t)  // query t sees keys 0 .. L - Tq + t
-    if (t >= Tq || j > p.L - Tq + t) s[t] = -INFINITY;
-  float m[TQM], w[TQM];
-#pragma unroll
-  for (int t = 0; t < TQM; ++t) m[t] = s[t];
-  dec_block_reduce<TQM>(m, true, red);
-#pragma unroll
-  for (int t = 0; t < TQM; ++t) {
-    w[t] = (s[t] == -INFINITY) ? 0.f : ex2(s[t] - m[t]);
-    ps[t * kDecChunk + tid] = w[t];
+  for (int i = 0; i < TH; ++i) {  // query t sees keys 0 .. L - Tq + t
+    const int t = th * TH + i;
+    if (t >= Tq || j > p.L - Tq + t) s[i] = -INFINITY;
   }
-  dec_block_reduce<TQM>(w, false, red + TQM * 4);  // w[t] now holds the chunk's sum for token t
+  float m[TH], w[TH];
+#pragma unroll
+  for (int i = 0; i < TH; ++i) m[i] = s[i];
+  dec_block_reduce<TH>(m, true, red + th * TH * 4);
+#pragma unroll
+  for (int i = 0; i < TH; ++i) {
+    w[i] = (s[i] == -INFINITY) ? 0.f : ex2(s[i] - m[i]);
+    ps[(th * TH + i) * kDecChunk + kr] = w[i];
+  }
+  // w[i] now holds the chunk's sum for token th * TH + i
+  dec_block_reduce<TH>(w, false, red + TQM * 4 + th * TH * 4);
   // V must have landed before the weighted sums (ps is complete after the reduction's barrier)
   {
     const bool vok = wait_bounded(bar_v, 0, g, 2);
@@ -220,9 +233,15 @@ __global__ void __launch_bounds__(kDecThreads)
     if (t >= Tq) break;
     const size_t row = (((size_t)b * p.H + h) * Tq + t) * p.n_chunks + c;
     if (grp == 0) p.part_o[row * D + col] = acc[t];
-    if (tid == 0) {
-      p.part_ml[row * 2] = m[t];
-      p.part_ml[row * 2 + 1] = w[t];
+  }
+  if (kr == 0) {  // the chunk maximum and sum of this half's tokens
+#pragma unroll
+    for (int i = 0; i < TH; ++i) {
+      const int t = th * TH + i;
+      if (t >= Tq) break;
+      const size_t row = (((size_t)b * p.H + h) * Tq + t) * p.n_chunks + c;
+      p.part_ml[row * 2] = m[i];
+      p.part_ml[row * 2 + 1] = w[i];
     }
   }
 }
