@@ -93,11 +93,8 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D, 1>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D, 1>::SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D, 4>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D, 4>::SMEM);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D, 16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D, 16>::SMEM);
+  e = cudaFuncSetAttribute(ca::attn_decode_chunk_tc_kernel<D>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecTcLayout<D>::SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(ca::attn_bwd_dq_kernel<D, true>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DqLayout<D>::SMEM);
@@ -500,17 +497,14 @@ int decode_impl(const void* q, const void* kc, const void* vc, void* o, float* l
   p.scale_log2 = scale * ca::kLog2e;
   p.wait_limit_ns = kWaitLimitNs;
   dim3 grid((unsigned)p.n_chunks, (unsigned)H, (unsigned)B);
-  // the smallest token capacity that holds Tq (registers and shared memory scale with it)
+  // one new token: CUDA cores, a thread per key row; two or more: tensor cores
   {
   NvtxRange nvtx("attn_decode_chunk");
-  if (Tq <= 1)
-    ca::attn_decode_chunk_kernel<D, 1><<<grid, ca::dec_threads<1>(), ca::DecLayout<D, 1>::SMEM, st>>>(
-        mk, mv, p);
-  else if (Tq <= 4)
-    ca::attn_decode_chunk_kernel<D, 4><<<grid, ca::dec_threads<4>(), ca::DecLayout<D, 4>::SMEM, st>>>(
-        mk, mv, p);
+  if (Tq >= ca::kDecTcMinTq)
+    ca::attn_decode_chunk_tc_kernel<D><<<grid, ca::DecTcLayout<D>::THREADS, ca::DecTcLayout<D>::SMEM,
+                                         st>>>(mk, mv, p);
   else
-    ca::attn_decode_chunk_kernel<D, 16><<<grid, ca::dec_threads<16>(), ca::DecLayout<D, 16>::SMEM, st>>>(
+    ca::attn_decode_chunk_kernel<D, 1><<<grid, ca::dec_threads<1>(), ca::DecLayout<D, 1>::SMEM, st>>>(
         mk, mv, p);
   }
   int s = launch_status();

@@ -9,14 +9,16 @@
 // engine keeps a KV cache and calls FlashAttention-3's kv-cache entry point on
 // (B, T, H, D) tensors) is what this reproduces; the cache uses that layout.
 //
-// The work is one pass over the cache, so the kernel is bound by HBM
-// bandwidth, not by arithmetic: each CTA takes one 128-key chunk of one
-// (batch, head), brings the chunk's K and V rows in by TMA (128-byte swizzle,
-// so that a thread per key row and a thread per column both read shared
-// memory without bank conflicts), and computes, for every new token, the
+// The work is one pass over the cache, so HBM bandwidth bounds it: each CTA
+// takes one 128-key chunk of one (batch, head), brings the chunk's K and V
+// rows in by TMA (128-byte swizzle), and computes, for every new token, the
 // chunk's scores, their maximum, the sum of their exponentials and the
-// unnormalised weighted sum of V rows on CUDA cores (one key row or one
-// output column per thread).  A second kernel merges the chunks of each
+// unnormalised weighted sum of V rows.  With one new token that is a
+// matrix-vector product, done on CUDA cores (one key row or one output column
+// per thread, conflict-free shared-memory reads thanks to the swizzle); with
+// two or more the arithmetic per cache byte outgrows the CUDA cores and the
+// chunk kernel runs its two products on the tensor cores instead
+// (attn_decode_chunk_tc_kernel).  A second kernel merges the chunks of each
 // (batch, head, token) in chunk order -- deterministic, no atomics.
 #pragma once
 
@@ -26,12 +28,14 @@ namespace ca {
 
 constexpr int kDecChunk = 128;   // keys per CTA (one TMA box of rows)
 constexpr int kDecThreads = 128;
-// Threads of a chunk CTA: one token, a thread per key row; several tokens, two threads per key
-// row (each taking half of the tokens in the score pass) -- the multi-token path is bound by
-// shared-memory and L1 latency, and twice the warps hide twice as much of it.
+// Threads of a CUDA-core chunk CTA holding up to TQM tokens: one token, a thread per key row;
+// several, two threads per key row (each taking half of the tokens in the score pass).  The
+// library instantiates it for one token (several go to the tensor-core kernel, which is
+// 1.3-3x faster from two tokens on).
 template <int TQM>
 constexpr int dec_threads() { return TQM > 1 ? 2 * kDecThreads : kDecThreads; }
 constexpr int kDecMaxTq = 16;    // new tokens per call
+constexpr int kDecTcMinTq = 2;   // from this many new tokens on, the tensor-core chunk kernel
 
 struct DecParams {
   const __nv_bfloat16* q;  // [B, Tq, H, D]
@@ -243,6 +247,245 @@ __global__ void __launch_bounds__(dec_threads<TQM>())
       p.part_ml[row * 2] = m[i];
       p.part_ml[row * 2 + 1] = w[i];
     }
+  }
+}
+
+// Tensor-core form of the chunk kernel for two or more new tokens.  With Tq tokens a cached
+// key row (2d bytes of K and of V) feeds 4 d Tq flops, so from Tq = 4 or so the CUDA-core
+// form runs out of arithmetic before HBM runs out of bandwidth (~16 flops per cache byte at
+// Tq = 16, above the fp32 rate per byte the B200 can stream).  Here the chunk's scores
+// S = Q K^T and its weighted sum P V are two chains of tcgen05 MMAs with M = 128: the Tq
+// query rows are rows 0 .. Tq-1 of a 128-row bf16 tile in shared memory (the other rows
+// are zero and their results are never read), so every new token is one TMEM lane, read by
+// one thread of warp 0.  Warp 0 issues the MMAs (lane 0), computes the chunk maximum, the
+// weights 2^(s - max) and their sums in its lanes (row max and sums in-thread), writes the
+// weights back over S as packed bf16 (the A operand of P V) and finally reads its row of O.
+// The partial output is scaled by (sum of the fp32 weights) / (sum of the bf16-rounded
+// weights the MMA multiplied), so that the merge, which weighs chunks by the fp32 sums,
+// normalises each chunk by the weights actually used, as the training forward does.
+//
+// The query operand holds only its first 16 rows: its swizzle chunks are 16 rows apart
+// (QCH bytes), so the MMA's rows 16 .. 127 of a chunk read the next chunk or the K tile
+// behind it -- finite bf16 values whose score rows no thread reads.  O takes 64 TMEM columns
+// (over S's columns 64 .. 127, read by then): at d = 128 P V runs as two N = 64 halves, each
+// read out before the next.  So a CTA needs 128 TMEM columns and, at d = 128, 69 KB of shared
+// memory: three CTAs share an SM and overlap one another's loads and chains.
+template <int D>
+struct DecTcLayout {
+  static constexpr int QROWS = 16;                      // >= kDecMaxTq
+  static constexpr int QCH = QROWS * Tile<D>::SW;       // one swizzle chunk of the query rows
+  static constexpr int Q_OFF = 0;                       // bf16 [16][D], rows >= Tq zero
+  static constexpr int K_OFF = Tile<D>::CHUNKS * QCH;   // 1024-byte multiple
+  static constexpr int V_OFF = K_OFF + Tile<D>::BYTES;
+  static constexpr int BAR_OFF = V_OFF + Tile<D>::BYTES;  // K landed, V landed, S done, PV done
+  static constexpr int MISC_OFF = BAR_OFF + 32;           // TMEM base slot, abort flag
+  static constexpr int BYTES = MISC_OFF + 16;
+  // below d = 128 the dynamic shared memory is padded so that at most four CTAs share an SM:
+  // four TMEM allocations of 128 columns fill its 512
+  static constexpr int SMEM = (D == 128) ? BYTES + 1024 : (BYTES + 1024 > 56 * 1024 ? BYTES + 1024 : 56 * 1024);
+  static constexpr int THREADS = 128;
+  static constexpr int OH = (D == 128) ? 2 : 1;         // P V passes (64 columns of d each)
+  static constexpr int ON = D / OH;                     // their N
+  static constexpr uint32_t T_S = 0, T_O = 64u;
+  static constexpr uint32_t TMEM_COLS = 128u;
+  static_assert(QROWS * Tile<D>::CHUNKS * Tile<D>::SW + (kRows - QROWS) * Tile<D>::SW <=
+                    K_OFF + Tile<D>::BYTES, "query operand reads stay inside the K tile");
+};
+
+// Byte offset of element (r, col), r < 16, of the compact query operand.
+template <int D>
+__device__ __forceinline__ uint32_t qtile_elem_offset(int r, int col) {
+  using Tl = Tile<D>;
+  const int ch = col / Tl::BOX_COLS, cu = (col % Tl::BOX_COLS) / 8;
+  const int phys = (Tl::SW == 128) ? (cu ^ (r & 7)) : (cu ^ ((r >> 1) & 3));
+  return (uint32_t)(ch * DecTcLayout<D>::QCH + r * Tl::SW + phys * 16 + (col % 8) * 2);
+}
+
+// K-major descriptor of the compact query operand for MMA-K step kk.
+template <int D>
+__device__ __forceinline__ uint64_t qdesc_k(uint32_t tile, int kk) {
+  using Tl = Tile<D>;
+  const uint32_t byte = (uint32_t)kk * 32u;
+  const uint32_t addr = tile + (byte / Tl::SW) * DecTcLayout<D>::QCH + (byte % Tl::SW);
+  return sdesc(addr, 16u, 8u * Tl::SW, Tl::LAYOUT);
+}
+
+template <int D>
+__global__ void __launch_bounds__(128)
+    attn_decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                                const __grid_constant__ CUtensorMap tmV, const DecParams p) {
+  using Tl = Tile<D>;
+  using L = DecTcLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* gsm;
+  const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
+  if (sbase - smem_u32(smem_raw) + L::BYTES > dynamic_smem_bytes()) {
+    if (threadIdx.x == 0) report_smem_shortfall();
+    return;
+  }
+  const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF, sQ = sbase + L::Q_OFF;
+  const uint32_t bar_k = sbase + L::BAR_OFF, bar_v = bar_k + 8u, bar_s = bar_k + 16u,
+                 bar_o = bar_k + 24u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gsm + L::MISC_OFF + 4);
+
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Tq = p.Tq;
+  if (tid == 0) {
+    mbar_init(bar_k, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    // this chunk's 128 key and value rows of head h (rows past L read as zero)
+    mbar_arrive_expect_tx(bar_k, Tl::BYTES);
+    mbar_arrive_expect_tx(bar_v, Tl::BYTES);
+#pragma unroll
+    for (int ch = 0; ch < Tl::CHUNKS; ++ch)
+      tma_load_4d(sK + ch * Tl::CHUNK_BYTES, &tmK, ch * Tl::BOX_COLS, h, c * kDecChunk, b, bar_k);
+#pragma unroll
+    for (int ch = 0; ch < Tl::CHUNKS; ++ch)
+      tma_load_4d(sV + ch * Tl::CHUNK_BYTES, &tmV, ch * Tl::BOX_COLS, h, c * kDecChunk, b, bar_v);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  // the query rows: row t < Tq is new token t's query (bf16, as given), the rest zero
+  for (int i = tid; i < L::QROWS * (D / 8); i += L::THREADS) {
+    const int r = i / (D / 8), u = i % (D / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < Tq)
+      v = *reinterpret_cast<const uint4*>(p.q + (((size_t)b * Tq + r) * p.H + h) * D + 8 * u);
+    *reinterpret_cast<uint4*>(gsm + L::Q_OFF + qtile_elem_offset<D>(r, 8 * u)) = v;
+  }
+  fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Guard g{abort_flag, p.wait_limit_ns};
+
+  if (warp == 0) {
+    const uint32_t tS = tmem + L::T_S, tO = tmem + L::T_O;
+    bool issued_s = false;
+    bool ok = true;
+    if (lane == 0) {
+      ok = wait_bounded(bar_k, 0, g, 1);
+      if (ok) {
+        tc_fence_after();
+        constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tS, qdesc_k<D>(sQ, kk), desc_k<D>(sK, kk), kIdS, kk > 0);
+        tc_commit(bar_s);
+        issued_s = true;
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0) && wait_bounded_warp(bar_s, 0, g, 2);
+    float m = -INFINITY, l = 0.f, lr = 0.f;
+    if (ok) {
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32u * q4, sr[q4]);
+      tc_wait_ld();
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) reg_fence(sr[q4]);
+      // my token (lane) sees the chunk's keys e <= vis
+      const int vis = p.L - Tq + lane - c * kDecChunk;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < kDecChunk; ++e) {
+        if (e > vis) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf
+        mx = fmaxf(mx, __uint_as_float(sr[e >> 5][e & 31]));
+      }
+      m = mx * p.scale_log2;
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      const uint64_t sl2x2 = f2(p.scale_log2, p.scale_log2), nmu2 = f2(-mu, -mu);
+      uint64_t acc_l = f2(0.f, 0.f), acc_lr = f2(0.f, 0.f);
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 xx = f2split(ffma2(f2u(sr[q4][2 * e], sr[q4][2 * e + 1]), sl2x2, nmu2));
+          const float w0 = ex2(xx.x), w1 = ex2(xx.y);
+          const uint32_t v = pack_bf16(w0, w1);
+          acc_l = fadd2(acc_l, f2(w0, w1));
+          acc_lr = fadd2(acc_lr, bf16x2_to_f2(v));
+          pk[e] = v;
+        }
+        tmem_st16(tS + 16u * q4, pk);
+      }
+      const float2 a = f2split(acc_l), ar = f2split(acc_lr);
+      l = a.x + a.y;
+      lr = ar.x + ar.y;
+      tc_wait_st();
+      tc_fence_before();
+    }
+    __syncwarp();
+    // P V in OH passes of ON columns of d; each pass's O is read out before the next
+    // overwrites it
+    int n_o = 0;  // passes issued
+    const float fix = lr > 0.f ? l / lr : 0.f;  // fp32 over bf16-rounded weight sum (0: no key)
+    const bool mine = lane < Tq;
+    const size_t row = (((size_t)b * p.H + h) * Tq + (mine ? lane : 0)) * p.n_chunks + c;
+#pragma unroll
+    for (int hf = 0; hf < L::OH; ++hf) {
+      if (lane == 0 && ok) {
+        if (hf == 0) ok = wait_bounded(bar_v, 0, g, 3);
+        if (ok) {
+          tc_fence_after();
+          constexpr uint32_t kIdO = idesc_bf16_f32(128, L::ON, true);
+#pragma unroll
+          for (int kk = 0; kk < kDecChunk / 16; ++kk)
+            mma_ts(tO, tS + 8u * kk, desc_mn<D>(sV + hf * Tl::CHUNK_BYTES, kk), kIdO, kk > 0);
+          tc_commit(bar_o);
+          ++n_o;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0) && wait_bounded_warp(bar_o, hf & 1, g, 4);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int w2 = 0; w2 < L::ON / 32; ++w2) {
+        uint32_t r[32];
+        tmem_ld32(tO + 32u * w2, r);
+        tc_wait_ld();
+        reg_fence(r);
+        if (mine) {
+          float* dst = p.part_o + row * D + hf * L::ON + 32 * w2;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + e) =
+                make_float4(__uint_as_float(r[e]) * fix, __uint_as_float(r[e + 1]) * fix,
+                            __uint_as_float(r[e + 2]) * fix, __uint_as_float(r[e + 3]) * fix);
+        }
+      }
+      tc_fence_before();  // this pass's O is read: the next pass may overwrite it
+      __syncwarp();
+    }
+    if (ok && mine) {
+      p.part_ml[row * 2] = m;
+      p.part_ml[row * 2 + 1] = l;
+    }
+    if (lane == 0) {  // after a failed wait: no copy or MMA of this CTA may still be in flight
+      if (!ok) {
+        drain_wait(bar_k, 0, p.wait_limit_ns);
+        drain_wait(bar_v, 0, p.wait_limit_ns);
+        if (issued_s) drain_wait(bar_s, 0, p.wait_limit_ns);
+        if (n_o > 0) drain_wait(bar_o, (n_o - 1) & 1, p.wait_limit_ns);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
   }
 }
 

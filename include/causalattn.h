@@ -171,7 +171,8 @@ int gpt_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, float desca
  * Limits: 1 <= Tq <= 16, Tq <= L, B and H <= 65535, B*L*H*d < 2^31.  Fails
  * with GPT_ATTN_ERR_BAD_SHAPE for a too-small workspace.  Layout, ownership,
  * asynchrony and error rules as above.  Split over 128-key chunks of the cache
- * and merged in chunk order: the result is deterministic.
+ * (one new token: CUDA cores; two or more: tensor cores) and merged in chunk
+ * order: the result is deterministic.
  */
 size_t gpt_attn_decode_workspace_size(int B, int H, int Tq, int L, int d);
 

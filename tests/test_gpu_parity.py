@@ -204,7 +204,8 @@ def decode_inputs(B, H, Tq, L, d, seed):
 @pytest.mark.parametrize("B,H,Tq,L,d", [
     (1, 1, 1, 1, 32), (2, 3, 1, 17, 64), (1, 4, 1, 128, 128), (2, 2, 1, 129, 128),
     (3, 2, 4, 300, 64), (1, 8, 16, 1000, 128), (2, 4, 3, 4096, 128), (1, 2, 16, 16, 32),
-    (4, 16, 1, 2048, 128),
+    (4, 16, 1, 2048, 128), (2, 3, 2, 77, 64), (1, 5, 8, 700, 32), (2, 2, 16, 129, 128),
+    (1, 2, 2, 2, 128), (2, 4, 16, 16, 64),
 ])
 def test_decode_parity(B, H, Tq, L, d, cuda_device):
     """gpt_attn_decode against the fp64 decode oracle: O max-abs <= 1e-2, LSE <= 1e-3."""
