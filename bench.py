@@ -56,10 +56,11 @@ def parse():
     return ap.parse_args()
 
 
-# Per-kernel times come from a phase of their own after the timed region: PROFILE_STEPS steps,
-# per-kernel CUDA events in every EVENT_EVERY-th of them at offset EVENT_EVERY // 2, so that no
-# sampled step follows a synchronize (the host must be ahead of the GPU for the gaps between
-# events to be kernel time) and the events' own cost stays out of the headline.
+# Per-kernel times come from the timed region itself: every EVENT_EVERY-th step at offset
+# EVENT_EVERY // 2 carries CUDA events between its launches, so that no sampled step follows a
+# synchronize (the host must be ahead of the GPU for the gaps between events to be kernel time)
+# and the durations see the clocks and power state of the step time they are checked against.
+# Runs too short to sample use PROFILE_STEPS steps of a profile phase of their own after it.
 EVENT_EVERY = 4
 PROFILE_STEPS = 64
 KERNEL_SUM_TOL = 0.03  # the kernel times must add up to the step time within 3 %
@@ -100,6 +101,32 @@ def profile_kernels(step, stream, n_kernels: int, dev):
         for j in range(n_kernels):
             per[j] += ev[j].elapsed_time(ev[j + 1])
     return [x / len(events) for x in per]
+
+
+def timed_steps(step, stream, steps: int, n_kernels: int, dev):
+    """The timed region: `steps` steps between two CUDA events on `stream`.  Every
+    EVENT_EVERY-th step at offset EVENT_EVERY // 2 (never the first, so the host is already
+    ahead of the GPU) also carries CUDA events between its n_kernels launches: the per-kernel
+    durations come from the same region, clocks and power state as the step time.
+    Returns (elapsed ms, average ms per launch j); with too few steps to sample, the
+    per-kernel durations come from a profile phase of their own right after."""
+    import torch
+    idx = set(sampled_indices(steps))
+    events = {i: [torch.cuda.Event(enable_timing=True) for _ in range(n_kernels + 1)] for i in idx}
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        step(events.get(i))
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    elapsed = start.elapsed_time(end)
+    if not events:
+        return elapsed, profile_kernels(step, stream, n_kernels, dev)
+    per = [0.0] * n_kernels
+    for ev in events.values():
+        for j in range(n_kernels):
+            per[j] += ev[j].elapsed_time(ev[j + 1])
+    return elapsed, [x / len(events) for x in per]
 
 
 def host_us_per_call(step, calls_per_step: int, dev, steps: int = 32) -> float:
@@ -542,16 +569,10 @@ def main_prologue(args):
     sampler = ClockSampler(local)
     time.sleep(0.5)
     t_wall0 = time.time()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize(dev)
+    elapsed_local, (fwd_ms, bwd_ms) = timed_steps(step, stream, args.steps, 2, dev)
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
-    ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
-    fwd_ms, bwd_ms = profile_kernels(step, stream, 2, dev)
+    ms = max_over_ranks(elapsed_local / args.steps, dev)
     sum_ratio, sum_warning = kernel_sum_check([fwd_ms, bwd_ms], ms)
     status = abi.gpt_attn_device_status(clear=True)
     # end to end: Q, K, dQ', dK' in from pinned host memory, Q', K', dQ, dK back out
@@ -708,16 +729,10 @@ def main_fp8(args):
     sampler = ClockSampler(local)
     time.sleep(0.5)
     t_wall0 = time.time()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize(dev)
+    elapsed_local, (kernel_ms,) = timed_steps(step, stream, args.steps, 1, dev)
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
-    ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
-    (kernel_ms,) = profile_kernels(step, stream, 1, dev)
+    ms = max_over_ranks(elapsed_local / args.steps, dev)
     host_us = host_us_per_call(step, 1, dev)
     status = abi.gpt_attn_device_status(clear=True)
     # end to end: e4m3 Q, K, V in from pinned host memory, O and LSE back out, every step
@@ -860,21 +875,15 @@ def main():
 
     sampler = ClockSampler(local)
     time.sleep(0.5)  # let the sampler start before the timed region
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    start.record(stream)
-    for _ in range(args.steps):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize(dev)
+    elapsed_local, per_kernel_ms = timed_steps(step, stream, args.steps, len(kernels), dev)
     barrier()
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
-    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
-    # per-kernel durations and host cost per call, outside the timed region
-    per_kernel_ms = profile_kernels(step, stream, len(kernels), dev)
+    elapsed_ms = max_over_ranks(elapsed_local, dev)
+    # host cost per call, outside the timed region
     host_us = host_us_per_call(step, len(kernels), dev)
     host_us_checked = host_us_per_call(step_plain, len(kernels), dev)
     status = abi.gpt_attn_device_status(clear=True)
