@@ -408,6 +408,7 @@ def main_decode(args):
     if world > 1:
         dist.barrier()
     sampler = ClockSampler(local)
+    time.sleep(0.5)  # let the sampler start: a short timed region may otherwise see no sample
     t_wall0 = time.time()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)

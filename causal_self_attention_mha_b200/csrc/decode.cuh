@@ -254,27 +254,27 @@ __global__ void __launch_bounds__(dec_threads<TQM>())
 // key row (2d bytes of K and of V) feeds 4 d Tq flops, so from Tq = 4 or so the CUDA-core
 // form runs out of arithmetic before HBM runs out of bandwidth (~16 flops per cache byte at
 // Tq = 16, above the fp32 rate per byte the B200 can stream).  Here the chunk's scores
-// S = Q K^T and its weighted sum P V are two chains of tcgen05 MMAs with M = 128: the Tq
-// query rows are rows 0 .. Tq-1 of a 128-row bf16 tile in shared memory (the other rows
-// are zero and their results are never read), so every new token is one TMEM lane, read by
-// one thread of warp 0.  Warp 0 issues the MMAs (lane 0), computes the chunk maximum, the
-// weights 2^(s - max) and their sums in its lanes (row max and sums in-thread), writes the
-// weights back over S as packed bf16 (the A operand of P V) and finally reads its row of O.
-// The partial output is scaled by (sum of the fp32 weights) / (sum of the bf16-rounded
-// weights the MMA multiplied), so that the merge, which weighs chunks by the fp32 sums,
-// normalises each chunk by the weights actually used, as the training forward does.
-//
-// The query operand holds only its first 16 rows: its swizzle chunks are 16 rows apart
-// (QCH bytes), so the MMA's rows 16 .. 127 of a chunk read the next chunk or the K tile
-// behind it -- finite bf16 values whose score rows no thread reads.  O takes 64 TMEM columns
-// (over S's columns 64 .. 127, read by then): at d = 128 P V runs as two N = 64 halves, each
-// read out before the next.  So a CTA needs 128 TMEM columns and, at d = 128, 69 KB of shared
-// memory: three CTAs share an SM and overlap one another's loads and chains.
+// S = Q K^T and its weighted sum P V are two chains of tcgen05 MMAs with M = 128 whose rows
+// 0 .. 15 are the new tokens (rows past Tq are zero queries; rows 16 .. 127 of an operand
+// are whatever lies behind its 16 or 32 rows in shared memory, and their results are never
+// read).  Warp 0 does the rest: lane 0 issues the MMAs; the query rows are stored twice
+// (rows 16 .. 31 repeat rows 0 .. 15), so token t's scores are in TMEM lanes t and t + 16,
+// and lane t takes keys 0 .. 63, lane t + 16 keys 64 .. 127 (row maximum and sums combined
+// with one shuffle).  Each lane writes its 64 weights, packed bf16, into row t of the P
+// operand in shared memory (over the query tile and the K tile, both read by then), so P V
+// is a single shared-memory MMA chain with N = d, accumulating over S's TMEM columns.  The
+// partial output is scaled by (sum of the fp32 weights) / (sum of the bf16-rounded weights
+// the MMA multiplied), so that the merge, which weighs chunks by the fp32 sums, normalises
+// each chunk by the weights actually used, as the training forward does.  A CTA needs 128
+// TMEM columns and, at d = 128, 73 KB of shared memory: three CTAs share an SM and overlap
+// one another's loads and chains.
 template <int D>
 struct DecTcLayout {
-  static constexpr int QROWS = 16;                      // >= kDecMaxTq
+  static constexpr int QROWS = 32;                      // tokens 0 .. 15, twice
   static constexpr int QCH = QROWS * Tile<D>::SW;       // one swizzle chunk of the query rows
-  static constexpr int Q_OFF = 0;                       // bf16 [16][D], rows >= Tq zero
+  static constexpr int PCH = 16 * 128;                  // one 64-key chunk of the P rows
+  static constexpr int Q_OFF = 0;                       // bf16 [32][D], rows of tokens >= Tq zero
+  static constexpr int P_OFF = 0;                       // bf16 [16][128 keys], after S is done
   static constexpr int K_OFF = Tile<D>::CHUNKS * QCH;   // 1024-byte multiple
   static constexpr int V_OFF = K_OFF + Tile<D>::BYTES;
   static constexpr int BAR_OFF = V_OFF + Tile<D>::BYTES;  // K landed, V landed, S done, PV done
@@ -284,15 +284,14 @@ struct DecTcLayout {
   // four TMEM allocations of 128 columns fill its 512
   static constexpr int SMEM = (D == 128) ? BYTES + 1024 : (BYTES + 1024 > 56 * 1024 ? BYTES + 1024 : 56 * 1024);
   static constexpr int THREADS = 128;
-  static constexpr int OH = (D == 128) ? 2 : 1;         // P V passes (64 columns of d each)
-  static constexpr int ON = D / OH;                     // their N
-  static constexpr uint32_t T_S = 0, T_O = 64u;
-  static constexpr uint32_t TMEM_COLS = 128u;
-  static_assert(QROWS * Tile<D>::CHUNKS * Tile<D>::SW + (kRows - QROWS) * Tile<D>::SW <=
-                    K_OFF + Tile<D>::BYTES, "query operand reads stay inside the K tile");
+  static constexpr uint32_t TMEM_COLS = 128u;           // S, then O over its first d columns
+  // what the 128-row operands read stays inside this CTA's shared memory, and P stays clear
+  // of V (still needed when P is written)
+  static_assert((Tile<D>::CHUNKS - 1) * QCH + kRows * Tile<D>::SW <= BAR_OFF, "query operand");
+  static_assert(PCH + kRows * 128 <= BAR_OFF && 2 * PCH <= V_OFF, "weight operand");
 };
 
-// Byte offset of element (r, col), r < 16, of the compact query operand.
+// Byte offset of element (r, col), r < 32, of the query operand.
 template <int D>
 __device__ __forceinline__ uint32_t qtile_elem_offset(int r, int col) {
   using Tl = Tile<D>;
@@ -301,13 +300,22 @@ __device__ __forceinline__ uint32_t qtile_elem_offset(int r, int col) {
   return (uint32_t)(ch * DecTcLayout<D>::QCH + r * Tl::SW + phys * 16 + (col % 8) * 2);
 }
 
-// K-major descriptor of the compact query operand for MMA-K step kk.
+// K-major descriptor of the query operand for MMA-K step kk (16 columns of d).
 template <int D>
 __device__ __forceinline__ uint64_t qdesc_k(uint32_t tile, int kk) {
   using Tl = Tile<D>;
   const uint32_t byte = (uint32_t)kk * 32u;
   const uint32_t addr = tile + (byte / Tl::SW) * DecTcLayout<D>::QCH + (byte % Tl::SW);
   return sdesc(addr, 16u, 8u * Tl::SW, Tl::LAYOUT);
+}
+
+// K-major descriptor of the weight operand (keys along K, 64-key chunks of 128-byte rows,
+// 128-byte swizzle) for MMA-K step kk (16 keys).
+template <int D>
+__device__ __forceinline__ uint64_t pdesc_k(uint32_t tile, int kk) {
+  const uint32_t byte = (uint32_t)kk * 32u;
+  const uint32_t addr = tile + (byte / 128u) * DecTcLayout<D>::PCH + (byte % 128u);
+  return sdesc(addr, 16u, 8u * 128u, 2u);
 }
 
 template <int D>
@@ -323,7 +331,8 @@ __global__ void __launch_bounds__(128)
     if (threadIdx.x == 0) report_smem_shortfall();
     return;
   }
-  const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF, sQ = sbase + L::Q_OFF;
+  const uint32_t sK = sbase + L::K_OFF, sV = sbase + L::V_OFF, sQ = sbase + L::Q_OFF,
+                 sP = sbase + L::P_OFF;
   const uint32_t bar_k = sbase + L::BAR_OFF, bar_v = bar_k + 8u, bar_s = bar_k + 16u,
                  bar_o = bar_k + 24u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gsm + L::MISC_OFF);
@@ -353,12 +362,12 @@ __global__ void __launch_bounds__(128)
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
-  // the query rows: row t < Tq is new token t's query (bf16, as given), the rest zero
+  // the query rows: rows t and t + 16 hold new token t's query (bf16, as given), zero past Tq
   for (int i = tid; i < L::QROWS * (D / 8); i += L::THREADS) {
-    const int r = i / (D / 8), u = i % (D / 8);
+    const int r = i / (D / 8), u = i % (D / 8), t = r & 15;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < Tq)
-      v = *reinterpret_cast<const uint4*>(p.q + (((size_t)b * Tq + r) * p.H + h) * D + 8 * u);
+    if (t < Tq)
+      v = *reinterpret_cast<const uint4*>(p.q + (((size_t)b * Tq + t) * p.H + h) * D + 8 * u);
     *reinterpret_cast<uint4*>(gsm + L::Q_OFF + qtile_elem_offset<D>(r, 8 * u)) = v;
   }
   fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
@@ -369,8 +378,7 @@ __global__ void __launch_bounds__(128)
   const Guard g{abort_flag, p.wait_limit_ns};
 
   if (warp == 0) {
-    const uint32_t tS = tmem + L::T_S, tO = tmem + L::T_O;
-    bool issued_s = false;
+    bool issued_s = false, issued_o = false;
     bool ok = true;
     if (lane == 0) {
       ok = wait_bounded(bar_k, 0, g, 1);
@@ -379,105 +387,106 @@ __global__ void __launch_bounds__(128)
         constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tS, qdesc_k<D>(sQ, kk), desc_k<D>(sK, kk), kIdS, kk > 0);
+          mma_ss(tmem, qdesc_k<D>(sQ, kk), desc_k<D>(sK, kk), kIdS, kk > 0);
         tc_commit(bar_s);
         issued_s = true;
       }
     }
     ok = __shfl_sync(0xffffffffu, ok, 0) && wait_bounded_warp(bar_s, 0, g, 2);
+    const int t = lane & 15, hh = lane >> 4;  // my token, my half of the chunk's keys
     float m = -INFINITY, l = 0.f, lr = 0.f;
     if (ok) {
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32u * q4, sr[q4]);
+      for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tmem + 32u * q4, sr[q4]);
       tc_wait_ld();
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) reg_fence(sr[q4]);
-      // my token (lane) sees the chunk's keys e <= vis
-      const int vis = p.L - Tq + lane - c * kDecChunk;
+      // keys e (in my half: 64 hh + e) <= vis are visible to token t
+      const int vis = p.L - Tq + t - c * kDecChunk - 64 * hh;
+      uint32_t s64[64];
       float mx = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < kDecChunk; ++e) {
-        if (e > vis) sr[e >> 5][e & 31] = 0xFF800000u;  // -inf
-        mx = fmaxf(mx, __uint_as_float(sr[e >> 5][e & 31]));
+      for (int e = 0; e < 64; ++e) {
+        const uint32_t v = hh ? sr[2 + (e >> 5)][e & 31] : sr[e >> 5][e & 31];
+        s64[e] = (e > vis) ? 0xFF800000u : v;  // -inf past the token's position
+        mx = fmaxf(mx, __uint_as_float(s64[e]));
       }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       m = mx * p.scale_log2;
       const float mu = (m == -INFINITY) ? 0.f : m;
       const uint64_t sl2x2 = f2(p.scale_log2, p.scale_log2), nmu2 = f2(-mu, -mu);
       uint64_t acc_l = f2(0.f, 0.f), acc_lr = f2(0.f, 0.f);
+      uint32_t pk[32];
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 xx = f2split(ffma2(f2u(sr[q4][2 * e], sr[q4][2 * e + 1]), sl2x2, nmu2));
-          const float w0 = ex2(xx.x), w1 = ex2(xx.y);
-          const uint32_t v = pack_bf16(w0, w1);
-          acc_l = fadd2(acc_l, f2(w0, w1));
-          acc_lr = fadd2(acc_lr, bf16x2_to_f2(v));
-          pk[e] = v;
-        }
-        tmem_st16(tS + 16u * q4, pk);
+      for (int e = 0; e < 32; ++e) {
+        const float2 xx = f2split(ffma2(f2u(s64[2 * e], s64[2 * e + 1]), sl2x2, nmu2));
+        const float w0 = ex2(xx.x), w1 = ex2(xx.y);
+        const uint32_t v = pack_bf16(w0, w1);
+        acc_l = fadd2(acc_l, f2(w0, w1));
+        acc_lr = fadd2(acc_lr, bf16x2_to_f2(v));
+        pk[e] = v;
       }
       const float2 a = f2split(acc_l), ar = f2split(acc_lr);
       l = a.x + a.y;
       lr = ar.x + ar.y;
-      tc_wait_st();
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      lr += __shfl_xor_sync(0xffffffffu, lr, 16);
+      // my 64 weights: row t of the weight operand, 64-key chunk hh (16-byte units swizzled
+      // with the row); S has been read into registers, so the query tile may be overwritten
+      uint8_t* prow = gsm + L::P_OFF + hh * L::PCH + t * 128;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(prow + ((u ^ (t & 7)) * 16)) =
+            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+      fence_proxy_async_smem();
       tc_fence_before();
     }
     __syncwarp();
-    // P V in OH passes of ON columns of d; each pass's O is read out before the next
-    // overwrites it
-    int n_o = 0;  // passes issued
-    const float fix = lr > 0.f ? l / lr : 0.f;  // fp32 over bf16-rounded weight sum (0: no key)
-    const bool mine = lane < Tq;
-    const size_t row = (((size_t)b * p.H + h) * Tq + (mine ? lane : 0)) * p.n_chunks + c;
+    if (lane == 0 && ok) {
+      ok = wait_bounded(bar_v, 0, g, 3);
+      if (ok) {
+        tc_fence_after();
+        constexpr uint32_t kIdO = idesc_bf16_f32(128, D, true);
 #pragma unroll
-    for (int hf = 0; hf < L::OH; ++hf) {
-      if (lane == 0 && ok) {
-        if (hf == 0) ok = wait_bounded(bar_v, 0, g, 3);
-        if (ok) {
-          tc_fence_after();
-          constexpr uint32_t kIdO = idesc_bf16_f32(128, L::ON, true);
-#pragma unroll
-          for (int kk = 0; kk < kDecChunk / 16; ++kk)
-            mma_ts(tO, tS + 8u * kk, desc_mn<D>(sV + hf * Tl::CHUNK_BYTES, kk), kIdO, kk > 0);
-          tc_commit(bar_o);
-          ++n_o;
-        }
+        for (int kk = 0; kk < kDecChunk / 16; ++kk)
+          mma_ss(tmem, pdesc_k<D>(sP, kk), desc_mn<D>(sV, kk), kIdO, kk > 0);
+        tc_commit(bar_o);
+        issued_o = true;
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0) && wait_bounded_warp(bar_o, hf & 1, g, 4);
-      if (!ok) break;
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0) && wait_bounded_warp(bar_o, 0, g, 4);
+    if (ok) {
       tc_fence_after();
+      const float fix = lr > 0.f ? l / lr : 0.f;  // fp32 over rounded weight sum (0: no key)
+      const bool mine = lane < Tq;                // lanes 0 .. Tq-1 hold the tokens' O rows
+      const size_t row = (((size_t)b * p.H + h) * Tq + (mine ? lane : 0)) * p.n_chunks + c;
 #pragma unroll
-      for (int w2 = 0; w2 < L::ON / 32; ++w2) {
+      for (int w2 = 0; w2 < D / 32; ++w2) {
         uint32_t r[32];
-        tmem_ld32(tO + 32u * w2, r);
+        tmem_ld32(tmem + 32u * w2, r);
         tc_wait_ld();
         reg_fence(r);
         if (mine) {
-          float* dst = p.part_o + row * D + hf * L::ON + 32 * w2;
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + e) =
+            *reinterpret_cast<float4*>(p.part_o + row * D + 32 * w2 + e) =
                 make_float4(__uint_as_float(r[e]) * fix, __uint_as_float(r[e + 1]) * fix,
                             __uint_as_float(r[e + 2]) * fix, __uint_as_float(r[e + 3]) * fix);
         }
       }
-      tc_fence_before();  // this pass's O is read: the next pass may overwrite it
-      __syncwarp();
-    }
-    if (ok && mine) {
-      p.part_ml[row * 2] = m;
-      p.part_ml[row * 2 + 1] = l;
+      if (mine) {
+        p.part_ml[row * 2] = m;
+        p.part_ml[row * 2 + 1] = l;
+      }
     }
     if (lane == 0) {  // after a failed wait: no copy or MMA of this CTA may still be in flight
       if (!ok) {
         drain_wait(bar_k, 0, p.wait_limit_ns);
         drain_wait(bar_v, 0, p.wait_limit_ns);
         if (issued_s) drain_wait(bar_s, 0, p.wait_limit_ns);
-        if (n_o > 0) drain_wait(bar_o, (n_o - 1) & 1, p.wait_limit_ns);
+        if (issued_o) drain_wait(bar_o, 0, p.wait_limit_ns);
       }
     }
   }
