@@ -62,6 +62,28 @@ struct DecLayout {
   static constexpr int SMEM = BYTES + 1024;
 };
 
+// An L2 cache policy that marks the lines an access brings in as first to evict: for data
+// read exactly once (a KV cache streamed past), so that it does not push out lines that will
+// be read again soon.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 4-D tiled load with an L2 cache policy (from createpolicy), otherwise as tma_load_4d.
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap* m, int c0,
+                                                 int c1, int c2, int c3, uint32_t bar,
+                                                 uint64_t policy) {
+  if (!tma_coords_ok(c0, c1 | c3)) return;
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar),
+      "l"(policy)
+      : "memory");
+}
+
 // Element (row r, column col) of a staged 128-row tile (the layout load_tile produces).
 template <int D>
 __device__ __forceinline__ uint32_t tile_elem_offset(int r, int col) {
@@ -126,16 +148,17 @@ __global__ void __launch_bounds__(dec_threads<TQM>())
   }
   __syncthreads();
   if (tid == 0) {  // this chunk's 128 key and value rows of head h (rows past L read as zero)
+    const uint64_t pol = l2_policy_evict_first();  // read once: first out of L2
     mbar_arrive_expect_tx(bar_k, Tl::BYTES);
     mbar_arrive_expect_tx(bar_v, Tl::BYTES);
 #pragma unroll
     for (int ch = 0; ch < Tl::CHUNKS; ++ch)
-      tma_load_4d(sbase + L::K_OFF + ch * Tl::CHUNK_BYTES, &tmK, ch * Tl::BOX_COLS, h,
-                  c * kDecChunk, b, bar_k);
+      tma_load_4d_hint(sbase + L::K_OFF + ch * Tl::CHUNK_BYTES, &tmK, ch * Tl::BOX_COLS, h,
+                       c * kDecChunk, b, bar_k, pol);
 #pragma unroll
     for (int ch = 0; ch < Tl::CHUNKS; ++ch)
-      tma_load_4d(sbase + L::V_OFF + ch * Tl::CHUNK_BYTES, &tmV, ch * Tl::BOX_COLS, h,
-                  c * kDecChunk, b, bar_v);
+      tma_load_4d_hint(sbase + L::V_OFF + ch * Tl::CHUNK_BYTES, &tmV, ch * Tl::BOX_COLS, h,
+                       c * kDecChunk, b, bar_v, pol);
   }
   // the new tokens' queries, times scale * log2(e), while the rows arrive (zero past Tq)
   for (int i = tid; i < TQM * D; i += L::NT) {
@@ -348,15 +371,19 @@ __global__ void __launch_bounds__(128)
     mbar_init(bar_o, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    // this chunk's 128 key and value rows of head h (rows past L read as zero)
+    // this chunk's 128 key and value rows of head h (rows past L read as zero), read once:
+    // first out of L2, so that the chunk partials stay there for the merge
+    const uint64_t pol = l2_policy_evict_first();
     mbar_arrive_expect_tx(bar_k, Tl::BYTES);
     mbar_arrive_expect_tx(bar_v, Tl::BYTES);
 #pragma unroll
     for (int ch = 0; ch < Tl::CHUNKS; ++ch)
-      tma_load_4d(sK + ch * Tl::CHUNK_BYTES, &tmK, ch * Tl::BOX_COLS, h, c * kDecChunk, b, bar_k);
+      tma_load_4d_hint(sK + ch * Tl::CHUNK_BYTES, &tmK, ch * Tl::BOX_COLS, h, c * kDecChunk, b,
+                       bar_k, pol);
 #pragma unroll
     for (int ch = 0; ch < Tl::CHUNKS; ++ch)
-      tma_load_4d(sV + ch * Tl::CHUNK_BYTES, &tmV, ch * Tl::BOX_COLS, h, c * kDecChunk, b, bar_v);
+      tma_load_4d_hint(sV + ch * Tl::CHUNK_BYTES, &tmV, ch * Tl::BOX_COLS, h, c * kDecChunk, b,
+                       bar_v, pol);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
