@@ -90,8 +90,8 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(ca::attn_fwd_fp8_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            ca::Fwd8Layout<D>::SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D, 1>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D, 1>::SMEM);
+  e = cudaFuncSetAttribute(ca::attn_decode_chunk_kernel<D>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecLayout<D>::SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(ca::attn_decode_chunk_tc_kernel<D>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, ca::DecTcLayout<D>::SMEM);
@@ -504,8 +504,7 @@ int decode_impl(const void* q, const void* kc, const void* vc, void* o, float* l
     ca::attn_decode_chunk_tc_kernel<D><<<grid, ca::DecTcLayout<D>::THREADS, ca::DecTcLayout<D>::SMEM,
                                          st>>>(mk, mv, p);
   else
-    ca::attn_decode_chunk_kernel<D, 1><<<grid, ca::dec_threads<1>(), ca::DecLayout<D, 1>::SMEM, st>>>(
-        mk, mv, p);
+    ca::attn_decode_chunk_kernel<D><<<grid, ca::kDecThreads, ca::DecLayout<D>::SMEM, st>>>(mk, mv, p);
   }
   int s = launch_status();
   if (s) return s;

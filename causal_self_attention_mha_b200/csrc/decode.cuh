@@ -27,13 +27,7 @@
 namespace ca {
 
 constexpr int kDecChunk = 128;   // keys per CTA (one TMA box of rows)
-constexpr int kDecThreads = 128;
-// Threads of a CUDA-core chunk CTA holding up to TQM tokens: one token, a thread per key row;
-// several, two threads per key row (each taking half of the tokens in the score pass).  The
-// library instantiates it for one token (several go to the tensor-core kernel, which is
-// 1.3-3x faster from two tokens on).
-template <int TQM>
-constexpr int dec_threads() { return TQM > 1 ? 2 * kDecThreads : kDecThreads; }
+constexpr int kDecThreads = 128; // CUDA-core chunk kernel: a thread per key row
 constexpr int kDecMaxTq = 16;    // new tokens per call
 constexpr int kDecTcMinTq = 2;   // from this many new tokens on, the tensor-core chunk kernel
 
@@ -46,17 +40,17 @@ struct DecParams {
   uint64_t wait_limit_ns;
 };
 
-template <int D, int TQM>
+// Shared memory of the CUDA-core chunk kernel (one new token).
+template <int D>
 struct DecLayout {
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = Tile<D>::BYTES;
-  static constexpr int Q_OFF = 2 * Tile<D>::BYTES;                 // fp32 [TQM][D], times scale*log2e
-  static constexpr int P_OFF = Q_OFF + TQM * D * 4;                // fp32 [TQM][128] weights
-  static constexpr int NT = dec_threads<TQM>();
-  static constexpr int RED_OFF = P_OFF + TQM * kDecChunk * 4;      // fp32 [2][TQM][4] warp partials
-  static constexpr int G = NT / D;                                 // key groups in the V pass
-  static constexpr int ACC_OFF = RED_OFF + 2 * TQM * 4 * 4;        // fp32 [G][TQM][D] group sums
-  static constexpr int BAR_OFF = ACC_OFF + (G > 1 ? G * TQM * D * 4 : 0);  // K landed, V landed
+  static constexpr int Q_OFF = 2 * Tile<D>::BYTES;                 // fp32 [D], times scale*log2e
+  static constexpr int P_OFF = Q_OFF + D * 4;                      // fp32 [128] weights
+  static constexpr int RED_OFF = P_OFF + kDecChunk * 4;            // fp32 [2][4] warp partials
+  static constexpr int G = kDecThreads / D;                        // key groups in the V pass
+  static constexpr int ACC_OFF = RED_OFF + 2 * 4 * 4;              // fp32 [G][D] group sums
+  static constexpr int BAR_OFF = ACC_OFF + (G > 1 ? G * D * 4 : 0);  // K landed, V landed
   static constexpr int MISC_OFF = BAR_OFF + 16;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int SMEM = BYTES + 1024;
@@ -93,38 +87,28 @@ __device__ __forceinline__ uint32_t tile_elem_offset(int r, int col) {
   return (uint32_t)(ch * Tl::CHUNK_BYTES + r * Tl::SW + phys * 16 + (col % 8) * 2);
 }
 
-// Max or sum of v[t] (t < TQM) over the 4 warps of this thread's group of 128 threads (the
-// group's own slice of `red`); every thread of the group gets the results.
-template <int TQM>
-__device__ __forceinline__ void dec_block_reduce(float (&v)[TQM], bool is_max, float* red) {
+// Max or sum of v over the CTA's 4 warps (through `red`, 4 floats); every thread gets it.
+__device__ __forceinline__ float dec_block_reduce(float v, bool is_max, float* red) {
 #pragma unroll
-  for (int t = 0; t < TQM; ++t)
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float o = __shfl_xor_sync(0xffffffffu, v[t], off);
-      v[t] = is_max ? fmaxf(v[t], o) : v[t] + o;
-    }
-  const int warp = (threadIdx.x >> 5) & 3;
-  if ((threadIdx.x & 31) == 0) {
-#pragma unroll
-    for (int t = 0; t < TQM; ++t) red[t * 4 + warp] = v[t];
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = is_max ? fmaxf(v, o) : v + o;
   }
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
   __syncthreads();
-#pragma unroll
-  for (int t = 0; t < TQM; ++t) {
-    const float4 r = *reinterpret_cast<const float4*>(red + t * 4);
-    v[t] = is_max ? fmaxf(fmaxf(r.x, r.y), fmaxf(r.z, r.w)) : (r.x + r.y) + (r.z + r.w);
-  }
+  const float4 r = *reinterpret_cast<const float4*>(red);
+  return is_max ? fmaxf(fmaxf(r.x, r.y), fmaxf(r.z, r.w)) : (r.x + r.y) + (r.z + r.w);
 }
 
-// One CTA: one 128-key chunk of one (batch, head), every new token at once: each key row
-// and each V element is read from shared memory once for all Tq tokens.
-template <int D, int TQM>
-__global__ void __launch_bounds__(dec_threads<TQM>())
+// One new token, on CUDA cores.  One CTA: one 128-key chunk of one (batch, head); thread kr
+// scores key row kr, then a thread per output column (in G groups of keys for d < 128)
+// sums weights times V.
+template <int D>
+__global__ void __launch_bounds__(kDecThreads)
     attn_decode_chunk_kernel(const __grid_constant__ CUtensorMap tmK,
                              const __grid_constant__ CUtensorMap tmV, const DecParams p) {
   using Tl = Tile<D>;
-  using L = DecLayout<D, TQM>;
+  using L = DecLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* gsm;
   const uint32_t sbase = aligned_smem_base(smem_raw, &gsm);
@@ -139,7 +123,6 @@ __global__ void __launch_bounds__(dec_threads<TQM>())
 
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
-  const int Tq = p.Tq;
   if (tid == 0) {
     mbar_init(bar_k, 1);
     mbar_init(bar_v, 1);
@@ -160,12 +143,9 @@ __global__ void __launch_bounds__(dec_threads<TQM>())
       tma_load_4d_hint(sbase + L::V_OFF + ch * Tl::CHUNK_BYTES, &tmV, ch * Tl::BOX_COLS, h,
                        c * kDecChunk, b, bar_v, pol);
   }
-  // the new tokens' queries, times scale * log2(e), while the rows arrive (zero past Tq)
-  for (int i = tid; i < TQM * D; i += L::NT) {
-    const int t = i / D, col = i % D;
-    qs[i] = t < Tq ? __bfloat162float(p.q[(((size_t)b * Tq + t) * p.H + h) * D + col]) * p.scale_log2
-                   : 0.f;
-  }
+  // the query, times scale * log2(e), while the rows arrive (q is [B, 1, H, D])
+  for (int i = tid; i < D; i += kDecThreads)
+    qs[i] = __bfloat162float(p.q[((size_t)b * p.H + h) * D + i]) * p.scale_log2;
   const Guard g{abort_flag, p.wait_limit_ns};
   // the scores need only K: V keeps landing while they are computed
   const bool ok = wait_bounded(bar_k, 0, g, 1);
@@ -178,51 +158,28 @@ __global__ void __launch_bounds__(dec_threads<TQM>())
     return;
   }
 
-  // scores of my key row against my half of the new tokens (base 2; -inf where not visible)
-  constexpr int TH = TQM / (L::NT / kDecChunk);  // tokens per score thread
-  const int kr = tid % kDecChunk, th = tid / kDecChunk;
-  const int j = c * kDecChunk + kr;
-  float s[TH];
-#pragma unroll
-  for (int i = 0; i < TH; ++i) s[i] = 0.f;
+  // the score of my key row (base 2; -inf past the cache: the token sees keys 0 .. L - 1)
+  const int kr = tid, j = c * kDecChunk + kr;
+  float s = 0.f;
 #pragma unroll
   for (int u = 0; u < D / 8; ++u) {
     const uint4 kv = *reinterpret_cast<const uint4*>(sK + tile_elem_offset<D>(kr, 8 * u));
-    const float k8[8] = {bf16_lo(kv.x), bf16_hi(kv.x), bf16_lo(kv.y), bf16_hi(kv.y),
-                         bf16_lo(kv.z), bf16_hi(kv.z), bf16_lo(kv.w), bf16_hi(kv.w)};
-#pragma unroll
-    for (int i = 0; i < TH; ++i) {
-      const int t = th * TH + i;
-      const float4 q0 = *reinterpret_cast<const float4*>(qs + t * D + 8 * u);
-      const float4 q1 = *reinterpret_cast<const float4*>(qs + t * D + 8 * u + 4);
-      float a = s[i];
-      a = fmaf(k8[0], q0.x, a);
-      a = fmaf(k8[1], q0.y, a);
-      a = fmaf(k8[2], q0.z, a);
-      a = fmaf(k8[3], q0.w, a);
-      a = fmaf(k8[4], q1.x, a);
-      a = fmaf(k8[5], q1.y, a);
-      a = fmaf(k8[6], q1.z, a);
-      a = fmaf(k8[7], q1.w, a);
-      s[i] = a;
-    }
+    const float4 q0 = *reinterpret_cast<const float4*>(qs + 8 * u);
+    const float4 q1 = *reinterpret_cast<const float4*>(qs + 8 * u + 4);
+    s = fmaf(bf16_lo(kv.x), q0.x, s);
+    s = fmaf(bf16_hi(kv.x), q0.y, s);
+    s = fmaf(bf16_lo(kv.y), q0.z, s);
+    s = fmaf(bf16_hi(kv.y), q0.w, s);
+    s = fmaf(bf16_lo(kv.z), q1.x, s);
+    s = fmaf(bf16_hi(kv.z), q1.y, s);
+    s = fmaf(bf16_lo(kv.w), q1.z, s);
+    s = fmaf(bf16_hi(kv.w), q1.w, s);
   }
-#pragma unroll
-  for (int i = 0; i < TH; ++i) {  // query t sees keys 0 .. L - Tq + t
-    const int t = th * TH + i;
-    if (t >= Tq || j > p.L - Tq + t) s[i] = -INFINITY;
-  }
-  float m[TH], w[TH];
-#pragma unroll
-  for (int i = 0; i < TH; ++i) m[i] = s[i];
-  dec_block_reduce<TH>(m, true, red + th * TH * 4);
-#pragma unroll
-  for (int i = 0; i < TH; ++i) {
-    w[i] = (s[i] == -INFINITY) ? 0.f : ex2(s[i] - m[i]);
-    ps[(th * TH + i) * kDecChunk + kr] = w[i];
-  }
-  // w[i] now holds the chunk's sum for token th * TH + i
-  dec_block_reduce<TH>(w, false, red + TQM * 4 + th * TH * 4);
+  if (j > p.L - 1) s = -INFINITY;
+  const float m = dec_block_reduce(s, true, red);
+  const float w = (s == -INFINITY) ? 0.f : ex2(s - m);
+  ps[kr] = w;
+  const float lsum = dec_block_reduce(w, false, red + 4);  // the chunk's sum of weights
   // V must have landed before the weighted sums (ps is complete after the reduction's barrier)
   {
     const bool vok = wait_bounded(bar_v, 0, g, 2);
@@ -232,44 +189,26 @@ __global__ void __launch_bounds__(dec_threads<TQM>())
       return;
     }
   }
-  // my column of V over my group's keys, for every token
+  // my column of V over my group's keys
   const int col = tid % D, grp = tid / D;
   constexpr int KPG = kDecChunk / L::G;
-  float acc[TQM];
-#pragma unroll
-  for (int t = 0; t < TQM; ++t) acc[t] = 0.f;
+  float acc = 0.f;
 #pragma unroll 4
   for (int k = grp * KPG; k < (grp + 1) * KPG; ++k) {
     const uint16_t bits = *reinterpret_cast<const uint16_t*>(sV + tile_elem_offset<D>(k, col));
-    const float v = __uint_as_float((uint32_t)bits << 16);
-#pragma unroll
-    for (int t = 0; t < TQM; ++t) acc[t] = fmaf(ps[t * kDecChunk + k], v, acc[t]);
+    acc = fmaf(ps[k], __uint_as_float((uint32_t)bits << 16), acc);
   }
   if (L::G > 1) {
-#pragma unroll
-    for (int t = 0; t < TQM; ++t) acc_s[(grp * TQM + t) * D + col] = acc[t];
+    acc_s[grp * D + col] = acc;
     __syncthreads();
-    if (grp == 0) {
-      for (int gg = 1; gg < L::G; ++gg)
-#pragma unroll
-        for (int t = 0; t < TQM; ++t) acc[t] += acc_s[(gg * TQM + t) * D + col];
-    }
+    if (grp == 0)
+      for (int gg = 1; gg < L::G; ++gg) acc += acc_s[gg * D + col];
   }
-#pragma unroll
-  for (int t = 0; t < TQM; ++t) {
-    if (t >= Tq) break;
-    const size_t row = (((size_t)b * p.H + h) * Tq + t) * p.n_chunks + c;
-    if (grp == 0) p.part_o[row * D + col] = acc[t];
-  }
-  if (kr == 0) {  // the chunk maximum and sum of this half's tokens
-#pragma unroll
-    for (int i = 0; i < TH; ++i) {
-      const int t = th * TH + i;
-      if (t >= Tq) break;
-      const size_t row = (((size_t)b * p.H + h) * Tq + t) * p.n_chunks + c;
-      p.part_ml[row * 2] = m[i];
-      p.part_ml[row * 2 + 1] = w[i];
-    }
+  const size_t row = (((size_t)b * p.H + h) * p.Tq) * p.n_chunks + c;  // Tq = 1
+  if (grp == 0) p.part_o[row * D + col] = acc;
+  if (tid == 0) {  // the chunk maximum and sum
+    p.part_ml[row * 2] = m;
+    p.part_ml[row * 2 + 1] = lsum;
   }
 }
 
