@@ -217,9 +217,10 @@ __global__ void __launch_bounds__(kDecThreads)
 // form runs out of arithmetic before HBM runs out of bandwidth (~16 flops per cache byte at
 // Tq = 16, above the fp32 rate per byte the B200 can stream).  Here the chunk's scores
 // S = Q K^T and its weighted sum P V are two chains of tcgen05 MMAs with M = 128 whose rows
-// 0 .. 15 are the new tokens (rows past Tq are zero queries; rows 16 .. 127 of an operand
-// are whatever lies behind its 16 or 32 rows in shared memory, and their results are never
-// read).  Warp 0 does the rest: lane 0 issues the MMAs; the query rows are stored twice
+// 0 .. 15 are the new tokens (rows past Tq are zero queries; the A-operand rows past the 32
+// stored query rows or the 16 stored weight rows are whatever lies behind them in shared
+// memory, and their results are never read).  Warp 0 does the rest: lane 0 issues the
+// MMAs; the query rows are stored twice
 // (rows 16 .. 31 repeat rows 0 .. 15), so token t's scores are in TMEM lanes t and t + 16,
 // and lane t takes keys 0 .. 63, lane t + 16 keys 64 .. 127 (row maximum and sums combined
 // with one shuffle).  Each lane writes its 64 weights, packed bf16, into row t of the P
